@@ -1,0 +1,357 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-MoE layer stack over a shared LRU expert cache.
+
+Workload (one step = one decode token through every MoE layer): 4 MoE layers,
+128 experts, hidden 2048, SwiGLU intermediate 768, top-8 softmax gating,
+bf16 weights N(0, 0.02); the expert pool in pinned host memory; 204 HBM slots
+(40% of all experts) as one LRU shared by the layers; hidden states from an
+AR(1) process x_t = 0.9 x_{t-1} + 0.436 eps_t (routing locality), batch 1.
+Synthetic data stands in for the agent workloads and replayed traces of the
+FreeToken pages.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Reports (one JSON line, rank 0): decode tokens/s timed on the device with
+CUDA events (max over ranks), an end-to-end figure through host buffers, the
+roofline of the dominant kernel (the gate/up expert GEMV, HBM-bound) from
+live CUDA events, cache miss rate and H2D fill bandwidth, SM clocks sampled
+during the timed region, and the CPU oracle timed on a bounded sample.
+N > 1 runs independent replicas (one stack per GPU, its own token chain):
+the path has no exchange step.
+"""
+import argparse
+import datetime
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+CONFIG_ID = 2
+METRIC = "routed-MoE tokens/s (decode, prefill) and expert-weight HBM GB/s vs peak"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def workload_desc(cfg):
+    return {
+        "workload": "%s: %d MoE layers, E=%d, H=%d, I=%d, top-%d %s, %s weights, %d cache slots "
+                    "(%.0f%% of experts), %s tokens, batch %d, decode" % (
+                        cfg.name, cfg.L, cfg.E, cfg.H, cfg.I, cfg.k, cfg.gating, cfg.wdtype, cfg.C,
+                        100.0 * cfg.C / (cfg.L * cfg.E), "AR(1)" if cfg.process == "ar1" else "N(0,1)",
+                        cfg.batches[0]),
+        "layers": cfg.L, "experts": cfg.E, "hidden": cfg.H, "inter": cfg.I, "top_k": cfg.k,
+        "cache_slots": cfg.C, "batch": cfg.batches[0], "step": "one decode token through all layers",
+        "l2": "not flushed: each step streams ~%d MB of expert weights, above the 126 MB L2"
+              % round(cfg.L * (cfg.k * cfg.blob_bytes + cfg.E * cfg.H * 4) / 1e6),
+    }
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def token_chain(cfg, chain, n):
+    x = synth.ar1_chain(cfg.seed, chain, n, cfg.H)
+    bits = synth.round_bf16(x)
+    return (bits.astype(np.uint32) << 16).view(np.float32), bits
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                p = [v.strip() for v in ln.split(",")]
+                if len(p) >= 7 and p[0].isdigit():
+                    rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [int(r[0]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": int(rows[0][1]), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------ distributed --
+
+def dist_setup(n_gpus):
+    """torchrun environment -> (rank, world, local_rank).  One process per GPU."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if os.environ.get("FT_BENCH_BACKEND", "nccl") == "nccl" else "gloo"
+        if backend == "nccl":
+            import torch
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def aggregate(tokens, seconds, device=None):
+    """Whole-job throughput over replicas: total tokens of all ranks / the slowest
+    rank's time.  Returns (total_tokens, max_seconds)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return tokens, seconds
+    t = torch.tensor([float(tokens)], dtype=torch.float64, device=device)
+    s = torch.tensor([float(seconds)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    dist.all_reduce(s, op=dist.ReduceOp.MAX)
+    return t.item(), s.item()
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and str(device).startswith("cuda"):
+            dist.barrier(device_ids=[int(str(device).split(":")[1])])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------- CPU oracle leg --
+
+def cpu_oracle_rate(cfg, vals, budget_s=20.0, blob_of=None, max_tokens=None):
+    """Decode tokens/s of the CPU oracle on a bounded sample of the same workload:
+    tokens of the chain are pushed through every layer (router, top-k, gates, LRU,
+    expert FFN, combine) until the time budget is spent.  Returns (rate, tokens, cores)."""
+    from oracle import lru as olru
+    from oracle import moe
+    try:
+        import threadpoolctl
+        cores = max([p.get("num_threads", 1) for p in threadpoolctl.threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    cache = {}
+
+    def blob(l, e):
+        if blob_of is not None:
+            return blob_of(l, e)
+        if (l, e) not in cache:
+            cache[(l, e)] = synth.expert_blob(cfg, l, e)
+        return cache[(l, e)]
+
+    routers = [synth.router_weights(cfg, l) for l in range(cfg.L)]
+    c = olru.SharedLru(cfg.C)
+    done = 0
+    t0 = time.perf_counter()
+    for s in range(len(vals)):
+        x = vals[s:s + 1]
+        for l in range(cfg.L):
+            r = moe.route(x, routers[l], cfg.k, cfg.gating)
+            c.access_set(s * cfg.L + l, l, moe.selected_set(r["ids"]))
+            moe.experts_and_combine(x, r["ids"], r["gates"], cfg.E, cfg.wdtype, cfg.H, cfg.I,
+                                    lambda e, l=l: blob(l, e))
+        done += 1
+        if time.perf_counter() - t0 > budget_s or (max_tokens and done >= max_tokens):
+            break
+    dt = time.perf_counter() - t0
+    return done / dt, done, cores, dt
+
+
+# ------------------------------------------------------------ reference arm --
+
+def run_reference(args):
+    rank, world, local = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
+    if rank != 0:
+        return 0
+    cfg = synth.CONFIGS[CONFIG_ID]
+    vals, _ = token_chain(cfg, 0, args.warmup + args.steps)
+    # warm-up steps untimed, then the timed steps, bounded to a few minutes in all
+    cpu_oracle_rate(cfg, vals[:args.warmup], budget_s=30.0, max_tokens=args.warmup)
+    rate, n, cores, dt = cpu_oracle_rate(cfg, vals[args.warmup:], budget_s=args.reference_budget_s,
+                                         max_tokens=args.steps)
+    sample = ("CPU oracle (float64 numpy), %d of the %d timed decode tokens through all %d layers "
+              "(stopped after %.0f s)" % (n, args.steps, cfg.L, args.reference_budget_s))
+    line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": n, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(n, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_desc(cfg),
+            "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- our arm --
+
+def run_ours(args):
+    import torch
+
+    import moe_expert_offload_top_b200 as ft
+    from moe_expert_offload_top_b200.workload import GpuStack
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = synth.CONFIGS[CONFIG_ID]
+    W, K = args.warmup, args.steps
+    vals, bits = token_chain(cfg, rank, W + 2 * K)      # device leg, then e2e leg
+    stack = GpuStack(cfg, device=dev)
+    x_dev = torch.from_numpy(bits).view(torch.bfloat16).to(dev).view(W + 2 * K, 1, cfg.H)
+    out = torch.empty((cfg.L, 1, cfg.H), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for s in range(W):
+        stack.step(x_dev[s], out, stream)
+    torch.cuda.synchronize(dev)
+
+    # ---- device-timed leg: inputs resident in HBM
+    stack.reset_stats()
+    ft.ft_moe_reset_perf(stack.h)
+    ft.ft_moe_set_stage_timing(stack.h, 1)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(W, W + K):
+        stack.step(x_dev[s], out, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    clk = clocks.stop()
+    dt = e0.elapsed_time(e1) * 1e-3
+    perf = ft.ft_moe_perf(stack.h)
+    st = stack.stats()
+    ft.ft_moe_set_stage_timing(stack.h, 0)
+    tokens, t_max = aggregate(K * cfg.batches[0], dt, dev)
+
+    # ---- end-to-end leg through host buffers (pinned): H2D of the step's token and
+    # D2H of the step's layer outputs inside the timed region, read back every step
+    x_host = torch.from_numpy(bits[W + K:W + 2 * K]).view(torch.bfloat16).view(K, 1, cfg.H).pin_memory()
+    out_host = torch.empty((K, cfg.L, 1, cfg.H), dtype=torch.bfloat16).pin_memory()
+    x_in = torch.empty((1, cfg.H), dtype=torch.bfloat16, device=dev)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for s in range(K):
+        x_in.copy_(x_host[s], non_blocking=True)
+        stack.step(x_in, out, stream)
+        out_host[s].copy_(out, non_blocking=True)
+        stream.synchronize()
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_dt = a0.elapsed_time(a1) * 1e-3
+    e2e_tokens, e2e_max = aggregate(K * cfg.batches[0], e2e_dt, dev)
+
+    if rank == 0:
+        peak, peak_src = measured_peaks()
+        gu_launches = max(perf["timed_forwards"], 1)
+        gu_s = perf["ffn_gate_up_ms"] * 1e-3
+        achieved = perf["ffn_gate_up_bytes"] / gu_s / 1e9 if gu_s > 0 else None
+        line = {
+            "metric": METRIC, "value": tokens / t_max, "unit": "tokens/s", "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": 1e3 * t_max / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,0.02) weights, AR(1) hidden states)",
+            "config": dict(workload_desc(cfg), parallelism="replicas x%d" % world),
+            "roofline": {
+                "kernel": "grouped_gemv_kernel (expert gate/up + SwiGLU, decode)",
+                "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak if achieved else None, "peak_source": peak_src,
+                "traffic": None,
+                "bytes_per_launch": perf["ffn_gate_up_bytes"] / gu_launches,
+                "avg_launch_us": 1e6 * gu_s / gu_launches,
+                "down_proj_gbs": perf["ffn_down_bytes"] / (perf["ffn_down_ms"] * 1e-3) / 1e9
+                if perf["ffn_down_ms"] > 0 else None,
+            },
+            "e2e": {"value": e2e_tokens / e2e_max, "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(cfg.H * 2 * cfg.batches[0]),
+                    "d2h_bytes_per_step": int(cfg.L * cfg.H * 2 * cfg.batches[0])},
+            "gpu_launches": int(perf["kernel_launches"]),
+            "clocks": clk,
+            "cache": {"miss_rate": st["misses"] / max(st["routed"], 1), "routed": st["routed"],
+                      "misses": st["misses"], "h2d_bytes": st["h2d_bytes"],
+                      "h2d_gbs": st["h2d_bytes"] / st["h2d_seconds"] / 1e9 if st["h2d_seconds"] > 0 else None},
+            "stages_us_per_forward": {k2: 1e3 * perf[k2 + "_ms"] / gu_launches for k2 in
+                                      ("router", "permute", "ffn_gate_up", "ffn_down", "combine")},
+            "host_wait_us_per_forward": 1e3 * perf["host_wait_ms"] / max(perf["forwards"], 1),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            rate, n, cores, cdt = cpu_oracle_rate(cfg, vals[W:W + K], budget_s=args.cpu_budget_s,
+                                                  blob_of=stack.pool_blob)
+            line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                    "sample": "%d decode tokens of the timed chain through all %d layers "
+                                              "(float64 numpy oracle, %.1f s)" % (n, cfg.L, cdt)}
+        print(json.dumps(line), flush=True)
+    stack.close()
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--reference-budget-s", type=float, default=120.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,305 @@
+/*
+ * ftmoe.h - C ABI of a routed mixture-of-experts layer stack executed against
+ * a shared LRU cache of expert slots in GPU memory (NVIDIA B200, sm_100a).
+ *
+ * The method (FreeToken pages):
+ *  - The router activates a few experts per token, e.g. 6 of 256 routed
+ *    experts ("FreeToken linux", section "FreeToken's MoE memory handling").
+ *  - The full routed-expert pool lives in host memory and stays the reference
+ *    copy.  Spare GPU memory holds expert slots.  One LRU policy, shared by
+ *    every MoE layer, decides which experts the slots hold (same section;
+ *    "FreeToken gguf", MoE backends, `offload`).
+ *  - A missed expert is copied over PCIe into a slot and kept for reuse (same
+ *    sections).  Executing misses on the CPU is not part of this library.
+ *  - Prefill streams the next layer's experts while the current layer runs
+ *    (whole-layer double buffering; "FreeToken linux", same section;
+ *    "FreeToken RTX 5090", prefill and decode).
+ *  - The cache can be resized at a safe point without a restart.  Capacity
+ *    changes speed, never the result ("FreeToken RTX 5090", dynamic
+ *    reconfiguration; "FreeToken linux", elastic cache resize).
+ *
+ * The pages give no API.  The names below follow their problem statement.
+ *
+ * Conventions for every entry point:
+ *  - "device" pointers are CUDA global-memory addresses on the device that was
+ *    current when the handle was created.  "host" pointers are CPU memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *  - Calls returning int return an ft_status.  On error they leave a message
+ *    in ft_last_error(h).
+ *  - The caller owns x, router weights, out and all ft_* argument buffers.
+ *    The library owns the pinned pool, the slot arena, shared-expert memory,
+ *    scratch, its copy stream and its events.
+ *  - A handle is not thread-safe: use one host thread per handle at a time.
+ */
+#ifndef FTMOE_H
+#define FTMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FT_API __attribute__((visibility("default")))
+#else
+#define FT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ft_moe ft_moe; /* opaque; owned by the library */
+
+enum ft_status {
+  FT_OK = 0,
+  FT_ERR_INVALID = 1,      /* bad argument or call order; nothing was changed */
+  FT_ERR_OOM = 2,          /* device or pinned-host allocation failed */
+  FT_ERR_CUDA = 3,         /* a CUDA call failed; cache state of the failed fills is rolled back */
+  FT_ERR_CAPACITY = 4,     /* one step needs more distinct experts than there are slots */
+  FT_ERR_BUSY = 5,         /* resize or destroy requested while a forward is in flight */
+  FT_ERR_TIMEOUT = 6,      /* a host wait on the GPU passed its deadline */
+  FT_ERR_DEVICE_CHECK = 7  /* a kernel's own bounds check failed (the kernel skipped the access) */
+};
+
+enum ft_wdtype { FT_W_F32 = 0, FT_W_BF16 = 1, FT_W_INT4_G128 = 2 };
+enum ft_gating { FT_GATE_SOFTMAX = 0, FT_GATE_SIGMOID = 1 };
+enum ft_access_kind { FT_ROUTED = 0, FT_PREFETCH = 1 };
+
+/* Largest supported number of routed experts per layer. */
+#define FT_MAX_EXPERTS 256
+/* Largest supported top-k. */
+#define FT_MAX_TOPK 16
+
+/* Cache counters since creation (or since the last ft_cache_reset_stats). */
+typedef struct {
+  long long routed;           /* routed accesses: one per distinct expert per layer per forward */
+  long long hits;             /* routed accesses found resident */
+  long long misses;           /* routed accesses filled from the host pool */
+  long long evictions;        /* entries dropped to make room (fills and shrinks) */
+  long long prefetch;         /* prefetch accesses (prefill mode) */
+  long long prefetch_hits;
+  long long prefetch_misses;  /* prefetch accesses that copied an expert */
+  long long h2d_bytes;        /* bytes copied host -> slot */
+  double h2d_seconds;         /* copy-stream time of those copies, from CUDA events */
+  int resident;               /* occupied slots */
+  int capacity;               /* slots */
+} ft_cache_stats_t;
+
+/* One cache access, in the order the cache saw them. */
+typedef struct {
+  int call;       /* forward-call index of the handle, from 0 */
+  int layer;
+  int expert;
+  int kind;       /* ft_access_kind */
+  int hit;        /* 1 = resident already */
+  int slot;       /* slot used */
+  int ev_layer;   /* key evicted to make room, or -1 */
+  int ev_expert;
+} ft_access_t;
+
+/* ------------------------------------------------------------------------ *
+ * Cache-level API
+ * ------------------------------------------------------------------------ */
+
+/* Creates a stack description with `cache_slots` expert slots of one blob each.
+ *   num_experts E (1..FT_MAX_EXPERTS), top_k k (1..min(E, FT_MAX_TOPK)),
+ *   hidden H and inter I (SwiGLU intermediate): multiples of 8.  For
+ *   FT_W_INT4_G128 they must be multiples of 128.  wdtype is an ft_wdtype.
+ * The stack starts with 1 layer, softmax gating and no shared expert.  Call
+ * ft_moe_set_layers before filling the pool.  Allocates the slot arena on the
+ * current device; the pinned pool is allocated by ft_moe_set_layers.
+ * Returns NULL on failure, with the reason in ft_last_error(NULL). */
+FT_API ft_moe* ft_moe_create(int num_experts, int top_k, int hidden, int inter, int wdtype,
+                      int cache_slots);
+
+/* Sets the number of layers L, the gating (ft_gating) and whether each layer has one
+ * always-on shared expert (gate weight 1).  (Re)allocates the pinned host pool of
+ * L*E expert blobs (contents undefined until written) and the resident shared-expert
+ * memory (zeroed).  The cache is emptied.  Not allowed while a forward is in flight. */
+FT_API int ft_moe_set_layers(ft_moe* h, int num_layers, int gating, int has_shared_expert);
+
+/* Bytes of one expert blob (the runtime layout below). */
+FT_API size_t ft_moe_blob_bytes(const ft_moe* h);
+
+/* Host address of routed expert (layer, expert) in the library-owned pinned pool,
+ * or NULL for bad indices.  Blobs are contiguous in (layer, expert) order:
+ * ft_moe_pool_ptr(h, l, e) = ft_moe_pool_ptr(h, 0, 0) + (l*E + e) * ft_moe_blob_bytes(h).  The caller writes the expert's blob there before the
+ * first forward that can read it.  A blob already copied into a slot is not copied
+ * again until evicted.
+ * Runtime blob layout (row-major, K = reduction axis contiguous):
+ *   f32 / bf16: W_gate [I][H], W_up [I][H], W_down [H][I].
+ *   int4 g128:  packed W_gate [I][H/2], W_up [I][H/2], W_down [H][I/2] bytes.  Byte b
+ *               of a row holds element 2b in its low nibble and 2b+1 in its high
+ *               nibble, two's complement in [-8, 7].  Then the bf16 scales
+ *               S_gate [I][H/128], S_up [I][H/128], S_down [H][I/128], one per 128
+ *               consecutive K elements of a row.  w = q * s. */
+FT_API void* ft_moe_pool_ptr(ft_moe* h, int layer, int expert);
+
+/* Copies the shared expert of `layer` (a host blob in the same layout) into resident
+ * device memory.  Synchronous. */
+FT_API int ft_moe_set_shared(ft_moe* h, int layer, const void* host_blob);
+
+/* Decode (0) or prefill (1) cache policy.  Prefill: a forward of layer 0 first
+ * prefetches every expert of layer 0, and each forward of layer l issues the
+ * prefetch of every expert of layer l+1 on the copy stream after its own routed
+ * accesses, so the copy overlaps layer l's kernels. */
+FT_API int ft_moe_set_mode(ft_moe* h, int prefill);
+
+/* Grows the per-forward scratch for up to max_tokens tokens (forward grows it on
+ * demand too, with a device synchronisation). */
+FT_API int ft_moe_reserve(ft_moe* h, int max_tokens);
+
+/* One MoE layer on n_tokens tokens.
+ *   x        device [n_tokens][H], float32 for FT_W_F32 stacks, bf16 otherwise.
+ *   router_w device [E][H] float32.
+ *   out      device [n_tokens][H], same type as x.
+ *   stream   caller's stream; every kernel and the wait for slot fills run on it.
+ * Steps: router logits (fp32) and top-k with normalised gates; one host read of
+ * the selected expert ids (the host waits for it, with a deadline); the LRU
+ * lookup and update over the distinct selected experts (hits in ascending expert
+ * order first, then misses in ascending order, each taking the lowest free slot or
+ * evicting the least recently used entry); copies of missed experts from the
+ * pinned pool into their slots on the library's copy stream, each after the
+ * kernels that last read the slot; token permutation by expert; the SwiGLU FFN of
+ * every selected expert reading its weights from its slot; the gate-weighted sum of
+ * the k outputs in ascending k order, plus the shared expert.
+ * Returns FT_ERR_CAPACITY, before any state changes, if the distinct experts of
+ * the call exceed the cache slots.  All forwards of a handle are ordered: a
+ * forward on another stream first waits for the previous forward's kernels. */
+FT_API int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const float* router_w,
+                   void* out, void* stream);
+
+/* Copies the routing of the last forward to host memory: ids [n_tokens][k] (expert
+ * indices, by descending logit, ties to the lower index) and gates [n_tokens][k].
+ * Either pointer may be NULL. */
+FT_API int ft_moe_last_routing(const ft_moe* h, int* ids, float* gates, int* n_tokens);
+
+/* Changes the number of slots at a safe point: waits for all work of the handle,
+ * then grows (entries keep slot and recency; new slots are free) or shrinks
+ * (least recently used entries are evicted down to the new size; survivors in
+ * slots >= slots are moved, most recent first, into the lowest free slots below
+ * it, keeping recency).  Reallocates the arena and copies resident slots on the
+ * device.  FT_ERR_BUSY if a forward is in flight on another thread. */
+FT_API int ft_cache_resize(ft_moe* h, int slots);
+
+/* Reads the counters (waits for the copy stream so h2d_seconds is complete). */
+FT_API int ft_cache_stats(const ft_moe* h, ft_cache_stats_t* out);
+FT_API int ft_cache_reset_stats(ft_moe* h);
+
+/* Copies up to `cap` trace records, oldest first, into buf and sets *n to the
+ * number recorded since the trace was last cleared (may exceed cap).  Tracing is
+ * on by default; ft_cache_set_trace(h, 0) turns it off and clears it. */
+FT_API int ft_cache_trace(const ft_moe* h, ft_access_t* buf, int cap, int* n);
+FT_API int ft_cache_set_trace(ft_moe* h, int enabled);
+
+/* Slot currently holding (layer, expert), or -1. */
+FT_API int ft_cache_slot_of(const ft_moe* h, int layer, int expert);
+
+/* Device address of slot s in the arena (valid until the next resize). */
+FT_API void* ft_cache_slot_ptr(ft_moe* h, int slot);
+
+/* Per-stage device time and launch counts of the handle's forwards.  Stage times are
+ * summed CUDA-event intervals on the forward's stream, taken only while stage timing
+ * is on; ffn_gate_up and ffn_down start after the wait for slot fills, so they hold
+ * kernel time only.  *_bytes are the algorithmic bytes of those launches: the weight
+ * bytes of every selected expert (and the shared expert) plus their input and output
+ * vectors. */
+typedef struct {
+  long long forwards;
+  long long kernel_launches;
+  long long timed_forwards;
+  double router_ms;        /* router logits + top-k/gates */
+  double permute_ms;
+  double ffn_gate_up_ms;   /* gate/up GEMV or GEMM + SwiGLU */
+  double ffn_down_ms;
+  double combine_ms;
+  double ffn_gate_up_bytes;
+  double ffn_down_bytes;
+  double ffn_flops;        /* 2 * (3 * H * I) per (token, expert) pair */
+  double host_wait_ms;     /* host time spent waiting for the routing ids */
+} ft_perf_t;
+
+FT_API int ft_moe_set_stage_timing(ft_moe* h, int enabled);
+/* Waits for the timed forwards and reads the counters. */
+FT_API int ft_moe_perf(ft_moe* h, ft_perf_t* out);
+FT_API int ft_moe_reset_perf(ft_moe* h);
+
+/* Deadline of every host wait on the GPU, in milliseconds (default 20000). */
+FT_API int ft_moe_set_timeout_ms(ft_moe* h, int ms);
+
+/* Message of the last failed call on h, or of the last failed ft_moe_create when
+ * h is NULL (per host thread). */
+FT_API const char* ft_last_error(const ft_moe* h);
+
+/* Waits for the handle's work and frees everything it owns. */
+FT_API void ft_moe_destroy(ft_moe* h);
+
+/* Host-only replay of the cache policy (no GPU, no allocation on the device): runs the
+ * library's own slot table over a script and reports what the cache would do.  For
+ * capacity planning and for checking the policy without a GPU.
+ * ops is a flat int array of records:
+ *   {0, call, layer, kind, n, e_1 .. e_n}  one access set (distinct experts of one layer;
+ *                                           any order, they are sorted first)
+ *   {1, new_capacity}                      a resize at a safe point
+ * A set larger than the capacity is skipped, changes nothing, and is counted in
+ * *n_capacity_errors.  trace receives up to trace_cap records; *n_trace is the total.
+ * stats (may be NULL) receives the counters (h2d fields zero).  Returns FT_ERR_INVALID
+ * for a malformed script or out-of-range ids. */
+FT_API int ft_cache_simulate(int num_layers, int num_experts, int capacity, const int* ops,
+                             int n_ops_ints, ft_access_t* trace, int trace_cap, int* n_trace,
+                             ft_cache_stats_t* stats, int* n_capacity_errors);
+
+/* ------------------------------------------------------------------------ *
+ * Step-level kernels.  Each runs one step of the forward on caller-owned device
+ * buffers, on `stream`, without the cache.  They are the same kernels the
+ * forward launches.  They allocate nothing, return after the launch, and report
+ * launch errors only.
+ * ------------------------------------------------------------------------ */
+
+/* Router + gating ("FreeToken linux", MoE memory handling: a few experts per token).
+ * z[t][e] = sum_h x[t][h] * router_w[e][h] in fp32.  ids[t][:] = the top_k experts
+ * by z (descending, ties to the lower index).  gates[t][j] = softmax or sigmoid of
+ * the selected logits, normalised over the k selected.
+ *   x: [T][H] (x_is_bf16 ? bf16 : f32), router_w: [E][H] f32, logits: [T][E] f32
+ *   (written), ids: [T][k] int32, gates: [T][k] f32. */
+FT_API int ft_router_topk(const void* x, int x_is_bf16, const float* router_w, int T, int H, int E,
+                   int top_k, int gating, float* logits, int* ids, float* gates, void* stream);
+
+/* Token permutation by expert.  counts[e] = pairs routed to e; offsets = exclusive
+ * prefix sum (E+1 entries); perm[q] = flat pair index t*k + j for q in expert-major
+ * order, ascending token inside an expert (a stable counting sort); inv (optional,
+ * may be NULL) is its inverse: inv[t*k + j] = q.
+ *   ids: [T][k] int32 in [0, E).  counts: [E], offsets: [E+1], perm, inv: [T*k] int32.
+ * One CTA; T*k up to 2^31. */
+FT_API int ft_permute(const int* ids, int T, int top_k, int E, int* counts, int* offsets, int* perm,
+               int* inv, void* stream);
+
+/* SwiGLU FFN of a list of experts for decode-sized batches: every weight byte is
+ * read once per launch.  blobs and experts are HOST arrays of n_list entries
+ * (n_list <= FT_MAX_EXPERTS + 1); blobs[i] is the DEVICE address of entry i's blob
+ * (runtime layout, see ft_moe_pool_ptr).  Entry i owns the pairs q in
+ * [offsets[e], offsets[e+1]) with e = experts[i], whose token is perm[q] / k; or, for
+ * experts[i] = -1 (a shared expert), the pairs q = T*k + t for every token t.
+ *     h[q] = silu(W_gate x_t) * (W_up x_t)        (h: [T*k + T][I] f32, device)
+ *     y[q] = W_down h[q]                          (y: [T*k + T][H] f32, device)
+ *   x: [T][H] device, f32 for FT_W_F32, else bf16.  max_pairs_per_expert: the largest
+ *   pair count of one entry (sizes the per-CTA token staging; larger values are
+ *   processed in chunks of 8).  Rows of h / y that no entry owns are not written. */
+FT_API int ft_expert_ffn_decode(const void* x, int T, int H, int I, int top_k, int wdtype,
+                         const void* const* blobs, const int* experts, int n_list,
+                         int max_pairs_per_expert, const int* offsets, const int* perm, float* h,
+                         float* y, void* stream);
+
+/* Gate-weighted combine: out[t] = sum_{j<k} gates[t][j] * y[inv[t*k+j]], summed in
+ * ascending j in fp32, plus y[T*k + t] (weight 1) when has_shared.
+ *   y: device f32 rows (see ft_expert_ffn_decode), gates: [T][k] f32, inv: [T*k] int32,
+ *   out: [T][H], bf16 if out_is_bf16 else f32 (round to nearest even).  H % 4 == 0. */
+FT_API int ft_combine(const float* y, const float* gates, const int* inv, int T, int H, int top_k,
+               int has_shared, int out_is_bf16, void* out, void* stream);
+
+/* Version string of the library build. */
+FT_API const char* ft_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FTMOE_H */

@@ -1,0 +1,862 @@
+// C ABI of the routed-MoE layer stack over a shared LRU expert-slot cache.
+//
+// Method (FreeToken pages): the full routed-expert pool stays in pinned host
+// memory; a fixed number of GPU expert slots, managed by one LRU shared by all
+// MoE layers, hold recently used experts; a miss is copied over PCIe into a
+// slot and kept ("FreeToken linux", "FreeToken's MoE memory handling";
+// "FreeToken gguf", `offload` backend).  Prefill copies the next layer's
+// experts while the current layer runs (whole-layer double buffering, same
+// section).  The cache is resized at a safe point ("FreeToken RTX 5090",
+// dynamic reconfiguration).
+//
+// Ordering (all CUDA work of a handle):
+//   compute stream = the caller's stream of each forward; copies run on the
+//   library's copy stream.  Before a slot is overwritten, the copy stream waits
+//   for the event recorded after the last forward that read it (use ring).
+//   Before a forward's kernels read a slot, the compute stream waits for the
+//   event recorded after the slot's last fill (fill ring).  Both rings are
+//   FIFO-ordered, so waiting on the newest relevant event covers older ones.
+#include <algorithm>
+#include <atomic>
+#include <chrono>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <thread>
+#include <vector>
+
+#include "../../include/ftmoe.h"
+#include "cache.hpp"
+#include "kernels.hpp"
+
+namespace {
+
+thread_local std::string g_create_error;
+constexpr int kRing = 128;
+
+struct FillTiming {
+  cudaEvent_t a, b;
+};
+
+// Stage boundaries of one timed forward, on its stream.
+enum { SE_R0, SE_R1, SE_P0, SE_P1, SE_G0, SE_G1, SE_D1, SE_C1, SE_N };
+struct StageEvents {
+  cudaEvent_t ev[SE_N];
+  double gu_bytes, d_bytes, flops;
+};
+
+}  // namespace
+
+struct ft_moe {
+  int device = 0;
+  int E = 0, k = 0, H = 0, I = 0, wdtype = 0;
+  int L = 1, gating = 0, has_shared = 0, prefill = 0;
+  size_t blob = 0;
+  uint8_t* pool = nullptr;
+  size_t pool_bytes = 0;
+  uint8_t* arena = nullptr;
+  int C = 0;
+  uint8_t* shared = nullptr;
+  ftc::SlotLru lru;
+  cudaStream_t copy = nullptr;
+
+  cudaEvent_t use_ev[kRing];
+  long long use_ev_call[kRing];
+  cudaEvent_t fill_ev[kRing];
+  long long fill_ev_batch[kRing];
+  long long call = 0;
+  long long fill_batches = 0;
+  std::vector<long long> slot_last_use;    // last forward call that read the slot
+  std::vector<long long> slot_fill_batch;  // last fill batch that wrote the slot
+  long long copy_waited_use = -1;
+  long long compute_waited_fill = -1;
+  cudaStream_t last_stream = nullptr;
+  bool has_last_stream = false;
+
+  std::vector<FillTiming> timing_pending, timing_free;
+  double h2d_seconds = 0.0;
+
+  int cap_tokens = 0;
+  float* d_logits = nullptr;
+  int* d_ids = nullptr;
+  float* d_gates = nullptr;
+  int* d_counts = nullptr;
+  int* d_offsets = nullptr;
+  int* d_perm = nullptr;
+  int* d_inv = nullptr;
+  float* d_h = nullptr;
+  float* d_y = nullptr;
+  int* h_ids = nullptr;
+  cudaEvent_t route_ev = nullptr;
+  int last_T = 0;
+
+  ft_cache_stats_t st{};
+  ft_perf_t perf{};
+  bool stage_timing = false;
+  std::vector<StageEvents> stage_pending, stage_free;
+  bool trace_on = true;
+  std::vector<ftc::Access> trace;
+  int timeout_ms = 20000;
+  std::string err;
+  std::atomic<int> busy{0};
+};
+
+namespace {
+
+int fail(ft_moe* h, int code, const std::string& msg) {
+  if (h) h->err = msg;
+  return code;
+}
+
+int cuda_fail(ft_moe* h, cudaError_t e, const char* what) {
+  return fail(h, FT_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+#define FT_CUDA(h, call)                                   \
+  do {                                                     \
+    cudaError_t _e = (call);                               \
+    if (_e != cudaSuccess) return cuda_fail((h), _e, #call); \
+  } while (0)
+
+struct BusyGuard {
+  ft_moe* h;
+  bool ok;
+  explicit BusyGuard(ft_moe* hh) : h(hh) { ok = h->busy.exchange(1) == 0; }
+  ~BusyGuard() {
+    if (ok) h->busy.store(0);
+  }
+};
+
+// Host wait on an event, polling with a deadline.
+int wait_event(ft_moe* h, cudaEvent_t ev, const char* what) {
+  auto t0 = std::chrono::steady_clock::now();
+  for (;;) {
+    cudaError_t q = cudaEventQuery(ev);
+    if (q == cudaSuccess) return FT_OK;
+    if (q != cudaErrorNotReady) return cuda_fail(h, q, what);
+    auto dt = std::chrono::steady_clock::now() - t0;
+    if (std::chrono::duration_cast<std::chrono::milliseconds>(dt).count() > h->timeout_ms)
+      return fail(h, FT_ERR_TIMEOUT, std::string("timed out waiting for ") + what);
+  }
+}
+
+void free_scratch(ft_moe* h) {
+  cudaFree(h->d_logits); cudaFree(h->d_ids); cudaFree(h->d_gates); cudaFree(h->d_counts);
+  cudaFree(h->d_offsets); cudaFree(h->d_perm); cudaFree(h->d_inv); cudaFree(h->d_h);
+  cudaFree(h->d_y);
+  if (h->h_ids) cudaFreeHost(h->h_ids);
+  h->d_logits = nullptr; h->d_ids = nullptr; h->d_gates = nullptr; h->d_counts = nullptr;
+  h->d_offsets = nullptr; h->d_perm = nullptr; h->d_inv = nullptr; h->d_h = nullptr;
+  h->d_y = nullptr; h->h_ids = nullptr;
+  h->cap_tokens = 0;
+}
+
+int ensure_scratch(ft_moe* h, int T) {
+  if (T <= h->cap_tokens) return FT_OK;
+  // the old buffers may still be read by queued kernels
+  if (h->has_last_stream) FT_CUDA(h, cudaStreamSynchronize(h->last_stream));
+  free_scratch(h);
+  const size_t pairs = (size_t)T * h->k, rows = pairs + T;
+  bool ok = cudaMalloc(&h->d_logits, sizeof(float) * (size_t)T * h->E) == cudaSuccess &&
+            cudaMalloc(&h->d_ids, sizeof(int) * pairs) == cudaSuccess &&
+            cudaMalloc(&h->d_gates, sizeof(float) * pairs) == cudaSuccess &&
+            cudaMalloc(&h->d_counts, sizeof(int) * h->E) == cudaSuccess &&
+            cudaMalloc(&h->d_offsets, sizeof(int) * (h->E + 1)) == cudaSuccess &&
+            cudaMalloc(&h->d_perm, sizeof(int) * pairs) == cudaSuccess &&
+            cudaMalloc(&h->d_inv, sizeof(int) * pairs) == cudaSuccess &&
+            cudaMalloc(&h->d_h, sizeof(float) * rows * h->I) == cudaSuccess &&
+            cudaMalloc(&h->d_y, sizeof(float) * rows * h->H) == cudaSuccess &&
+            cudaHostAlloc(&h->h_ids, sizeof(int) * pairs, cudaHostAllocDefault) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    free_scratch(h);
+    return fail(h, FT_ERR_OOM, "scratch allocation failed");
+  }
+  h->cap_tokens = T;
+  return FT_OK;
+}
+
+int ensure_pool(ft_moe* h) {
+  if (h->pool) return FT_OK;
+  size_t bytes = (size_t)h->L * h->E * h->blob;
+  if (cudaHostAlloc(&h->pool, bytes, cudaHostAllocPortable) != cudaSuccess) {
+    cudaGetLastError();
+    h->pool = nullptr;
+    return fail(h, FT_ERR_OOM, "pinned pool allocation failed");
+  }
+  h->pool_bytes = bytes;
+  return FT_OK;
+}
+
+void reset_cache_state(ft_moe* h) {
+  h->lru.reset(h->L * h->E, h->C);
+  h->slot_last_use.assign(h->C, -1);
+  h->slot_fill_batch.assign(h->C, -1);
+}
+
+FillTiming get_timing(ft_moe* h) {
+  if (!h->timing_free.empty()) {
+    FillTiming t = h->timing_free.back();
+    h->timing_free.pop_back();
+    return t;
+  }
+  FillTiming t;
+  cudaEventCreate(&t.a);
+  cudaEventCreate(&t.b);
+  return t;
+}
+
+// Adds finished fill intervals to h2d_seconds.  block: wait for all of them.
+void harvest_timing(ft_moe* h, bool block) {
+  std::vector<FillTiming> keep;
+  for (auto& t : h->timing_pending) {
+    if (block) cudaEventSynchronize(t.b);
+    if (cudaEventQuery(t.b) == cudaSuccess) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, t.a, t.b) == cudaSuccess) h->h2d_seconds += ms * 1e-3;
+      h->timing_free.push_back(t);
+    } else {
+      keep.push_back(t);
+    }
+  }
+  h->timing_pending.swap(keep);
+}
+
+// Copies the experts of the missed accesses in recs[first..] into their slots.
+int issue_fills(ft_moe* h, std::vector<ftc::Access>& recs, size_t first) {
+  std::vector<int> slots;
+  long long need_use = -1;
+  for (size_t i = first; i < recs.size(); ++i)
+    if (!recs[i].hit) {
+      slots.push_back(recs[i].slot);
+      need_use = std::max(need_use, h->slot_last_use[recs[i].slot]);
+    }
+  if (slots.empty()) return FT_OK;
+  if (need_use > h->copy_waited_use) {
+    const int r = (int)(need_use % kRing);
+    FT_CUDA(h, cudaStreamWaitEvent(h->copy, h->use_ev[r], 0));
+    h->copy_waited_use = h->use_ev_call[r];
+  }
+  FillTiming tm = get_timing(h);
+  cudaEventRecord(tm.a, h->copy);
+  for (size_t i = first; i < recs.size(); ++i) {
+    if (recs[i].hit) continue;
+    const ftc::Access& a = recs[i];
+    const uint8_t* src = h->pool + ((size_t)a.layer * h->E + a.expert) * h->blob;
+    uint8_t* dst = h->arena + (size_t)a.slot * h->blob;
+    cudaError_t e = cudaMemcpyAsync(dst, src, h->blob, cudaMemcpyHostToDevice, h->copy);
+    if (e != cudaSuccess) {
+      // roll back this and every later fill of the set to "not resident"
+      for (size_t j = i; j < recs.size(); ++j)
+        if (!recs[j].hit) h->lru.drop(recs[j].slot);
+      h->timing_free.push_back(tm);
+      return cuda_fail(h, e, "cudaMemcpyAsync (slot fill)");
+    }
+    h->st.h2d_bytes += (long long)h->blob;
+  }
+  cudaEventRecord(tm.b, h->copy);
+  h->timing_pending.push_back(tm);
+  if (h->timing_pending.size() > 64) harvest_timing(h, false);
+  const long long b = h->fill_batches++;
+  const int r = (int)(b % kRing);
+  FT_CUDA(h, cudaEventRecord(h->fill_ev[r], h->copy));
+  h->fill_ev_batch[r] = b;
+  for (int s : slots) h->slot_fill_batch[s] = b;
+  return FT_OK;
+}
+
+StageEvents* stage_begin(ft_moe* h) {
+  if (!h->stage_timing) return nullptr;
+  if (h->stage_free.empty()) {
+    StageEvents se;
+    for (int i = 0; i < SE_N; ++i) cudaEventCreate(&se.ev[i]);
+    h->stage_free.push_back(se);
+  }
+  h->stage_pending.push_back(h->stage_free.back());
+  h->stage_free.pop_back();
+  StageEvents* se = &h->stage_pending.back();
+  se->gu_bytes = se->d_bytes = se->flops = 0.0;
+  return se;
+}
+
+void stage_mark(StageEvents* se, int which, cudaStream_t s) {
+  if (se) cudaEventRecord(se->ev[which], s);
+}
+
+void harvest_stages(ft_moe* h, bool block) {
+  std::vector<StageEvents> keep;
+  for (auto& se : h->stage_pending) {
+    if (block) cudaEventSynchronize(se.ev[SE_C1]);
+    if (cudaEventQuery(se.ev[SE_C1]) != cudaSuccess) {
+      keep.push_back(se);
+      continue;
+    }
+    auto ms = [&](int a, int b) {
+      float t = 0.f;
+      cudaEventElapsedTime(&t, se.ev[a], se.ev[b]);
+      return (double)t;
+    };
+    h->perf.router_ms += ms(SE_R0, SE_R1);
+    h->perf.permute_ms += ms(SE_P0, SE_P1);
+    h->perf.ffn_gate_up_ms += ms(SE_G0, SE_G1);
+    h->perf.ffn_down_ms += ms(SE_G1, SE_D1);
+    h->perf.combine_ms += ms(SE_D1, SE_C1);
+    h->perf.ffn_gate_up_bytes += se.gu_bytes;
+    h->perf.ffn_down_bytes += se.d_bytes;
+    h->perf.ffn_flops += se.flops;
+    h->perf.timed_forwards++;
+    h->stage_free.push_back(se);
+  }
+  h->stage_pending.swap(keep);
+}
+
+void account(ft_moe* h, const std::vector<ftc::Access>& recs, size_t first) {
+  for (size_t i = first; i < recs.size(); ++i) {
+    const ftc::Access& a = recs[i];
+    if (a.kind == FT_ROUTED) {
+      h->st.routed++;
+      if (a.hit) h->st.hits++; else h->st.misses++;
+    } else {
+      h->st.prefetch++;
+      if (a.hit) h->st.prefetch_hits++; else h->st.prefetch_misses++;
+    }
+    if (a.ev_layer >= 0) h->st.evictions++;
+    if (h->trace_on) h->trace.push_back(a);
+  }
+}
+
+std::vector<int> all_keys(const ft_moe* h, int layer) {
+  std::vector<int> keys(h->E);
+  for (int e = 0; e < h->E; ++e) keys[e] = layer * h->E + e;
+  return keys;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ft_version(void) { return "ftmoe 0.1 sm_100a"; }
+
+ft_moe* ft_moe_create(int num_experts, int top_k, int hidden, int inter, int wdtype,
+                      int cache_slots) {
+  if (num_experts < 1 || num_experts > FT_MAX_EXPERTS || top_k < 1 || top_k > num_experts ||
+      top_k > FT_MAX_TOPK || hidden < 8 || inter < 8 || hidden % 8 || inter % 8 ||
+      wdtype < FT_W_F32 || wdtype > FT_W_INT4_G128 || cache_slots < 1) {
+    g_create_error = "ft_moe_create: invalid argument";
+    return nullptr;
+  }
+  if (wdtype == FT_W_INT4_G128 && (hidden % 128 || inter % 128)) {
+    g_create_error = "ft_moe_create: int4 needs hidden and inter multiples of 128";
+    return nullptr;
+  }
+  ft_moe* h = new ft_moe();
+  cudaGetDevice(&h->device);
+  h->E = num_experts; h->k = top_k; h->H = hidden; h->I = inter; h->wdtype = wdtype;
+  h->C = cache_slots;
+  const size_t n = 3ull * hidden * inter;
+  h->blob = wdtype == FT_W_F32 ? 4 * n : wdtype == FT_W_BF16 ? 2 * n : n / 2 + 2 * (n / 128);
+  if (cudaMalloc(&h->arena, (size_t)cache_slots * h->blob) != cudaSuccess) {
+    cudaGetLastError();
+    g_create_error = "ft_moe_create: slot arena allocation failed";
+    delete h;
+    return nullptr;
+  }
+  cudaStreamCreateWithFlags(&h->copy, cudaStreamNonBlocking);
+  for (int i = 0; i < kRing; ++i) {
+    cudaEventCreateWithFlags(&h->use_ev[i], cudaEventDisableTiming);
+    cudaEventCreateWithFlags(&h->fill_ev[i], cudaEventDisableTiming);
+    h->use_ev_call[i] = -1;
+    h->fill_ev_batch[i] = -1;
+  }
+  cudaEventCreateWithFlags(&h->route_ev, cudaEventDisableTiming);
+  reset_cache_state(h);
+  if (cudaGetLastError() != cudaSuccess) {
+    g_create_error = "ft_moe_create: CUDA setup failed";
+    ft_moe_destroy(h);
+    return nullptr;
+  }
+  return h;
+}
+
+int ft_moe_set_layers(ft_moe* h, int num_layers, int gating, int has_shared_expert) {
+  if (!h) return FT_ERR_INVALID;
+  if (num_layers < 1 || (gating != FT_GATE_SOFTMAX && gating != FT_GATE_SIGMOID))
+    return fail(h, FT_ERR_INVALID, "ft_moe_set_layers: invalid argument");
+  BusyGuard g(h);
+  if (!g.ok) return fail(h, FT_ERR_BUSY, "ft_moe_set_layers: forward in flight");
+  cudaStreamSynchronize(h->copy);
+  if (h->has_last_stream) cudaStreamSynchronize(h->last_stream);
+  if (num_layers != h->L && h->pool) {
+    cudaFreeHost(h->pool);
+    h->pool = nullptr;
+  }
+  if (h->shared) {
+    cudaFree(h->shared);
+    h->shared = nullptr;
+  }
+  h->L = num_layers;
+  h->gating = gating;
+  h->has_shared = has_shared_expert ? 1 : 0;
+  int rc = ensure_pool(h);
+  if (rc) return rc;
+  if (h->has_shared) {
+    if (cudaMalloc(&h->shared, (size_t)h->L * h->blob) != cudaSuccess) {
+      cudaGetLastError();
+      h->shared = nullptr;
+      return fail(h, FT_ERR_OOM, "shared-expert allocation failed");
+    }
+    FT_CUDA(h, cudaMemset(h->shared, 0, (size_t)h->L * h->blob));
+  }
+  reset_cache_state(h);
+  return FT_OK;
+}
+
+size_t ft_moe_blob_bytes(const ft_moe* h) { return h ? h->blob : 0; }
+
+void* ft_moe_pool_ptr(ft_moe* h, int layer, int expert) {
+  if (!h || layer < 0 || layer >= h->L || expert < 0 || expert >= h->E) return nullptr;
+  if (ensure_pool(h) != FT_OK) return nullptr;
+  return h->pool + ((size_t)layer * h->E + expert) * h->blob;
+}
+
+int ft_moe_set_shared(ft_moe* h, int layer, const void* host_blob) {
+  if (!h) return FT_ERR_INVALID;
+  if (!h->has_shared || !h->shared || layer < 0 || layer >= h->L || !host_blob)
+    return fail(h, FT_ERR_INVALID, "ft_moe_set_shared: no shared expert or bad layer");
+  FT_CUDA(h, cudaMemcpy(h->shared + (size_t)layer * h->blob, host_blob, h->blob,
+                        cudaMemcpyHostToDevice));
+  return FT_OK;
+}
+
+int ft_moe_set_mode(ft_moe* h, int prefill) {
+  if (!h) return FT_ERR_INVALID;
+  h->prefill = prefill ? 1 : 0;
+  return FT_OK;
+}
+
+int ft_moe_reserve(ft_moe* h, int max_tokens) {
+  if (!h || max_tokens < 0) return FT_ERR_INVALID;
+  BusyGuard g(h);
+  if (!g.ok) return fail(h, FT_ERR_BUSY, "ft_moe_reserve: forward in flight");
+  return ensure_scratch(h, max_tokens);
+}
+
+int ft_moe_set_timeout_ms(ft_moe* h, int ms) {
+  if (!h || ms < 1) return FT_ERR_INVALID;
+  h->timeout_ms = ms;
+  return FT_OK;
+}
+
+int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const float* router_w,
+                   void* out, void* stream_) {
+  if (!h) return FT_ERR_INVALID;
+  if (layer < 0 || layer >= h->L || n_tokens < 0 || (n_tokens > 0 && (!x || !router_w || !out)))
+    return fail(h, FT_ERR_INVALID, "ft_moe_forward: invalid argument");
+  if (!h->pool) return fail(h, FT_ERR_INVALID, "ft_moe_forward: pool not allocated");
+  if (n_tokens == 0) return FT_OK;
+  BusyGuard g(h);
+  if (!g.ok) return fail(h, FT_ERR_BUSY, "ft_moe_forward: another call in flight");
+  cudaStream_t s = static_cast<cudaStream_t>(stream_);
+  const int T = n_tokens, E = h->E, k = h->k;
+  int rc = ensure_scratch(h, T);
+  if (rc) return rc;
+  // keep forwards of this handle ordered across streams
+  if (h->has_last_stream && s != h->last_stream && h->call > 0) {
+    const int r = (int)((h->call - 1) % kRing);
+    FT_CUDA(h, cudaStreamWaitEvent(s, h->use_ev[r], 0));
+  }
+  const bool xbf16 = h->wdtype != FT_W_F32;
+  if (h->stage_pending.size() > 256) harvest_stages(h, false);
+  StageEvents* se = stage_begin(h);
+  stage_mark(se, SE_R0, s);
+  FT_CUDA(h, ftk::launch_router_logits(x, xbf16, router_w, T, h->H, E, h->d_logits, s));
+  FT_CUDA(h, ftk::launch_topk_gates(h->d_logits, T, E, k, h->gating, h->d_ids, h->d_gates, s));
+  stage_mark(se, SE_R1, s);
+  FT_CUDA(h, cudaMemcpyAsync(h->h_ids, h->d_ids, sizeof(int) * (size_t)T * k,
+                             cudaMemcpyDeviceToHost, s));
+  FT_CUDA(h, cudaEventRecord(h->route_ev, s));
+  stage_mark(se, SE_P0, s);
+  FT_CUDA(h, ftk::launch_permute(h->d_ids, T, k, E, h->d_counts, h->d_offsets, h->d_perm,
+                                 h->d_inv, s));
+  stage_mark(se, SE_P1, s);
+  h->perf.kernel_launches += 3;
+  h->perf.forwards++;
+  {
+    auto w0 = std::chrono::steady_clock::now();
+    rc = wait_event(h, h->route_ev, "routing ids");
+    h->perf.host_wait_ms +=
+        std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - w0).count();
+  }
+  if (rc) return rc;
+  h->last_T = T;
+
+  // distinct selected experts, ascending, and the largest token count of one expert
+  std::vector<int> cnt(E, 0);
+  for (int i = 0; i < T * k; ++i) {
+    const int e = h->h_ids[i];
+    if (e < 0 || e >= E) return fail(h, FT_ERR_DEVICE_CHECK, "router produced an invalid expert id");
+    cnt[e]++;
+  }
+  std::vector<int> S, keys;
+  int max_pairs = 0;
+  for (int e = 0; e < E; ++e)
+    if (cnt[e]) {
+      S.push_back(e);
+      keys.push_back(layer * E + e);
+      max_pairs = std::max(max_pairs, cnt[e]);
+    }
+  const bool pre0 = h->prefill && layer == 0;
+  const bool pre_next = h->prefill && layer + 1 < h->L;
+  if ((int)S.size() > h->C || ((pre0 || pre_next) && E > h->C))
+    return fail(h, FT_ERR_CAPACITY, "cache has fewer slots than one step needs");
+
+  const long long call = h->call;
+  std::vector<ftc::Access> recs;
+  if (pre0) {
+    h->lru.access_set(all_keys(h, 0), E, (int)call, FT_PREFETCH, recs);
+    rc = issue_fills(h, recs, 0);
+    account(h, recs, 0);
+    if (rc) return rc;
+  }
+  const size_t first_routed = recs.size();
+  h->lru.access_set(keys, E, (int)call, FT_ROUTED, recs);
+  rc = issue_fills(h, recs, first_routed);
+  account(h, recs, first_routed);
+  if (rc) return rc;
+
+  // the kernels read the slots of S: wait for their newest fill
+  ftk::ExpertList list;
+  list.n = 0;
+  long long need_fill = -1;
+  for (size_t i = 0; i < S.size(); ++i) {
+    const int slot = h->lru.slot_of(keys[i]);
+    list.expert[list.n] = S[i];
+    list.blob[list.n] = h->arena + (size_t)slot * h->blob;
+    list.n++;
+    need_fill = std::max(need_fill, h->slot_fill_batch[slot]);
+  }
+  if (h->has_shared) {
+    list.expert[list.n] = -1;
+    list.blob[list.n] = h->shared + (size_t)layer * h->blob;
+    list.n++;
+  }
+  if (need_fill > h->compute_waited_fill || (need_fill >= 0 && s != h->last_stream)) {
+    const int r = (int)(need_fill % kRing);
+    FT_CUDA(h, cudaStreamWaitEvent(s, h->fill_ev[r], 0));
+    h->compute_waited_fill = h->fill_ev_batch[r];
+  }
+  if (se) {
+    // algorithmic bytes: every weight of the listed experts once, their inputs and outputs
+    const double xb = xbf16 ? 2.0 : 4.0;
+    const size_t mat = (size_t)h->H * h->I;
+    const double wmat = h->wdtype == FT_W_INT4_G128 ? mat / 2.0 + 2.0 * (mat / 128) :
+                        (double)mat * (h->wdtype == FT_W_F32 ? 4 : 2);
+    const double pairs = (double)T * k + (h->has_shared ? T : 0);
+    se->gu_bytes = list.n * 2.0 * wmat + pairs * (h->H * xb + h->I * 4.0);
+    se->d_bytes = list.n * wmat + pairs * (h->I * 4.0 + h->H * 4.0);
+    se->flops = pairs * 6.0 * mat;
+  }
+  stage_mark(se, SE_G0, s);
+  FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, list, max_pairs, h->d_offsets,
+                                    h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr));
+  stage_mark(se, SE_D1, s);
+  FT_CUDA(h, ftk::launch_combine(h->d_y, h->d_gates, h->d_inv, T, h->H, k, h->has_shared != 0,
+                                 xbf16, out, s));
+  stage_mark(se, SE_C1, s);
+  h->perf.kernel_launches += 3;
+  {
+    const int r = (int)(call % kRing);
+    FT_CUDA(h, cudaEventRecord(h->use_ev[r], s));
+    h->use_ev_call[r] = call;
+    for (int key : keys) h->slot_last_use[h->lru.slot_of(key)] = call;
+  }
+  h->last_stream = s;
+  h->has_last_stream = true;
+  h->call++;
+
+  if (pre_next) {
+    const size_t first_pre = recs.size();
+    h->lru.access_set(all_keys(h, layer + 1), E, (int)call, FT_PREFETCH, recs);
+    rc = issue_fills(h, recs, first_pre);
+    account(h, recs, first_pre);
+    if (rc) return rc;
+  }
+  return FT_OK;
+}
+
+int ft_moe_set_stage_timing(ft_moe* h, int enabled) {
+  if (!h) return FT_ERR_INVALID;
+  h->stage_timing = enabled != 0;
+  return FT_OK;
+}
+
+int ft_moe_perf(ft_moe* h, ft_perf_t* out) {
+  if (!h || !out) return FT_ERR_INVALID;
+  harvest_stages(h, true);
+  *out = h->perf;
+  return FT_OK;
+}
+
+int ft_moe_reset_perf(ft_moe* h) {
+  if (!h) return FT_ERR_INVALID;
+  harvest_stages(h, true);
+  h->perf = ft_perf_t{};
+  return FT_OK;
+}
+
+int ft_moe_last_routing(const ft_moe* hc, int* ids, float* gates, int* n_tokens) {
+  ft_moe* h = const_cast<ft_moe*>(hc);
+  if (!h) return FT_ERR_INVALID;
+  if (n_tokens) *n_tokens = h->last_T;
+  if (h->last_T == 0) return FT_OK;
+  if (h->has_last_stream) FT_CUDA(h, cudaStreamSynchronize(h->last_stream));
+  const size_t n = (size_t)h->last_T * h->k;
+  if (ids) FT_CUDA(h, cudaMemcpy(ids, h->d_ids, sizeof(int) * n, cudaMemcpyDeviceToHost));
+  if (gates) FT_CUDA(h, cudaMemcpy(gates, h->d_gates, sizeof(float) * n, cudaMemcpyDeviceToHost));
+  return FT_OK;
+}
+
+int ft_cache_resize(ft_moe* h, int slots) {
+  if (!h) return FT_ERR_INVALID;
+  if (slots < 1) return fail(h, FT_ERR_INVALID, "ft_cache_resize: slots must be >= 1");
+  BusyGuard g(h);
+  if (!g.ok) return fail(h, FT_ERR_BUSY, "ft_cache_resize: forward in flight");
+  FT_CUDA(h, cudaStreamSynchronize(h->copy));
+  if (h->has_last_stream) FT_CUDA(h, cudaStreamSynchronize(h->last_stream));
+  if (slots == h->C) return FT_OK;
+  uint8_t* na = nullptr;
+  if (cudaMalloc(&na, (size_t)slots * h->blob) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(h, FT_ERR_OOM, "ft_cache_resize: arena allocation failed");
+  }
+  std::vector<int> evicted;
+  std::vector<std::pair<int, int>> moves;
+  const int old_c = h->C;
+  std::vector<int> old_key_of(old_c);
+  for (int s2 = 0; s2 < old_c; ++s2) old_key_of[s2] = h->lru.key_of(s2);
+  h->lru.resize(slots, evicted, moves);
+  cudaError_t e = cudaSuccess;
+  if (slots > old_c) {
+    e = cudaMemcpyAsync(na, h->arena, (size_t)old_c * h->blob, cudaMemcpyDeviceToDevice, h->copy);
+  } else {
+    for (int s2 = 0; s2 < slots && e == cudaSuccess; ++s2)
+      if (h->lru.key_of(s2) >= 0 && old_key_of[s2] == h->lru.key_of(s2))
+        e = cudaMemcpyAsync(na + (size_t)s2 * h->blob, h->arena + (size_t)s2 * h->blob, h->blob,
+                            cudaMemcpyDeviceToDevice, h->copy);
+    for (auto& m : moves)
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(na + (size_t)m.second * h->blob, h->arena + (size_t)m.first * h->blob,
+                            h->blob, cudaMemcpyDeviceToDevice, h->copy);
+  }
+  if (e == cudaSuccess) e = cudaStreamSynchronize(h->copy);
+  if (e != cudaSuccess) {
+    cudaFree(na);
+    reset_cache_state(h);   // contents unknown: start empty
+    return cuda_fail(h, e, "ft_cache_resize copy");
+  }
+  cudaFree(h->arena);
+  h->arena = na;
+  h->C = slots;
+  h->st.evictions += (long long)evicted.size();
+  h->slot_last_use.assign(slots, -1);
+  h->slot_fill_batch.assign(slots, -1);
+  return FT_OK;
+}
+
+int ft_cache_stats(const ft_moe* hc, ft_cache_stats_t* out) {
+  ft_moe* h = const_cast<ft_moe*>(hc);
+  if (!h || !out) return FT_ERR_INVALID;
+  cudaStreamSynchronize(h->copy);
+  harvest_timing(h, true);
+  *out = h->st;
+  out->h2d_seconds = h->h2d_seconds;
+  out->resident = h->lru.size();
+  out->capacity = h->C;
+  return FT_OK;
+}
+
+int ft_cache_reset_stats(ft_moe* h) {
+  if (!h) return FT_ERR_INVALID;
+  cudaStreamSynchronize(h->copy);
+  harvest_timing(h, true);
+  h->st = ft_cache_stats_t{};
+  h->h2d_seconds = 0.0;
+  return FT_OK;
+}
+
+int ft_cache_trace(const ft_moe* h, ft_access_t* buf, int cap, int* n) {
+  if (!h || !n || cap < 0 || (cap > 0 && !buf)) return FT_ERR_INVALID;
+  *n = (int)h->trace.size();
+  const int m = std::min(cap, *n);
+  for (int i = 0; i < m; ++i) {
+    const ftc::Access& a = h->trace[i];
+    buf[i] = ft_access_t{a.call, a.layer, a.expert, a.kind, a.hit, a.slot, a.ev_layer, a.ev_expert};
+  }
+  return FT_OK;
+}
+
+int ft_cache_set_trace(ft_moe* h, int enabled) {
+  if (!h) return FT_ERR_INVALID;
+  h->trace_on = enabled != 0;
+  if (!h->trace_on) h->trace.clear();
+  return FT_OK;
+}
+
+int ft_cache_slot_of(const ft_moe* h, int layer, int expert) {
+  if (!h || layer < 0 || layer >= h->L || expert < 0 || expert >= h->E) return -1;
+  return h->lru.slot_of(layer * h->E + expert);
+}
+
+void* ft_cache_slot_ptr(ft_moe* h, int slot) {
+  if (!h || slot < 0 || slot >= h->C) return nullptr;
+  return h->arena + (size_t)slot * h->blob;
+}
+
+const char* ft_last_error(const ft_moe* h) {
+  return h ? h->err.c_str() : g_create_error.c_str();
+}
+
+void ft_moe_destroy(ft_moe* h) {
+  if (!h) return;
+  if (h->copy) cudaStreamSynchronize(h->copy);
+  if (h->has_last_stream) cudaStreamSynchronize(h->last_stream);
+  harvest_timing(h, true);
+  for (auto& t : h->timing_free) { cudaEventDestroy(t.a); cudaEventDestroy(t.b); }
+  for (int i = 0; i < kRing; ++i) {
+    if (h->use_ev[i]) cudaEventDestroy(h->use_ev[i]);
+    if (h->fill_ev[i]) cudaEventDestroy(h->fill_ev[i]);
+  }
+  if (h->route_ev) cudaEventDestroy(h->route_ev);
+  harvest_stages(h, true);
+  for (auto& se : h->stage_free)
+    for (int i = 0; i < SE_N; ++i) cudaEventDestroy(se.ev[i]);
+  free_scratch(h);
+  if (h->copy) cudaStreamDestroy(h->copy);
+  cudaFree(h->arena);
+  cudaFree(h->shared);
+  if (h->pool) cudaFreeHost(h->pool);
+  delete h;
+}
+
+int ft_cache_simulate(int num_layers, int num_experts, int capacity, const int* ops,
+                      int n_ops_ints, ft_access_t* trace, int trace_cap, int* n_trace,
+                      ft_cache_stats_t* stats, int* n_capacity_errors) {
+  if (num_layers < 1 || num_experts < 1 || capacity < 1 || n_ops_ints < 0 ||
+      (n_ops_ints > 0 && !ops) || !n_trace || trace_cap < 0 || (trace_cap > 0 && !trace))
+    return FT_ERR_INVALID;
+  ftc::SlotLru lru;
+  lru.reset(num_layers * num_experts, capacity);
+  std::vector<ftc::Access> recs;
+  ft_cache_stats_t st{};
+  int cap_err = 0;
+  int i = 0;
+  while (i < n_ops_ints) {
+    if (ops[i] == 0) {
+      if (i + 5 > n_ops_ints) return FT_ERR_INVALID;
+      const int call = ops[i + 1], layer = ops[i + 2], kind = ops[i + 3], n = ops[i + 4];
+      if (layer < 0 || layer >= num_layers || n < 0 || i + 5 + n > n_ops_ints ||
+          (kind != FT_ROUTED && kind != FT_PREFETCH))
+        return FT_ERR_INVALID;
+      std::vector<int> keys;
+      for (int j = 0; j < n; ++j) {
+        const int e = ops[i + 5 + j];
+        if (e < 0 || e >= num_experts) return FT_ERR_INVALID;
+        keys.push_back(layer * num_experts + e);
+      }
+      std::sort(keys.begin(), keys.end());
+      keys.erase(std::unique(keys.begin(), keys.end()), keys.end());
+      const size_t first = recs.size();
+      if (!lru.access_set(keys, num_experts, call, kind, recs)) {
+        cap_err++;
+      } else {
+        for (size_t r = first; r < recs.size(); ++r) {
+          const ftc::Access& a = recs[r];
+          if (a.kind == FT_ROUTED) { st.routed++; if (a.hit) st.hits++; else st.misses++; }
+          else { st.prefetch++; if (a.hit) st.prefetch_hits++; else st.prefetch_misses++; }
+          if (a.ev_layer >= 0) st.evictions++;
+        }
+      }
+      i += 5 + n;
+    } else if (ops[i] == 1) {
+      if (i + 2 > n_ops_ints || ops[i + 1] < 1) return FT_ERR_INVALID;
+      std::vector<int> evicted;
+      std::vector<std::pair<int, int>> moves;
+      lru.resize(ops[i + 1], evicted, moves);
+      st.evictions += (long long)evicted.size();
+      i += 2;
+    } else {
+      return FT_ERR_INVALID;
+    }
+  }
+  *n_trace = (int)recs.size();
+  for (int r = 0; r < std::min(trace_cap, *n_trace); ++r) {
+    const ftc::Access& a = recs[r];
+    trace[r] = ft_access_t{a.call, a.layer, a.expert, a.kind, a.hit, a.slot, a.ev_layer, a.ev_expert};
+  }
+  st.resident = lru.size();
+  st.capacity = lru.capacity();
+  if (stats) *stats = st;
+  if (n_capacity_errors) *n_capacity_errors = cap_err;
+  return FT_OK;
+}
+
+// ------------------------------------------------------------ step level --
+
+int ft_router_topk(const void* x, int x_is_bf16, const float* router_w, int T, int H, int E,
+                   int top_k, int gating, float* logits, int* ids, float* gates, void* stream) {
+  if (T < 0 || H < 4 || H % 4 || E < 1 || E > FT_MAX_EXPERTS || top_k < 1 || top_k > E ||
+      top_k > FT_MAX_TOPK || (T > 0 && (!x || !router_w || !logits || !ids || !gates)))
+    return FT_ERR_INVALID;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (ftk::launch_router_logits(x, x_is_bf16 != 0, router_w, T, H, E, logits, s) != cudaSuccess)
+    return FT_ERR_CUDA;
+  if (ftk::launch_topk_gates(logits, T, E, top_k, gating, ids, gates, s) != cudaSuccess)
+    return FT_ERR_CUDA;
+  return FT_OK;
+}
+
+int ft_permute(const int* ids, int T, int top_k, int E, int* counts, int* offsets, int* perm,
+               int* inv, void* stream) {
+  if (T < 0 || top_k < 1 || E < 1 || E > FT_MAX_EXPERTS || !counts || !offsets ||
+      (T > 0 && (!ids || !perm)))
+    return FT_ERR_INVALID;
+  return ftk::launch_permute(ids, T, top_k, E, counts, offsets, perm, inv,
+                             static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FT_OK
+             : FT_ERR_CUDA;
+}
+
+int ft_expert_ffn_decode(const void* x, int T, int H, int I, int top_k, int wdtype,
+                         const void* const* blobs, const int* experts, int n_list,
+                         int max_pairs_per_expert, const int* offsets, const int* perm, float* h,
+                         float* y, void* stream) {
+  if (T < 0 || H < 8 || I < 8 || H % 8 || I % 8 || top_k < 1 || n_list < 0 ||
+      n_list > ftk::kMaxList || wdtype < FT_W_F32 || wdtype > FT_W_INT4_G128 ||
+      (wdtype == FT_W_INT4_G128 && (H % 128 || I % 128)) ||
+      (n_list > 0 && (!blobs || !experts || !offsets || !perm || !h || !y || !x)))
+    return FT_ERR_INVALID;
+  ftk::ExpertList list;
+  list.n = n_list;
+  for (int i = 0; i < n_list; ++i) {
+    if (experts[i] < -1 || experts[i] >= FT_MAX_EXPERTS || !blobs[i]) return FT_ERR_INVALID;
+    list.expert[i] = experts[i];
+    list.blob[i] = static_cast<const uint8_t*>(blobs[i]);
+  }
+  return ftk::launch_ffn_decode(x, T, H, I, top_k, wdtype, list, max_pairs_per_expert, offsets,
+                                perm, h, y, static_cast<cudaStream_t>(stream), nullptr) == cudaSuccess
+             ? FT_OK
+             : FT_ERR_CUDA;
+}
+
+int ft_combine(const float* y, const float* gates, const int* inv, int T, int H, int top_k,
+               int has_shared, int out_is_bf16, void* out, void* stream) {
+  if (T < 0 || H < 4 || H % 4 || top_k < 1 || (T > 0 && (!y || !gates || !inv || !out)))
+    return FT_ERR_INVALID;
+  return ftk::launch_combine(y, gates, inv, T, H, top_k, has_shared != 0, out_is_bf16 != 0, out,
+                             static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FT_OK
+             : FT_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,166 @@
+// K1 - router logits and top-k gating.
+//
+// Method ("FreeToken linux", "FreeToken's MoE memory handling"): the router
+// scores every routed expert and activates a few per token (6 of 256 in
+// DeepSeek-V4-Flash).  Logits are fp32; the k largest are selected (ties to
+// the lower expert index) and their gates are the softmax, or the sigmoid,
+// of the selected logits normalised to sum to 1.
+#include "common.cuh"
+#include "kernels.hpp"
+
+namespace ftk {
+
+namespace {
+
+constexpr int kRouterThreads = 256;
+constexpr int kRouterEPB = 2;   // experts per CTA
+constexpr int kRouterTPB = 8;   // tokens per CTA
+
+template <typename XT>
+FT_DEVICE void load_x4(const XT* x, float v[4]);
+template <>
+FT_DEVICE void load_x4<float>(const float* x, float v[4]) {
+  float4 a = *reinterpret_cast<const float4*>(x);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+template <>
+FT_DEVICE void load_x4<uint16_t>(const uint16_t* x, float v[4]) {
+  uint2 a = *reinterpret_cast<const uint2*>(x);
+  v[0] = bf16lo(a.x); v[1] = bf16hi(a.x); v[2] = bf16lo(a.y); v[3] = bf16hi(a.y);
+}
+
+// Grid (ceil(E/EPB), ceil(T/TPB)).  Thread i of the CTA owns elements
+// [4i + 1024 m, 4i + 1024 m + 4) of the hidden axis; partial sums are reduced
+// across the warp by butterfly and across the 8 warps in warp order, so the
+// summation order is fixed for a given H.
+template <typename XT>
+__global__ void __launch_bounds__(kRouterThreads)
+router_logits_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T, int H, int E,
+                     float* __restrict__ z) {
+  __shared__ float part[kRouterThreads / 32][kRouterEPB][kRouterTPB];
+  const int e0 = blockIdx.x * kRouterEPB, t0 = blockIdx.y * kRouterTPB;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float acc[kRouterEPB][kRouterTPB];
+#pragma unroll
+  for (int i = 0; i < kRouterEPB; ++i)
+#pragma unroll
+    for (int t = 0; t < kRouterTPB; ++t) acc[i][t] = 0.f;
+  for (int hh = threadIdx.x * 4; hh < H; hh += kRouterThreads * 4) {
+    float wv[kRouterEPB][4];
+#pragma unroll
+    for (int i = 0; i < kRouterEPB; ++i) {
+      if (e0 + i < E) {
+        float4 a = *reinterpret_cast<const float4*>(w + (size_t)(e0 + i) * H + hh);
+        wv[i][0] = a.x; wv[i][1] = a.y; wv[i][2] = a.z; wv[i][3] = a.w;
+      } else {
+        wv[i][0] = wv[i][1] = wv[i][2] = wv[i][3] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kRouterTPB; ++t) {
+      if (t0 + t < T) {
+        float xv[4];
+        load_x4<XT>(x + (size_t)(t0 + t) * H + hh, xv);
+#pragma unroll
+        for (int i = 0; i < kRouterEPB; ++i)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[i][t] = fmaf(wv[i][c], xv[c], acc[i][t]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kRouterEPB; ++i)
+#pragma unroll
+    for (int t = 0; t < kRouterTPB; ++t) {
+      float v = warp_sum(acc[i][t]);
+      if (lane == 0) part[warp][i][t] = v;
+    }
+  __syncthreads();
+  if (threadIdx.x < kRouterEPB * kRouterTPB) {
+    int i = threadIdx.x / kRouterTPB, t = threadIdx.x % kRouterTPB;
+    if (e0 + i < E && t0 + t < T) {
+      float s = 0.f;
+      for (int wp = 0; wp < kRouterThreads / 32; ++wp) s += part[wp][i][t];
+      z[(size_t)(t0 + t) * E + e0 + i] = s;
+    }
+  }
+}
+
+// One warp per token.  Lane l holds logits e = l + 32 m.  Each of the k rounds
+// takes the warp-wide maximum (ties: lower index) among unselected experts.
+__global__ void topk_gates_kernel(const float* __restrict__ z, int T, int E, int k, int gating,
+                                  int* __restrict__ ids, float* __restrict__ gates) {
+  constexpr int kPer = 8;   // E <= 256
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  float v[kPer];
+  bool taken[kPer];
+#pragma unroll
+  for (int m = 0; m < kPer; ++m) {
+    int e = lane + 32 * m;
+    v[m] = e < E ? z[(size_t)warp * E + e] : 0.f;
+    taken[m] = !(e < E);
+  }
+  float zsel[16];
+  int isel[16];
+  for (int r = 0; r < k; ++r) {
+    float best = 0.f;
+    int bi = 0x7FFFFFFF;
+#pragma unroll
+    for (int m = 0; m < kPer; ++m) {
+      int e = lane + 32 * m;
+      if (!taken[m] && (bi == 0x7FFFFFFF || v[m] > best)) { best = v[m]; bi = e; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      float ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+      int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+      bool better = (oi != 0x7FFFFFFF) &&
+                    (bi == 0x7FFFFFFF || ob > best || (ob == best && oi < bi));
+      if (better) { best = ob; bi = oi; }
+    }
+    zsel[r] = best;
+    isel[r] = bi;
+#pragma unroll
+    for (int m = 0; m < kPer; ++m)
+      if (lane + 32 * m == bi) taken[m] = true;
+  }
+  if (lane == 0) {
+    float wsum = 0.f, wv[16];
+    for (int r = 0; r < k; ++r) {
+      float a = gating == 0 ? expf(zsel[r] - zsel[0]) : 1.0f / (1.0f + expf(-zsel[r]));
+      wv[r] = a;
+      wsum += a;
+    }
+    for (int r = 0; r < k; ++r) {
+      ids[(size_t)warp * k + r] = isel[r];
+      gates[(size_t)warp * k + r] = wv[r] / wsum;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router_logits(const void* x, bool x_bf16, const float* w_router, int T, int H,
+                                 int E, float* logits, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  dim3 grid((E + kRouterEPB - 1) / kRouterEPB, (T + kRouterTPB - 1) / kRouterTPB);
+  if (x_bf16)
+    router_logits_kernel<uint16_t><<<grid, kRouterThreads, 0, s>>>(
+        static_cast<const uint16_t*>(x), w_router, T, H, E, logits);
+  else
+    router_logits_kernel<float><<<grid, kRouterThreads, 0, s>>>(static_cast<const float*>(x),
+                                                               w_router, T, H, E, logits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_gates(const float* logits, int T, int E, int k, int gating, int* ids,
+                              float* gates, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  const int threads = 256, warps = threads / 32;
+  topk_gates_kernel<<<(T + warps - 1) / warps, threads, 0, s>>>(logits, T, E, k, gating, ids,
+                                                               gates);
+  return cudaGetLastError();
+}
+
+}  // namespace ftk

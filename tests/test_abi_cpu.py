@@ -1,0 +1,122 @@
+"""CPU checks of the C ABI: the library loads, exports every function the
+header declares, rejects bad arguments without a GPU, and its own slot table
+(run host-only through ft_cache_simulate) matches the oracle's LRU."""
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import moe_expert_offload_top_b200 as ft
+from oracle import lru as olru
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GOLD = os.path.join(ROOT, "tests", "golden")
+
+
+def _declared():
+    names = []
+    with open(os.path.join(ROOT, "include", "ftmoe.h")) as f:
+        for ln in f:
+            m = re.match(r"^FT_API\s+[\w\s\*]+?\b(ft_\w+)\(", ln)
+            if m:
+                names.append(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    decl = _declared()
+    assert len(decl) >= 20
+    out = subprocess.run(["nm", "-D", "--defined-only", ft.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    missing = [n for n in decl if n not in exported]
+    assert not missing, missing
+    assert set(decl) == set(ft.EXPORTED)
+    assert ft.ft_version().startswith("ftmoe")
+
+
+def test_library_is_built_for_sm100a_only():
+    out = subprocess.run(["cuobjdump", "--list-elf", ft.LIB_PATH], capture_output=True, text=True).stdout
+    arches = set(re.findall(r"sm_(\d+a?)", out))
+    assert arches == {"100a"}, arches
+
+
+def test_invalid_arguments_are_rejected_without_a_gpu():
+    with pytest.raises(ft.FtError):
+        ft.ft_moe_create(0, 1, 8, 8, "bf16", 1)
+    with pytest.raises(ft.FtError):
+        ft.ft_moe_create(300, 1, 8, 8, "bf16", 1)             # > FT_MAX_EXPERTS
+    with pytest.raises(ft.FtError):
+        ft.ft_moe_create(16, 2, 200, 128, "int4", 4)          # int4 needs multiples of 128
+    assert "invalid" in ft.ft_last_error(None) or "int4" in ft.ft_last_error(None)
+    with pytest.raises(ft.FtError):
+        ft.ft_router_topk(0, 1, 0, 1, 8, 300, 2, 0, 0, 0, 0)
+    with pytest.raises(ft.FtError):
+        ft.ft_cache_simulate(1, 4, 2, [7, 1])                 # unknown op
+
+
+def _golden_script():
+    ops, expect, cap0 = [], [], None
+    with open(os.path.join(GOLD, "lru_hand_4slot.txt")) as f:
+        for ln in f:
+            t = ln.split()
+            if not t or t[0].startswith("#"):
+                continue
+            if t[0] == "capacity":
+                cap0 = int(t[1])
+            elif t[0] == "step":
+                es = [int(v) for v in t[3:]]
+                ops += [0, int(t[1]), int(t[2]), 0, len(es)] + es
+            elif t[0] == "capacity_error":
+                es = [int(v) for v in t[3:]]
+                ops += [0, int(t[1]), int(t[2]), 0, len(es)] + es
+            elif t[0] == "resize":
+                ops += [1, int(t[1])]
+            elif t[0] in ("hit", "miss"):
+                expect.append((int(t[0] == "hit"),) + tuple(int(v) for v in t[1:]))
+            elif t[0] == "stats":
+                stats = tuple(int(v) for v in t[1:])
+    return cap0, ops, expect, stats
+
+
+def test_library_lru_matches_hand_worked_golden():
+    cap, ops, expect, stats = _golden_script()
+    trace, st, nerr = ft.ft_cache_simulate(2, 16, cap, ops)
+    assert nerr == 1
+    got = [(a[4], a[1], a[2], a[5], a[6], a[7]) for a in trace]
+    assert got == expect
+    assert (st["routed"], st["hits"], st["misses"], st["evictions"]) == stats
+
+
+@pytest.mark.parametrize("C,L,E,smax,resizes", [
+    (1, 1, 4, 1, ()), (4, 1, 16, 2, ()), (7, 3, 10, 5, (12, 5)), (20, 4, 32, 8, (40, 9, 33)),
+    (64, 2, 64, 40, (100, 64)), (204, 4, 128, 8, ()),
+])
+def test_library_lru_matches_oracle_on_random_scripts(C, L, E, smax, resizes):
+    rng = np.random.default_rng(C + 7 * E)
+    ref = olru.SharedLru(C)
+    ops = []
+    cap = C
+    todo = list(resizes)
+    n_steps = 600
+    for call in range(n_steps):
+        if todo and call % (n_steps // (len(resizes) + 1)) == 0 and call > 0:
+            cap = todo.pop(0)
+            ops += [1, cap]
+            ref.resize(cap)
+        l = call % L
+        kind = int(rng.random() < 0.2)
+        m = int(rng.integers(1, min(smax, cap) + 1))
+        es = sorted(rng.choice(E, m, replace=False).tolist())
+        ops += [0, call, l, kind, m] + es
+        ref.access_set(call, l, es, kind)
+    trace, st, nerr = ft.ft_cache_simulate(L, E, C, ops)
+    want = [(a.call, a.layer, a.expert, a.kind, int(a.hit), a.slot, a.ev_layer, a.ev_expert) for a in ref.trace]
+    assert nerr == 0
+    assert trace == want
+    s = ref.stats
+    assert (st["routed"], st["hits"], st["misses"], st["prefetch"], st["prefetch_hits"],
+            st["prefetch_misses"], st["evictions"]) == (s.routed, s.hits, s.misses, s.prefetch,
+                                                        s.prefetch_hits, s.prefetch_misses, s.evictions)
+    assert st["resident"] == len(ref.order) and st["capacity"] == cap
