@@ -168,6 +168,18 @@ FT_API int ft_moe_reserve(ft_moe* h, int max_tokens);
 FT_API int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const float* router_w,
                    void* out, void* stream);
 
+/* Waits for every forward and copy of the handle, then checks the device error word
+ * that the prefill GEMM kernels set when one of their bounded waits gives up
+ * (FT_ERR_DEVICE_CHECK; the word is cleared).  A forward also reports a word set by
+ * an earlier forward. */
+FT_API int ft_moe_sync(ft_moe* h);
+
+/* Expert FFN path: bf16 stacks with H % 256 == 0 and I % 128 == 0 use the tcgen05
+ * grouped GEMMs when n_tokens * k >= min_avg_pairs * |S| (on average at least
+ * min_avg_pairs tokens per selected expert; default 32), else the streaming GEMV.
+ * Both compute the same function.  0 always selects the GEMMs where shapes allow. */
+FT_API int ft_moe_set_gemm_threshold(ft_moe* h, int min_avg_pairs);
+
 /* Copies the routing of the last forward to host memory: ids [n_tokens][k] (expert
  * indices, by descending logit, ties to the lower index) and gates [n_tokens][k].
  * Either pointer may be NULL. */

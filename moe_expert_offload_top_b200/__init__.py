@@ -86,6 +86,8 @@ _SIGS = {
     "ft_combine": ([_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "ft_version": ([], ctypes.c_char_p),
     "ft_moe_set_stage_timing": ([_vp, _i], _i),
+    "ft_moe_sync": ([_vp], _i),
+    "ft_moe_set_gemm_threshold": ([_vp, _i], _i),
     "ft_moe_perf": ([_vp, ctypes.POINTER(ft_perf_t)], _i),
     "ft_moe_reset_perf": ([_vp], _i),
     "ft_cache_simulate": ([_i, _i, _i, _vp, _i, _vp, _i, ctypes.POINTER(_i),
@@ -218,6 +220,14 @@ def ft_cache_slot_ptr(h, slot):
 
 def ft_moe_set_timeout_ms(h, ms):
     return _check(h, _lib.ft_moe_set_timeout_ms(h, ms))
+
+
+def ft_moe_sync(h):
+    return _check(h, _lib.ft_moe_sync(h))
+
+
+def ft_moe_set_gemm_threshold(h, min_avg_pairs):
+    return _check(h, _lib.ft_moe_set_gemm_threshold(h, min_avg_pairs))
 
 
 def ft_moe_set_stage_timing(h, enabled):

@@ -88,6 +88,13 @@ struct ft_moe {
   float* d_h = nullptr;
   float* d_y = nullptr;
   int* h_ids = nullptr;
+  int* d_err = nullptr;           // device-side error word (bounded waits that gave up)
+  int* h_err = nullptr;
+  uint16_t* d_ax = nullptr;       // gathered token rows for the prefill GEMMs
+  ftk::GemmMaps maps;
+  bool maps_dirty = true;
+  int num_sms = 148;
+  int gemm_min_avg_pairs = 32;    // tcgen05 path when bf16 and T*k/|S| >= this
   cudaEvent_t route_ev = nullptr;
   int last_T = 0;
 
@@ -145,6 +152,9 @@ void free_scratch(ft_moe* h) {
   cudaFree(h->d_logits); cudaFree(h->d_ids); cudaFree(h->d_gates); cudaFree(h->d_counts);
   cudaFree(h->d_offsets); cudaFree(h->d_perm); cudaFree(h->d_inv); cudaFree(h->d_h);
   cudaFree(h->d_y);
+  cudaFree(h->d_ax);
+  h->d_ax = nullptr;
+  h->maps_dirty = true;
   if (h->h_ids) cudaFreeHost(h->h_ids);
   h->d_logits = nullptr; h->d_ids = nullptr; h->d_gates = nullptr; h->d_counts = nullptr;
   h->d_offsets = nullptr; h->d_perm = nullptr; h->d_inv = nullptr; h->d_h = nullptr;
@@ -167,7 +177,9 @@ int ensure_scratch(ft_moe* h, int T) {
             cudaMalloc(&h->d_inv, sizeof(int) * pairs) == cudaSuccess &&
             cudaMalloc(&h->d_h, sizeof(float) * rows * h->I) == cudaSuccess &&
             cudaMalloc(&h->d_y, sizeof(float) * rows * h->H) == cudaSuccess &&
-            cudaHostAlloc(&h->h_ids, sizeof(int) * pairs, cudaHostAllocDefault) == cudaSuccess;
+            cudaHostAlloc(&h->h_ids, sizeof(int) * pairs, cudaHostAllocDefault) == cudaSuccess &&
+            (h->wdtype != FT_W_BF16 ||
+             cudaMalloc(&h->d_ax, sizeof(uint16_t) * rows * h->H) == cudaSuccess);
   if (!ok) {
     cudaGetLastError();
     free_scratch(h);
@@ -263,6 +275,30 @@ int issue_fills(ft_moe* h, std::vector<ftc::Access>& recs, size_t first) {
   FT_CUDA(h, cudaEventRecord(h->fill_ev[r], h->copy));
   h->fill_ev_batch[r] = b;
   for (int s : slots) h->slot_fill_batch[s] = b;
+  return FT_OK;
+}
+
+bool gemm_shapes_ok(const ft_moe* h) {
+  return h->wdtype == FT_W_BF16 && h->H % 256 == 0 && h->I % 128 == 0;
+}
+
+int ensure_maps(ft_moe* h) {
+  if (!h->maps_dirty) return FT_OK;
+  const uint64_t rows = (uint64_t)h->cap_tokens * (h->k + 1);
+  const uint64_t H = h->H, I = h->I;
+  bool ok = ftk::encode_map_2d(&h->maps.a_x, h->d_ax, H, rows, H * 2, 128) &&
+            ftk::encode_map_2d(&h->maps.a_h, h->d_h, I, rows, I * 2, 128) &&
+            ftk::encode_map_3d(&h->maps.b1_routed, h->arena, H, 2 * I, h->C, H * 2, h->blob, 128) &&
+            ftk::encode_map_3d(&h->maps.b2_routed, h->arena + 2 * I * H * 2, I, H, h->C, I * 2, h->blob, 256);
+  if (ok && h->shared) {
+    ok = ftk::encode_map_3d(&h->maps.b1_shared, h->shared, H, 2 * I, h->L, H * 2, h->blob, 128) &&
+         ftk::encode_map_3d(&h->maps.b2_shared, h->shared + 2 * I * H * 2, I, H, h->L, I * 2, h->blob, 256);
+  } else {
+    h->maps.b1_shared = h->maps.b1_routed;
+    h->maps.b2_shared = h->maps.b2_routed;
+  }
+  if (!ok) return fail(h, FT_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  h->maps_dirty = false;
   return FT_OK;
 }
 
@@ -370,6 +406,11 @@ ft_moe* ft_moe_create(int num_experts, int top_k, int hidden, int inter, int wdt
     h->fill_ev_batch[i] = -1;
   }
   cudaEventCreateWithFlags(&h->route_ev, cudaEventDisableTiming);
+  cudaMalloc(&h->d_err, sizeof(int));
+  cudaMemset(h->d_err, 0, sizeof(int));
+  cudaHostAlloc(&h->h_err, sizeof(int), cudaHostAllocDefault);
+  if (h->h_err) *h->h_err = 0;
+  cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
   reset_cache_state(h);
   if (cudaGetLastError() != cudaSuccess) {
     g_create_error = "ft_moe_create: CUDA setup failed";
@@ -395,6 +436,7 @@ int ft_moe_set_layers(ft_moe* h, int num_layers, int gating, int has_shared_expe
     cudaFree(h->shared);
     h->shared = nullptr;
   }
+  h->maps_dirty = true;
   h->L = num_layers;
   h->gating = gating;
   h->has_shared = has_shared_expert ? 1 : 0;
@@ -470,11 +512,15 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   if (h->stage_pending.size() > 256) harvest_stages(h, false);
   StageEvents* se = stage_begin(h);
   stage_mark(se, SE_R0, s);
-  FT_CUDA(h, ftk::launch_router_logits(x, xbf16, router_w, T, h->H, E, h->d_logits, s));
+  if (T > 64)
+    FT_CUDA(h, ftk::launch_router_logits_tiled(x, xbf16, router_w, T, h->H, E, h->d_logits, s));
+  else
+    FT_CUDA(h, ftk::launch_router_logits(x, xbf16, router_w, T, h->H, E, h->d_logits, s));
   FT_CUDA(h, ftk::launch_topk_gates(h->d_logits, T, E, k, h->gating, h->d_ids, h->d_gates, s));
   stage_mark(se, SE_R1, s);
   FT_CUDA(h, cudaMemcpyAsync(h->h_ids, h->d_ids, sizeof(int) * (size_t)T * k,
                              cudaMemcpyDeviceToHost, s));
+  FT_CUDA(h, cudaMemcpyAsync(h->h_err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost, s));
   FT_CUDA(h, cudaEventRecord(h->route_ev, s));
   stage_mark(se, SE_P0, s);
   FT_CUDA(h, ftk::launch_permute(h->d_ids, T, k, E, h->d_counts, h->d_offsets, h->d_perm,
@@ -490,6 +536,13 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   }
   if (rc) return rc;
   h->last_T = T;
+  if (*h->h_err) {
+    const int code = *h->h_err;
+    *h->h_err = 0;
+    cudaMemsetAsync(h->d_err, 0, sizeof(int), s);
+    return fail(h, FT_ERR_DEVICE_CHECK,
+                "a previous forward's kernel gave up waiting (code " + std::to_string(code) + ")");
+  }
 
   // distinct selected experts, ascending, and the largest token count of one expert
   std::vector<int> cnt(E, 0);
@@ -557,9 +610,34 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
     se->d_bytes = list.n * wmat + pairs * (h->I * 4.0 + h->H * 4.0);
     se->flops = pairs * 6.0 * mat;
   }
-  stage_mark(se, SE_G0, s);
-  FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, list, max_pairs, h->d_offsets,
-                                    h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr));
+  const bool use_gemm = gemm_shapes_ok(h) && (long long)T * k >= (long long)h->gemm_min_avg_pairs * (long long)S.size();
+  if (use_gemm) {
+    rc = ensure_maps(h);
+    if (rc) return rc;
+    ftk::GemmGroups groups;
+    groups.n = list.n;
+    for (int i = 0; i < list.n; ++i) {
+      groups.expert[i] = list.expert[i];
+      groups.z[i] = list.expert[i] >= 0 ? h->lru.slot_of(layer * E + list.expert[i]) : layer;
+    }
+    FT_CUDA(h, ftk::launch_gather_rows(x, h->d_perm, T, k, h->H, h->has_shared != 0, h->d_ax, s));
+    h->perf.kernel_launches += 1;
+    stage_mark(se, SE_G0, s);
+    FT_CUDA(h, ftk::launch_grouped_gemm(0, h->maps, groups, h->d_offsets, T, k, h->I, h->H, h->d_h,
+                                        h->d_err, h->num_sms, s));
+    stage_mark(se, SE_G1, s);
+    FT_CUDA(h, ftk::launch_grouped_gemm(1, h->maps, groups, h->d_offsets, T, k, h->I, h->H, h->d_y,
+                                        h->d_err, h->num_sms, s));
+    if (se) {   // bf16 h, and the weights of each listed expert read once
+      const double pairs = (double)T * k + (h->has_shared ? T : 0);
+      se->gu_bytes = list.n * 2.0 * h->H * h->I * 2 + pairs * (h->H * 2.0 + h->I * 2.0);
+      se->d_bytes = list.n * 1.0 * h->H * h->I * 2 + pairs * (h->I * 2.0 + h->H * 4.0);
+    }
+  } else {
+    stage_mark(se, SE_G0, s);
+    FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, list, max_pairs, h->d_offsets,
+                                      h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr));
+  }
   stage_mark(se, SE_D1, s);
   FT_CUDA(h, ftk::launch_combine(h->d_y, h->d_gates, h->d_inv, T, h->H, k, h->has_shared != 0,
                                  xbf16, out, s));
@@ -582,6 +660,25 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
     account(h, recs, first_pre);
     if (rc) return rc;
   }
+  return FT_OK;
+}
+
+int ft_moe_sync(ft_moe* h) {
+  if (!h) return FT_ERR_INVALID;
+  FT_CUDA(h, cudaStreamSynchronize(h->copy));
+  if (h->has_last_stream) FT_CUDA(h, cudaStreamSynchronize(h->last_stream));
+  int code = 0;
+  FT_CUDA(h, cudaMemcpy(&code, h->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (code) {
+    cudaMemset(h->d_err, 0, sizeof(int));
+    return fail(h, FT_ERR_DEVICE_CHECK, "a kernel gave up waiting (code " + std::to_string(code) + ")");
+  }
+  return FT_OK;
+}
+
+int ft_moe_set_gemm_threshold(ft_moe* h, int min_avg_pairs) {
+  if (!h || min_avg_pairs < 0) return FT_ERR_INVALID;
+  h->gemm_min_avg_pairs = min_avg_pairs;
   return FT_OK;
 }
 
@@ -658,6 +755,7 @@ int ft_cache_resize(ft_moe* h, int slots) {
   cudaFree(h->arena);
   h->arena = na;
   h->C = slots;
+  h->maps_dirty = true;
   h->st.evictions += (long long)evicted.size();
   h->slot_last_use.assign(slots, -1);
   h->slot_fill_batch.assign(slots, -1);
@@ -732,6 +830,8 @@ void ft_moe_destroy(ft_moe* h) {
   for (auto& se : h->stage_free)
     for (int i = 0; i < SE_N; ++i) cudaEventDestroy(se.ev[i]);
   free_scratch(h);
+  cudaFree(h->d_err);
+  if (h->h_err) cudaFreeHost(h->h_err);
   if (h->copy) cudaStreamDestroy(h->copy);
   cudaFree(h->arena);
   cudaFree(h->shared);

@@ -1,6 +1,8 @@
 // Internal launch functions of the sm_100a kernels (host side).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 namespace ftk {
@@ -36,5 +38,41 @@ cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdt
 // K5: out[t] = sum_j gates[t][j] * y[inv[t*k+j]] (ascending j) + y[T*k+t] if has_shared.
 cudaError_t launch_combine(const float* y, const float* gates, const int* inv, int T, int H, int k,
                            bool has_shared, bool out_bf16, void* out, cudaStream_t s);
+
+// K4 (prefill): groups of the grouped GEMM.  Group g = routed expert expert[g] (rows
+// offsets[e] .. offsets[e+1] of the gathered A) whose weights are slot z[g] of the
+// arena, or the shared expert (expert[g] = -1, rows T*k .. T*k+T-1, layer z[g] of the
+// shared-expert area).
+struct GemmGroups {
+  int n;
+  int expert[kMaxList];
+  int z[kMaxList];
+};
+
+// TMA descriptors of the prefill GEMMs (encoded on the host when buffers move).
+struct GemmMaps {
+  CUtensorMap a_x;        // gathered token rows  [rows][H] bf16, box 64 x 128
+  CUtensorMap a_h;        // SwiGLU output h      [rows][I] bf16, box 64 x 128
+  CUtensorMap b1_routed;  // gate|up rows of slots [C][2I][H], box 64 x 128 x 1
+  CUtensorMap b1_shared;  // gate|up rows of shared experts [L][2I][H]
+  CUtensorMap b2_routed;  // down rows of slots [C][H][I], box 64 x 256 x 1
+  CUtensorMap b2_shared;  // down rows of shared experts [L][H][I]
+};
+
+size_t gemm_smem_bytes();
+// A[q] = x[perm[q] / k] for q < T*k; A[T*k + t] = x[t] when with_shared (bf16 rows of H).
+cudaError_t launch_gather_rows(const void* x, const int* perm, int T, int k, int H, bool with_shared,
+                               void* A, cudaStream_t s);
+// mode 0: h = silu(A W_gate^T) * (A W_up^T) (bf16 [rows][I]); mode 1: y = h W_down^T (f32 [rows][H]).
+cudaError_t launch_grouped_gemm(int mode, const GemmMaps& maps, const GemmGroups& groups, const int* offsets,
+                                int T, int k, int I, int H, void* out, int* err, int num_sms, cudaStream_t s);
+// 2-D / 3-D bf16 tensor maps with 128-byte swizzle (box inner extent 64 elements).
+bool encode_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+                   uint32_t box_rows);
+bool encode_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                   uint64_t row_bytes, uint64_t depth_bytes, uint32_t box_rows);
+// Router logits for many tokens: tiled SIMT fp32 GEMM (64 tokens x 64 experts per CTA).
+cudaError_t launch_router_logits_tiled(const void* x, bool x_bf16, const float* w_router, int T, int H,
+                                       int E, float* logits, cudaStream_t s);
 
 }  // namespace ftk

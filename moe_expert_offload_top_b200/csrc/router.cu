@@ -139,7 +139,68 @@ __global__ void topk_gates_kernel(const float* __restrict__ z, int T, int E, int
   }
 }
 
+// Many tokens: CTA tile of 64 tokens x 64 experts, K step 16 through shared
+// memory, 256 threads each owning a 4 x 4 block of logits (fp32 FMAs in a fixed
+// order along H).
+constexpr int RT = 64, RE = 64, RK = 16;
+template <typename XT>
+__global__ void __launch_bounds__(256)
+router_logits_tiled_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T, int H, int E,
+                           float* __restrict__ z) {
+  __shared__ float xs[RK][RT + 4];
+  __shared__ float ws[RK][RE + 4];
+  const int t0 = blockIdx.x * RT, e0 = blockIdx.y * RE;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;   // 16 x 16 threads
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < H; k0 += RK) {
+    // 64 x 16 of x and of w: 1024 elements each, 4 per thread
+    for (int i = threadIdx.x; i < RT * RK; i += 256) {
+      const int r = i / RK, c = i % RK;
+      float xv = 0.f, wv = 0.f;
+      if (t0 + r < T && k0 + c < H) {
+        if constexpr (sizeof(XT) == 2) xv = bf16_to_f32(x[(size_t)(t0 + r) * H + k0 + c]);
+        else xv = x[(size_t)(t0 + r) * H + k0 + c];
+      }
+      if (e0 + r < E && k0 + c < H) wv = w[(size_t)(e0 + r) * H + k0 + c];
+      xs[c][r] = xv;
+      ws[c][r] = wv;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int c = 0; c < RK; ++c) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { a[i] = xs[c][ty * 4 + i]; b[i] = ws[c][tx * 4 + i]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = t0 + ty * 4 + i, e = e0 + tx * 4 + j;
+      if (t < T && e < E) z[(size_t)t * E + e] = acc[i][j];
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_router_logits_tiled(const void* x, bool x_bf16, const float* w_router, int T, int H,
+                                       int E, float* logits, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  dim3 grid((T + RT - 1) / RT, (E + RE - 1) / RE);
+  if (x_bf16)
+    router_logits_tiled_kernel<uint16_t><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), w_router, T, H,
+                                                              E, logits);
+  else
+    router_logits_tiled_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(x), w_router, T, H, E,
+                                                           logits);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_router_logits(const void* x, bool x_bf16, const float* w_router, int T, int H,
                                  int E, float* logits, cudaStream_t s) {

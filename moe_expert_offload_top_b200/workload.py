@@ -29,6 +29,8 @@ class GpuStack:
     def __init__(self, cfg, capacity=None, device="cuda", fill_threads=None, max_tokens=None):
         self.cfg = cfg
         self.device = torch.device(device)
+        if self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
         torch.cuda.set_device(self.device)
         self.C = cfg.C if capacity is None else capacity
         self.h = ft_moe_create(cfg.E, cfg.k, cfg.H, cfg.I, cfg.wdtype, self.C)
