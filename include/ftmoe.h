@@ -308,6 +308,37 @@ FT_API int ft_expert_ffn_decode(const void* x, int T, int H, int I, int top_k, i
 FT_API int ft_combine(const float* y, const float* gates, const int* inv, int T, int H, int top_k,
                int has_shared, int out_is_bf16, void* out, void* stream);
 
+/* Size, in floats, of the static device scratch of ft_expert_ffn_decode_noalloc
+ * (12 MiB).  Every GPU that loads this library holds it until the process exits. */
+#define FT_NOALLOC_SCRATCH_FLOATS (3u * 1024u * 1024u)
+
+/* The decode expert FFN followed by the gate-weighted combine, allocating nothing.
+ * No FreeToken page has a counterpart of this call: it exists for callers that may not
+ * allocate device memory while they run, such as a serving engine that fixes its whole
+ * device-memory plan at start-up and owns every byte after that, or a caller on a
+ * latency-critical decode loop that cannot pay cudaMalloc's implicit device
+ * synchronisation.  Such callers still pass every input and output buffer; only the
+ * intermediate rows that ft_expert_ffn_decode takes as caller buffers (h, y) move into a
+ * file-scope static device array of FT_NOALLOC_SCRATCH_FLOATS floats.
+ * Computes out[t] = sum_j gates[t][j] * y[inv[t*k+j]] (+ the shared expert's y with
+ * weight 1 when has_shared), with h and y as defined for ft_expert_ffn_decode;
+ * arguments as for ft_expert_ffn_decode and ft_combine (out: [T][H], f32 for FT_W_F32,
+ * else bf16).
+ *  - Limit: (T*k + T) * (I + H) <= FT_NOALLOC_SCRATCH_FLOATS; larger sizes return
+ *    FT_ERR_INVALID before any launch, with the reason in ft_last_error(NULL).
+ *  - Calls no cudaMalloc, cudaFree or other allocating routine.  The first call on a
+ *    device looks up the array's device address (cudaGetSymbolAddress, with that device
+ *    current) and caches it; make that first call before any stream capture.
+ *  - Every call on a device uses the same array, which keeps the last call's contents
+ *    (nothing in it needs to start at zero: each call writes every row it reads).  Calls
+ *    whose kernels overlap on the GPU (other streams, other threads) race on it: order
+ *    them on one stream. */
+FT_API int ft_expert_ffn_decode_noalloc(const void* x, int T, int H, int I, int top_k, int wdtype,
+                                        const void* const* blobs, const int* experts, int n_list,
+                                        int max_pairs_per_expert, const int* offsets, const int* perm,
+                                        const float* gates, const int* inv, int has_shared, void* out,
+                                        void* stream);
+
 /* Version string of the library build. */
 FT_API const char* ft_version(void);
 

@@ -84,6 +84,8 @@ _SIGS = {
     "ft_permute": ([_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp], _i),
     "ft_expert_ffn_decode": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp], _i),
     "ft_combine": ([_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp], _i),
+    "ft_expert_ffn_decode_noalloc": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _i,
+                                      _vp, _vp], _i),
     "ft_version": ([], ctypes.c_char_p),
     "ft_moe_set_stage_timing": ([_vp, _i], _i),
     "ft_moe_sync": ([_vp], _i),
@@ -295,6 +297,21 @@ def ft_cache_simulate(num_layers, num_experts, capacity, ops):
                                         ctypes.byref(st), ctypes.byref(nerr)))
     trace = [tuple(getattr(buf[i], f) for f, _ in ft_access_t._fields_) for i in range(n.value)]
     return trace, st.as_dict(), nerr.value
+
+
+FT_NOALLOC_SCRATCH_FLOATS = 3 * 1024 * 1024
+
+
+def ft_expert_ffn_decode_noalloc(x, T, H, I, top_k, wdtype, blobs, experts, max_pairs_per_expert, offsets,
+                                 perm, gates, inv, has_shared, out, stream=None):
+    """Decode FFN + combine with the library's static device scratch (no allocation)."""
+    n = len(experts)
+    bl = (ctypes.c_void_p * max(n, 1))(*[_p(b) for b in blobs])
+    ex = _int_array(list(experts) or [0])
+    return _check(None, _lib.ft_expert_ffn_decode_noalloc(
+        _p(x), T, H, I, top_k, WDTYPE.get(wdtype, wdtype), ctypes.cast(bl, ctypes.c_void_p),
+        ctypes.cast(ex, ctypes.c_void_p), n, max_pairs_per_expert, _p(offsets), _p(perm), _p(gates), _p(inv),
+        int(has_shared), _p(out), _s(stream)))
 
 
 def ft_version():

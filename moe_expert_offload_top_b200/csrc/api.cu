@@ -33,6 +33,15 @@
 namespace {
 
 thread_local std::string g_create_error;
+
+}  // namespace
+
+namespace ftk {
+// Message for ft_last_error(NULL) from a step-level entry point.
+void set_step_error(const std::string& msg) { g_create_error = msg; }
+}  // namespace ftk
+
+namespace {
 constexpr int kRing = 128;
 
 struct FillTiming {
