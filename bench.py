@@ -224,6 +224,80 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------ prefill leg --
+
+def run_prefill_leg(args, dev):
+    """Prefill of the DeepSeek-V4-Flash-shaped stack (8 layers, 256 experts, top-6
+    sigmoid + shared expert, bf16): N(0,1) tokens through every layer in prefill
+    mode.  Two caches: 512 slots (25%%, whole-layer double buffering over PCIe) and
+    every expert resident (2048 slots), which isolates the tcgen05 grouped GEMMs."""
+    import dataclasses
+
+    import torch
+
+    import moe_expert_offload_top_b200 as ft
+    from moe_expert_offload_top_b200.workload import GpuStack
+
+    base = synth.CONFIGS[4]
+    T = args.prefill_tokens or base.tokens
+    cfg = dataclasses.replace(base, tokens=T, batches=(T,))
+    stack = GpuStack(cfg, device=dev, max_tokens=T)
+    vals, x = stack.tokens(T)
+    out = torch.empty((cfg.L, T, cfg.H), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except Exception:
+        pass
+    res = {"workload": "%s: %d layers, E=%d, H=%d, I=%d, top-%d %s + shared expert, bf16, %d tokens, prefill"
+                       % (cfg.name, cfg.L, cfg.E, cfg.H, cfg.I, cfg.k, cfg.gating, T)}
+    for label, slots, passes in (("offload", base.C, args.prefill_passes), ("resident", cfg.L * cfg.E,
+                                                                             args.prefill_passes)):
+        if slots != stack.C:
+            stack.resize(slots)
+        stack.step(x[0], out, stream)                       # warm-up pass
+        ft.ft_moe_sync(stack.h)
+        stack.reset_stats()
+        ft.ft_moe_reset_perf(stack.h)
+        ft.ft_moe_set_stage_timing(stack.h, 1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(passes):
+            stack.step(x[0], out, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ft.ft_moe_sync(stack.h)
+        dt = e0.elapsed_time(e1) * 1e-3
+        perf = ft.ft_moe_perf(stack.h)
+        ft.ft_moe_set_stage_timing(stack.h, 0)
+        st = stack.stats()
+        gemm_s = (perf["ffn_gate_up_ms"] + perf["ffn_down_ms"]) * 1e-3
+        tf = perf["ffn_flops"] / gemm_s / 1e12 if gemm_s > 0 else None
+        gbs = (perf["ffn_gate_up_bytes"] + perf["ffn_down_bytes"]) / gemm_s / 1e9 if gemm_s > 0 else None
+        res[label] = {
+            "cache_slots": slots, "passes": passes, "tokens_per_s": T * passes / dt,
+            "ms_per_layer": 1e3 * dt / (passes * cfg.L),
+            "routed_misses": st["misses"], "prefetch_misses": st["prefetch_misses"],
+            "h2d_gbs": st["h2d_bytes"] / st["h2d_seconds"] / 1e9 if st["h2d_seconds"] > 0 else None,
+            "grouped_gemm": {
+                "kernel": "grouped_gemm_kernel<0>+<1> (tcgen05 kind::f16, TMEM, TMA)",
+                "ms_per_layer": 1e3 * gemm_s / max(perf["timed_forwards"], 1),
+                "tflops": tf, "gbs": gbs,
+                "tensor_frac_of_dense_peak": tf / peaks["bf16_tflops_sustained"] if tf and "bf16_tflops_sustained" in peaks else None,
+                "hbm_frac": gbs / peaks["hbm_gbs"] if gbs and "hbm_gbs" in peaks else None,
+                "intensity_flop_per_byte": perf["ffn_flops"] / (perf["ffn_gate_up_bytes"] + perf["ffn_down_bytes"])
+                if perf["ffn_gate_up_bytes"] > 0 else None,
+            },
+            "stages_ms_per_layer": {k2: perf[k2 + "_ms"] / max(perf["timed_forwards"], 1) for k2 in
+                                    ("router", "permute", "ffn_gate_up", "ffn_down", "combine")},
+        }
+    stack.close()
+    return res
+
+
 # ----------------------------------------------------------------- our arm --
 
 def run_ours(args):
@@ -243,6 +317,7 @@ def run_ours(args):
     out = torch.empty((cfg.L, 1, cfg.H), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    link_h2d, link_d2h = ft.ft_probe_host_link(256 << 20, 5)
     for s in range(W):
         stack.step(x_dev[s], out, stream)
     torch.cuda.synchronize(dev)
@@ -317,11 +392,16 @@ def run_ours(args):
             "clocks": clk,
             "cache": {"miss_rate": st["misses"] / max(st["routed"], 1), "routed": st["routed"],
                       "misses": st["misses"], "h2d_bytes": st["h2d_bytes"],
-                      "h2d_gbs": st["h2d_bytes"] / st["h2d_seconds"] / 1e9 if st["h2d_seconds"] > 0 else None},
+                      "h2d_gbs": st["h2d_bytes"] / st["h2d_seconds"] / 1e9 if st["h2d_seconds"] > 0 else None,
+                      "link_h2d_gbs_measured": link_h2d, "link_d2h_gbs_measured": link_d2h,
+                      "h2d_frac_of_link": (st["h2d_bytes"] / st["h2d_seconds"] / 1e9) / link_h2d
+                      if st["h2d_seconds"] > 0 and link_h2d else None},
             "stages_us_per_forward": {k2: 1e3 * perf[k2 + "_ms"] / gu_launches for k2 in
                                       ("router", "permute", "ffn_gate_up", "ffn_down", "combine")},
             "host_wait_us_per_forward": 1e3 * perf["host_wait_ms"] / max(perf["forwards"], 1),
         }
+        if world == 1 and args.prefill:
+            line["prefill"] = run_prefill_leg(args, dev)
         if world == 1 and not args.no_cpu_baseline:
             rate, n, cores, cdt = cpu_oracle_rate(cfg, vals[W:W + K], budget_s=args.cpu_budget_s,
                                                   blob_of=stack.pool_blob)
@@ -345,6 +425,10 @@ def main(argv=None):
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--reference-budget-s", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill", action="store_true",
+                    help="add the prefill leg (N=1 only; pins a 103 GB host pool)")
+    ap.add_argument("--prefill-tokens", type=int, default=None)
+    ap.add_argument("--prefill-passes", type=int, default=2)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -180,6 +180,37 @@ FT_API int ft_moe_sync(ft_moe* h);
  * Both compute the same function.  0 always selects the GEMMs where shapes allow. */
 FT_API int ft_moe_set_gemm_threshold(ft_moe* h, int min_avg_pairs);
 
+/* Routing launch shape for calls of up to 64 tokens: 1 (default) = one fused kernel
+ * (ft_route_decode), 0 = router, top-k and permutation as three launches.  Same results. */
+FT_API int ft_moe_set_fused_routing(ft_moe* h, int enabled);
+
+/* Decode GEMV kernel (process-wide; same results, different speed):
+ *   FT_DECODE_GEMV_REGISTER (default): 16-byte loads straight to registers, one CTA per
+ *     block of rows.
+ *   FT_DECODE_GEMV_BULK: weights streamed into shared memory by bulk copies, one
+ *     persistent CTA per SM, packed int4 dequant; used for up to 8 tokens per expert when
+ *     rows allow it (bf16/f32: H, I multiples of 8; int4: multiples of 1024), else the
+ *     register kernel. */
+enum ft_decode_gemv { FT_DECODE_GEMV_BULK = 0, FT_DECODE_GEMV_REGISTER = 1 };
+FT_API int ft_set_decode_gemv(int mode);
+
+/* Host-side fault injection for tests of failure handling (no GPU fault is made).
+ *   FT_INJECT_COPY_FAIL: the countdown-th slot fill from now is reported failed instead
+ *     of being issued.  The forward returns FT_ERR_CUDA before launching its FFN; the
+ *     entries of that fill and of the later fills of the same set become not resident
+ *     (their accesses stay in the trace).  The next forward works normally.
+ *   FT_INJECT_ROUTE_TIMEOUT: the countdown-th routing wait reports FT_ERR_TIMEOUT (after
+ *     the GPU work completes); the cache is unchanged.
+ * countdown 0 disarms. */
+enum ft_inject { FT_INJECT_COPY_FAIL = 1, FT_INJECT_ROUTE_TIMEOUT = 2 };
+FT_API int ft_moe_debug_inject(ft_moe* h, int what, int countdown);
+
+/* Runs one CTA that waits, with the same bounded wait the prefill GEMM kernels use, on a
+ * barrier that nothing arrives on, for limit_us microseconds (1..1e6).  The wait gives up,
+ * records the failure in an error word, and the kernel returns: FT_ERR_DEVICE_CHECK is the
+ * expected result, and the context stays usable.  Allocates 4 bytes stream-ordered. */
+FT_API int ft_debug_device_wait_selftest(int limit_us, void* stream);
+
 /* Copies the routing of the last forward to host memory: ids [n_tokens][k] (expert
  * indices, by descending logit, ties to the lower index) and gates [n_tokens][k].
  * Either pointer may be NULL. */
@@ -260,6 +291,27 @@ FT_API int ft_cache_simulate(int num_layers, int num_experts, int capacity, cons
                              int n_ops_ints, ft_access_t* trace, int trace_cap, int* n_trace,
                              ft_cache_stats_t* stats, int* n_capacity_errors);
 
+/* The same replay under another placement policy, to compare the shared LRU with the
+ * static layer split the pages contrast it with ("FreeToken linux", performance: at
+ * one RTX 5090 capacity the LRU missed 16% of expert reads where a static split missed
+ * 62%; "this tool runs datacenter AI on your PC": static placement vs dynamic caching).
+ *   FT_POLICY_LRU:    ft_cache_simulate.
+ *   FT_POLICY_STATIC: the first `capacity` keys in (layer, expert) order stay resident for
+ *                     good (slot = key); every other access is a miss that is served
+ *                     without being cached (slot -1, nothing evicted).  A resize changes
+ *                     which keys are resident.
+ * Arguments and script format as for ft_cache_simulate. */
+enum ft_policy { FT_POLICY_LRU = 0, FT_POLICY_STATIC = 1 };
+FT_API int ft_cache_simulate_policy(int policy, int num_layers, int num_experts, int capacity,
+                                    const int* ops, int n_ops_ints, ft_access_t* trace, int trace_cap,
+                                    int* n_trace, ft_cache_stats_t* stats, int* n_capacity_errors);
+
+/* Measures the host link the slot fills use ("FreeToken linux", setup: measure the
+ * pinned-memory PCIe bandwidth on the machine rather than trusting the specification):
+ * `iters` copies of `bytes` between pinned host memory and the current device, each way,
+ * timed with CUDA events on a private stream.  Allocates and frees its own buffers. */
+FT_API int ft_probe_host_link(size_t bytes, int iters, double* h2d_gbs, double* d2h_gbs);
+
 /* ------------------------------------------------------------------------ *
  * Step-level kernels.  Each runs one step of the forward on caller-owned device
  * buffers, on `stream`, without the cache.  They are the same kernels the
@@ -275,6 +327,14 @@ FT_API int ft_cache_simulate(int num_layers, int num_experts, int capacity, cons
  *   (written), ids: [T][k] int32, gates: [T][k] f32. */
 FT_API int ft_router_topk(const void* x, int x_is_bf16, const float* router_w, int T, int H, int E,
                    int top_k, int gating, float* logits, int* ids, float* gates, void* stream);
+
+/* Router + gating + token permutation in one launch, for decode-sized batches (T <= 64):
+ * the results of ft_router_topk followed by ft_permute (with inv), bit for bit the same
+ * selection and order.  ticket: a device int that is 0 before the first call; every call
+ * leaves it 0 again (one ticket per stream of calls). */
+FT_API int ft_route_decode(const void* x, int x_is_bf16, const float* router_w, int T, int H, int E,
+                           int top_k, int gating, float* logits, int* ids, float* gates, int* counts,
+                           int* offsets, int* perm, int* inv, int* ticket, void* stream);
 
 /* Token permutation by expert.  counts[e] = pairs routed to e; offsets = exclusive
  * prefix sum (E+1 entries); perm[q] = flat pair index t*k + j for q in expert-major

@@ -25,6 +25,9 @@ FT_OK, FT_ERR_INVALID, FT_ERR_OOM, FT_ERR_CUDA, FT_ERR_CAPACITY, FT_ERR_BUSY, FT
 FT_W_F32, FT_W_BF16, FT_W_INT4_G128 = 0, 1, 2
 FT_GATE_SOFTMAX, FT_GATE_SIGMOID = 0, 1
 FT_ROUTED, FT_PREFETCH = 0, 1
+FT_INJECT_COPY_FAIL, FT_INJECT_ROUTE_TIMEOUT = 1, 2
+FT_POLICY_LRU, FT_POLICY_STATIC = 0, 1
+FT_DECODE_GEMV_BULK, FT_DECODE_GEMV_REGISTER = 0, 1
 FT_MAX_EXPERTS, FT_MAX_TOPK = 256, 16
 WDTYPE = {"f32": FT_W_F32, "bf16": FT_W_BF16, "int4": FT_W_INT4_G128}
 GATING = {"softmax": FT_GATE_SOFTMAX, "sigmoid": FT_GATE_SIGMOID}
@@ -82,6 +85,7 @@ _SIGS = {
     "ft_moe_destroy": ([_vp], None),
     "ft_router_topk": ([_vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp], _i),
     "ft_permute": ([_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp], _i),
+    "ft_route_decode": ([_vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
     "ft_expert_ffn_decode": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp], _i),
     "ft_combine": ([_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "ft_expert_ffn_decode_noalloc": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _i,
@@ -90,8 +94,15 @@ _SIGS = {
     "ft_moe_set_stage_timing": ([_vp, _i], _i),
     "ft_moe_sync": ([_vp], _i),
     "ft_moe_set_gemm_threshold": ([_vp, _i], _i),
+    "ft_moe_debug_inject": ([_vp, _i, _i], _i),
+    "ft_set_decode_gemv": ([_i], _i),
+    "ft_moe_set_fused_routing": ([_vp, _i], _i),
+    "ft_debug_device_wait_selftest": ([_i, _vp], _i),
     "ft_moe_perf": ([_vp, ctypes.POINTER(ft_perf_t)], _i),
     "ft_moe_reset_perf": ([_vp], _i),
+    "ft_cache_simulate_policy": ([_i, _i, _i, _i, _vp, _i, _vp, _i, ctypes.POINTER(_i),
+                                  ctypes.POINTER(ft_cache_stats_t), ctypes.POINTER(_i)], _i),
+    "ft_probe_host_link": ([_sz, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)], _i),
     "ft_cache_simulate": ([_i, _i, _i, _vp, _i, _vp, _i, ctypes.POINTER(_i),
                            ctypes.POINTER(ft_cache_stats_t), ctypes.POINTER(_i)], _i),
 }
@@ -232,6 +243,23 @@ def ft_moe_set_gemm_threshold(h, min_avg_pairs):
     return _check(h, _lib.ft_moe_set_gemm_threshold(h, min_avg_pairs))
 
 
+def ft_moe_set_fused_routing(h, enabled):
+    return _check(h, _lib.ft_moe_set_fused_routing(h, int(enabled)))
+
+
+def ft_set_decode_gemv(mode):
+    return _check(None, _lib.ft_set_decode_gemv(mode))
+
+
+def ft_moe_debug_inject(h, what, countdown):
+    return _check(h, _lib.ft_moe_debug_inject(h, what, countdown))
+
+
+def ft_debug_device_wait_selftest(limit_us, stream=None):
+    """Returns the status code (FT_ERR_DEVICE_CHECK expected) without raising."""
+    return _lib.ft_debug_device_wait_selftest(limit_us, _s(stream))
+
+
 def ft_moe_set_stage_timing(h, enabled):
     return _check(h, _lib.ft_moe_set_stage_timing(h, int(enabled)))
 
@@ -260,6 +288,13 @@ def ft_router_topk(x, x_is_bf16, router_w, T, H, E, top_k, gating, logits, ids, 
     return _check(None, _lib.ft_router_topk(_p(x), int(x_is_bf16), _p(router_w), T, H, E, top_k,
                                             GATING.get(gating, gating), _p(logits), _p(ids), _p(gates),
                                             _s(stream)))
+
+
+def ft_route_decode(x, x_is_bf16, router_w, T, H, E, top_k, gating, logits, ids, gates, counts, offsets, perm,
+                    inv, ticket, stream=None):
+    return _check(None, _lib.ft_route_decode(_p(x), int(x_is_bf16), _p(router_w), T, H, E, top_k,
+                                             GATING.get(gating, gating), _p(logits), _p(ids), _p(gates),
+                                             _p(counts), _p(offsets), _p(perm), _p(inv), _p(ticket), _s(stream)))
 
 
 def ft_permute(ids, T, top_k, E, counts, offsets, perm, inv=None, stream=None):
@@ -312,6 +347,30 @@ def ft_expert_ffn_decode_noalloc(x, T, H, I, top_k, wdtype, blobs, experts, max_
         _p(x), T, H, I, top_k, WDTYPE.get(wdtype, wdtype), ctypes.cast(bl, ctypes.c_void_p),
         ctypes.cast(ex, ctypes.c_void_p), n, max_pairs_per_expert, _p(offsets), _p(perm), _p(gates), _p(inv),
         int(has_shared), _p(out), _s(stream)))
+
+
+def ft_cache_simulate_policy(policy, num_layers, num_experts, capacity, ops):
+    """Like ft_cache_simulate under FT_POLICY_LRU or FT_POLICY_STATIC."""
+    arr = _int_array(list(ops) or [0])
+    n = ctypes.c_int(0)
+    nerr = ctypes.c_int(0)
+    st = ft_cache_stats_t()
+    _check(None, _lib.ft_cache_simulate_policy(policy, num_layers, num_experts, capacity,
+                                               ctypes.cast(arr, ctypes.c_void_p), len(ops), None, 0,
+                                               ctypes.byref(n), None, None))
+    buf = (ft_access_t * max(n.value, 1))()
+    _check(None, _lib.ft_cache_simulate_policy(policy, num_layers, num_experts, capacity,
+                                               ctypes.cast(arr, ctypes.c_void_p), len(ops),
+                                               ctypes.cast(buf, ctypes.c_void_p), n.value, ctypes.byref(n),
+                                               ctypes.byref(st), ctypes.byref(nerr)))
+    trace = [tuple(getattr(buf[i], f) for f, _ in ft_access_t._fields_) for i in range(n.value)]
+    return trace, st.as_dict(), nerr.value
+
+
+def ft_probe_host_link(bytes_, iters=5):
+    a, b = ctypes.c_double(0), ctypes.c_double(0)
+    _check(None, _lib.ft_probe_host_link(bytes_, iters, ctypes.byref(a), ctypes.byref(b)))
+    return a.value, b.value
 
 
 def ft_version():

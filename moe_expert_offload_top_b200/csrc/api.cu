@@ -98,12 +98,16 @@ struct ft_moe {
   float* d_y = nullptr;
   int* h_ids = nullptr;
   int* d_err = nullptr;           // device-side error word (bounded waits that gave up)
+  int* d_ticket = nullptr;        // arrival counter of the fused decode routing kernel
   int* h_err = nullptr;
   uint16_t* d_ax = nullptr;       // gathered token rows for the prefill GEMMs
   ftk::GemmMaps maps;
   bool maps_dirty = true;
   int num_sms = 148;
   int gemm_min_avg_pairs = 32;    // tcgen05 path when bf16 and T*k/|S| >= this
+  int fused_routing = 1;          // one-launch routing for decode-sized calls
+  int inject_copy_fail = 0;       // countdown to a simulated failed slot fill (0 = off)
+  int inject_route_timeout = 0;   // countdown to a simulated routing-wait timeout
   cudaEvent_t route_ev = nullptr;
   int last_T = 0;
 
@@ -266,7 +270,11 @@ int issue_fills(ft_moe* h, std::vector<ftc::Access>& recs, size_t first) {
     const ftc::Access& a = recs[i];
     const uint8_t* src = h->pool + ((size_t)a.layer * h->E + a.expert) * h->blob;
     uint8_t* dst = h->arena + (size_t)a.slot * h->blob;
-    cudaError_t e = cudaMemcpyAsync(dst, src, h->blob, cudaMemcpyHostToDevice, h->copy);
+    cudaError_t e;
+    if (h->inject_copy_fail > 0 && --h->inject_copy_fail == 0)
+      e = cudaErrorUnknown;   // injected on the host: the copy is not issued
+    else
+      e = cudaMemcpyAsync(dst, src, h->blob, cudaMemcpyHostToDevice, h->copy);
     if (e != cudaSuccess) {
       // roll back this and every later fill of the set to "not resident"
       for (size_t j = i; j < recs.size(); ++j)
@@ -417,6 +425,8 @@ ft_moe* ft_moe_create(int num_experts, int top_k, int hidden, int inter, int wdt
   cudaEventCreateWithFlags(&h->route_ev, cudaEventDisableTiming);
   cudaMalloc(&h->d_err, sizeof(int));
   cudaMemset(h->d_err, 0, sizeof(int));
+  cudaMalloc(&h->d_ticket, sizeof(int));
+  cudaMemset(h->d_ticket, 0, sizeof(int));
   cudaHostAlloc(&h->h_err, sizeof(int), cudaHostAllocDefault);
   if (h->h_err) *h->h_err = 0;
   cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
@@ -521,24 +531,44 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   if (h->stage_pending.size() > 256) harvest_stages(h, false);
   StageEvents* se = stage_begin(h);
   stage_mark(se, SE_R0, s);
-  if (T > 64)
-    FT_CUDA(h, ftk::launch_router_logits_tiled(x, xbf16, router_w, T, h->H, E, h->d_logits, s));
-  else
-    FT_CUDA(h, ftk::launch_router_logits(x, xbf16, router_w, T, h->H, E, h->d_logits, s));
-  FT_CUDA(h, ftk::launch_topk_gates(h->d_logits, T, E, k, h->gating, h->d_ids, h->d_gates, s));
-  stage_mark(se, SE_R1, s);
-  FT_CUDA(h, cudaMemcpyAsync(h->h_ids, h->d_ids, sizeof(int) * (size_t)T * k,
-                             cudaMemcpyDeviceToHost, s));
-  FT_CUDA(h, cudaMemcpyAsync(h->h_err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost, s));
-  FT_CUDA(h, cudaEventRecord(h->route_ev, s));
-  stage_mark(se, SE_P0, s);
-  FT_CUDA(h, ftk::launch_permute(h->d_ids, T, k, E, h->d_counts, h->d_offsets, h->d_perm,
-                                 h->d_inv, s));
-  stage_mark(se, SE_P1, s);
-  h->perf.kernel_launches += 3;
+  const bool fused_route = h->fused_routing && T <= 64 && E <= 256 && k <= 16;
+  if (fused_route) {
+    // logits, top-k/gates and the permutation in one launch
+    FT_CUDA(h, ftk::launch_route_decode(x, xbf16, router_w, T, h->H, E, k, h->gating, h->d_logits, h->d_ids,
+                                        h->d_gates, h->d_counts, h->d_offsets, h->d_perm, h->d_inv,
+                                        h->d_ticket, s));
+    stage_mark(se, SE_R1, s);
+    FT_CUDA(h, cudaMemcpyAsync(h->h_ids, h->d_ids, sizeof(int) * (size_t)T * k,
+                               cudaMemcpyDeviceToHost, s));
+    FT_CUDA(h, cudaMemcpyAsync(h->h_err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost, s));
+    FT_CUDA(h, cudaEventRecord(h->route_ev, s));
+    stage_mark(se, SE_P0, s);
+    stage_mark(se, SE_P1, s);
+    h->perf.kernel_launches += 1;
+  } else {
+    if (T > 64)
+      FT_CUDA(h, ftk::launch_router_logits_tiled(x, xbf16, router_w, T, h->H, E, h->d_logits, s));
+    else
+      FT_CUDA(h, ftk::launch_router_logits(x, xbf16, router_w, T, h->H, E, h->d_logits, s));
+    FT_CUDA(h, ftk::launch_topk_gates(h->d_logits, T, E, k, h->gating, h->d_ids, h->d_gates, s));
+    stage_mark(se, SE_R1, s);
+    FT_CUDA(h, cudaMemcpyAsync(h->h_ids, h->d_ids, sizeof(int) * (size_t)T * k,
+                               cudaMemcpyDeviceToHost, s));
+    FT_CUDA(h, cudaMemcpyAsync(h->h_err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost, s));
+    FT_CUDA(h, cudaEventRecord(h->route_ev, s));
+    stage_mark(se, SE_P0, s);
+    FT_CUDA(h, ftk::launch_permute(h->d_ids, T, k, E, h->d_counts, h->d_offsets, h->d_perm,
+                                   h->d_inv, s));
+    stage_mark(se, SE_P1, s);
+    h->perf.kernel_launches += 3;
+  }
   h->perf.forwards++;
   {
     auto w0 = std::chrono::steady_clock::now();
+    if (h->inject_route_timeout > 0 && --h->inject_route_timeout == 0) {
+      cudaEventSynchronize(h->route_ev);   // the work itself completes; only the report is injected
+      return fail(h, FT_ERR_TIMEOUT, "timed out waiting for routing ids (injected)");
+    }
     rc = wait_event(h, h->route_ev, "routing ids");
     h->perf.host_wait_ms +=
         std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - w0).count();
@@ -645,7 +675,7 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   } else {
     stage_mark(se, SE_G0, s);
     FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, list, max_pairs, h->d_offsets,
-                                      h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr));
+                                      h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr, h->d_err));
   }
   stage_mark(se, SE_D1, s);
   FT_CUDA(h, ftk::launch_combine(h->d_y, h->d_gates, h->d_inv, T, h->H, k, h->has_shared != 0,
@@ -683,6 +713,42 @@ int ft_moe_sync(ft_moe* h) {
     return fail(h, FT_ERR_DEVICE_CHECK, "a kernel gave up waiting (code " + std::to_string(code) + ")");
   }
   return FT_OK;
+}
+
+int ft_moe_set_fused_routing(ft_moe* h, int enabled) {
+  if (!h) return FT_ERR_INVALID;
+  h->fused_routing = enabled != 0;
+  return FT_OK;
+}
+
+int ft_set_decode_gemv(int mode) {
+  if (mode != FT_DECODE_GEMV_BULK && mode != FT_DECODE_GEMV_REGISTER) return FT_ERR_INVALID;
+  ftk::set_decode_gemv_mode(mode);
+  return FT_OK;
+}
+
+int ft_moe_debug_inject(ft_moe* h, int what, int countdown) {
+  if (!h || countdown < 0) return FT_ERR_INVALID;
+  if (what == FT_INJECT_COPY_FAIL) h->inject_copy_fail = countdown;
+  else if (what == FT_INJECT_ROUTE_TIMEOUT) h->inject_route_timeout = countdown;
+  else return fail(h, FT_ERR_INVALID, "ft_moe_debug_inject: unknown fault");
+  return FT_OK;
+}
+
+int ft_debug_device_wait_selftest(int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return FT_ERR_INVALID;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* err = nullptr;
+  int code = 0;
+  if (cudaMallocAsync(&err, sizeof(int), s) != cudaSuccess) return FT_ERR_OOM;
+  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = ftk::launch_wait_selftest((unsigned long long)limit_us * 1000ull, err, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&code, err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  cudaFreeAsync(err, s);
+  cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return FT_ERR_CUDA;
+  return code == 199 ? FT_ERR_DEVICE_CHECK : FT_OK;
 }
 
 int ft_moe_set_gemm_threshold(ft_moe* h, int min_avg_pairs) {
@@ -840,12 +906,107 @@ void ft_moe_destroy(ft_moe* h) {
     for (int i = 0; i < SE_N; ++i) cudaEventDestroy(se.ev[i]);
   free_scratch(h);
   cudaFree(h->d_err);
+  cudaFree(h->d_ticket);
   if (h->h_err) cudaFreeHost(h->h_err);
   if (h->copy) cudaStreamDestroy(h->copy);
   cudaFree(h->arena);
   cudaFree(h->shared);
   if (h->pool) cudaFreeHost(h->pool);
   delete h;
+}
+
+// Static placement: the first `capacity` keys in (layer, expert) order are resident
+// for good; every other access is a miss served without caching.
+static int simulate_static(int num_layers, int num_experts, int capacity, const int* ops, int n_ops_ints,
+                           ft_access_t* trace, int trace_cap, int* n_trace, ft_cache_stats_t* stats) {
+  std::vector<ft_access_t> recs;
+  ft_cache_stats_t st{};
+  int cap = capacity;
+  int i = 0;
+  while (i < n_ops_ints) {
+    if (ops[i] == 0) {
+      if (i + 5 > n_ops_ints) return FT_ERR_INVALID;
+      const int call = ops[i + 1], layer = ops[i + 2], kind = ops[i + 3], n = ops[i + 4];
+      if (layer < 0 || layer >= num_layers || n < 0 || i + 5 + n > n_ops_ints) return FT_ERR_INVALID;
+      std::vector<int> es(ops + i + 5, ops + i + 5 + n);
+      std::sort(es.begin(), es.end());
+      es.erase(std::unique(es.begin(), es.end()), es.end());
+      for (int e : es) {
+        if (e < 0 || e >= num_experts) return FT_ERR_INVALID;
+        const int key = layer * num_experts + e;
+        const int hit = key < cap;
+        recs.push_back(ft_access_t{call, layer, e, kind, hit, hit ? key : -1, -1, -1});
+        if (kind == FT_ROUTED) { st.routed++; if (hit) st.hits++; else st.misses++; }
+        else { st.prefetch++; if (hit) st.prefetch_hits++; else st.prefetch_misses++; }
+      }
+      i += 5 + n;
+    } else if (ops[i] == 1) {
+      if (i + 2 > n_ops_ints || ops[i + 1] < 1) return FT_ERR_INVALID;
+      cap = ops[i + 1];
+      i += 2;
+    } else {
+      return FT_ERR_INVALID;
+    }
+  }
+  *n_trace = (int)recs.size();
+  for (int r = 0; r < std::min(trace_cap, *n_trace); ++r) trace[r] = recs[r];
+  st.resident = std::min(cap, num_layers * num_experts);
+  st.capacity = cap;
+  if (stats) *stats = st;
+  return FT_OK;
+}
+
+int ft_cache_simulate_policy(int policy, int num_layers, int num_experts, int capacity, const int* ops,
+                             int n_ops_ints, ft_access_t* trace, int trace_cap, int* n_trace,
+                             ft_cache_stats_t* stats, int* n_capacity_errors) {
+  if (policy == FT_POLICY_LRU)
+    return ft_cache_simulate(num_layers, num_experts, capacity, ops, n_ops_ints, trace, trace_cap, n_trace,
+                             stats, n_capacity_errors);
+  if (policy != FT_POLICY_STATIC || num_layers < 1 || num_experts < 1 || capacity < 1 || n_ops_ints < 0 ||
+      (n_ops_ints > 0 && !ops) || !n_trace || trace_cap < 0 || (trace_cap > 0 && !trace))
+    return FT_ERR_INVALID;
+  if (n_capacity_errors) *n_capacity_errors = 0;
+  return simulate_static(num_layers, num_experts, capacity, ops, n_ops_ints, trace, trace_cap, n_trace, stats);
+}
+
+int ft_probe_host_link(size_t bytes, int iters, double* h2d_gbs, double* d2h_gbs) {
+  if (bytes < 1024 || iters < 1 || !h2d_gbs || !d2h_gbs) return FT_ERR_INVALID;
+  void* hbuf = nullptr;
+  void* dbuf = nullptr;
+  cudaStream_t s = nullptr;
+  cudaEvent_t a = nullptr, b = nullptr;
+  int rc = FT_OK;
+  if (cudaHostAlloc(&hbuf, bytes, cudaHostAllocDefault) != cudaSuccess ||
+      cudaMalloc(&dbuf, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    rc = FT_ERR_OOM;
+  }
+  if (rc == FT_OK) {
+    memset(hbuf, 1, bytes);
+    cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+    cudaEventCreate(&a);
+    cudaEventCreate(&b);
+    for (int dir = 0; dir < 2 && rc == FT_OK; ++dir) {
+      const cudaMemcpyKind kind = dir == 0 ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToHost;
+      void* dst = dir == 0 ? dbuf : hbuf;
+      const void* src = dir == 0 ? hbuf : dbuf;
+      cudaMemcpyAsync(dst, src, bytes, kind, s);            // warm-up
+      cudaEventRecord(a, s);
+      for (int it = 0; it < iters; ++it) cudaMemcpyAsync(dst, src, bytes, kind, s);
+      cudaEventRecord(b, s);
+      float ms = 0.f;
+      if (cudaEventSynchronize(b) != cudaSuccess || cudaEventElapsedTime(&ms, a, b) != cudaSuccess || ms <= 0.f)
+        rc = FT_ERR_CUDA;
+      else
+        *(dir == 0 ? h2d_gbs : d2h_gbs) = (double)bytes * iters / (ms * 1e-3) / 1e9;
+    }
+  }
+  if (a) cudaEventDestroy(a);
+  if (b) cudaEventDestroy(b);
+  if (s) cudaStreamDestroy(s);
+  if (dbuf) cudaFree(dbuf);
+  if (hbuf) cudaFreeHost(hbuf);
+  return rc;
 }
 
 int ft_cache_simulate(int num_layers, int num_experts, int capacity, const int* ops,
@@ -923,6 +1084,20 @@ int ft_router_topk(const void* x, int x_is_bf16, const float* router_w, int T, i
   if (ftk::launch_topk_gates(logits, T, E, top_k, gating, ids, gates, s) != cudaSuccess)
     return FT_ERR_CUDA;
   return FT_OK;
+}
+
+int ft_route_decode(const void* x, int x_is_bf16, const float* router_w, int T, int H, int E, int top_k,
+                    int gating, float* logits, int* ids, float* gates, int* counts, int* offsets, int* perm,
+                    int* inv, int* ticket, void* stream) {
+  if (T < 0 || T > 64 || H < 4 || H % 4 || E < 1 || E > FT_MAX_EXPERTS || top_k < 1 || top_k > E ||
+      top_k > FT_MAX_TOPK || !ticket || !counts || !offsets ||
+      (T > 0 && (!x || !router_w || !logits || !ids || !gates || !perm || !inv)))
+    return FT_ERR_INVALID;
+  return ftk::launch_route_decode(x, x_is_bf16 != 0, router_w, T, H, E, top_k, gating, logits, ids, gates,
+                                  counts, offsets, perm, inv, ticket, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? FT_OK
+             : FT_ERR_CUDA;
 }
 
 int ft_permute(const int* ids, int T, int top_k, int E, int* counts, int* offsets, int* perm,

@@ -253,15 +253,32 @@ __global__ void combine_kernel(const float* __restrict__ y, const float* __restr
   }
 }
 
+int g_decode_mode = 1;   // FT_DECODE_GEMV_REGISTER: faster on the measured decode shapes
+int g_num_sms = 0;
+
 }  // namespace
+
+void set_decode_gemv_mode(int mode) { g_decode_mode = mode; }
 
 cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdtype,
                               const ExpertList& list, int max_pairs_per_expert, const int* offsets,
                               const int* perm, float* h, float* y, cudaStream_t s,
-                              cudaEvent_t between) {
+                              cudaEvent_t between, int* err) {
   if (list.n <= 0 || T <= 0) return cudaSuccess;
   int nt = max_pairs_per_expert < T ? max_pairs_per_expert : T;
   if (nt < 1) nt = 1;
+  int nt_all = nt;                        // the shared expert's entry owns all T tokens
+  for (int i = 0; i < list.n; ++i)
+    if (list.expert[i] < 0 && T > nt_all) nt_all = T;
+  if (g_decode_mode == 0 && nt_all <= 8 && tma_gemv_supported(H, I, wdtype)) {
+    if (g_num_sms <= 0) {
+      int dev = 0;
+      cudaGetDevice(&dev);
+      cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    return launch_ffn_decode_tma(x, T, H, I, k, wdtype, list, nt_all, offsets, perm, h, y, err, g_num_sms, s,
+                                 between);
+  }
   constexpr int RPW_GU = 2, RPW_D = 4;
   dim3 g1((I + kWarps * RPW_GU - 1) / (kWarps * RPW_GU), list.n);
   dim3 g2((H + kWarps * RPW_D - 1) / (kWarps * RPW_D), list.n);

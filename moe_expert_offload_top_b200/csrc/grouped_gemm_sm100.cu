@@ -28,6 +28,7 @@
 
 #include "common.cuh"
 #include "kernels.hpp"
+#include "sm100_sync.cuh"
 
 namespace ftk {
 
@@ -40,8 +41,6 @@ constexpr int B_BYTES = BN * BK * 2;      // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int GEMM_THREADS = 192;
 constexpr int TMEM_COLS = 512;            // two 128 x 256 fp32 accumulators
-constexpr long long WAIT_LIMIT = 1ll << 30;          // iteration cap of one wait
-constexpr unsigned long long WAIT_NS = 2000000000ull;  // and its time cap: 2 s
 
 struct GemmSmem {
   uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2];
@@ -51,58 +50,6 @@ struct GemmSmem {
   int row_start[kMaxList];
   int rows[kMaxList];
 };
-
-FT_DEVICE uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-FT_DEVICE void mbar_init(uint64_t* b, int count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
-}
-FT_DEVICE void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
-               : "memory");
-}
-FT_DEVICE void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-FT_DEVICE bool mbar_try(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-FT_DEVICE unsigned long long global_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-// Bounded wait.  Returns false (after flagging) on timeout or when the CTA aborts.
-FT_DEVICE bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* err, int code) {
-  if (mbar_try(b, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  for (long long i = 0; i < WAIT_LIMIT; ++i) {
-    if (mbar_try(b, parity)) return true;
-    if ((i & 255) == 255) {
-      if (*abort_flag) return false;
-      if (global_ns() - t0 > WAIT_NS) break;
-    }
-  }
-  *abort_flag = 1;
-  atomicExch(err, code);
-  return false;
-}
-// Bounded wait used while draining: no flagging.
-FT_DEVICE void mbar_drain(uint64_t* b, uint32_t parity) {
-  const unsigned long long t0 = global_ns();
-  for (long long i = 0; i < WAIT_LIMIT; ++i) {
-    if (mbar_try(b, parity)) return;
-    if ((i & 255) == 255 && global_ns() - t0 > WAIT_NS) return;
-  }
-}
 
 FT_DEVICE void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
   asm volatile(
@@ -338,6 +285,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
 }
 
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// arrives on; the wait must give up after limit_ns and leave code 199 in *err.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns, int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_wait(&bar, 0, &abort_flag, err, 199, limit_ns);
+  }
+}
+
 // A rows for the grouped GEMM: A[q] = x[perm[q] / k] (q < T*k), A[T*k + t] = x[t].
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int* __restrict__ perm, int T,
                                    int k, int H, int with_shared, uint16_t* __restrict__ A) {
@@ -352,6 +312,11 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int* __
 }
 
 }  // namespace
+
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, int* err, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns, err);
+  return cudaGetLastError();
+}
 
 size_t gemm_smem_bytes() { return 1024 + STAGES * STAGE_BYTES + sizeof(GemmSmem); }
 

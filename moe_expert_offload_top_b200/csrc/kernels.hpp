@@ -23,6 +23,12 @@ cudaError_t launch_router_logits(const void* x, bool x_bf16, const float* w_rout
                                  int E, float* logits, cudaStream_t s);
 cudaError_t launch_topk_gates(const float* logits, int T, int E, int k, int gating, int* ids,
                               float* gates, cudaStream_t s);
+// K1+K2 for decode (T <= 64, E <= 256, k <= 16) in one launch: logits, top-k + gates and
+// the stable permutation (the last router CTA does the second part).  *ticket must be 0
+// before the launch; the kernel leaves it 0.
+cudaError_t launch_route_decode(const void* x, bool x_bf16, const float* w_router, int T, int H, int E, int k,
+                                int gating, float* logits, int* ids, float* gates, int* counts, int* offsets,
+                                int* perm, int* inv, int* ticket, cudaStream_t s);
 // K2: stable counting sort of the T*k pairs by expert.
 // inv (optional): inv[t*k+j] = position of pair (t,j) in perm.
 cudaError_t launch_permute(const int* ids, int T, int k, int E, int* counts, int* offsets,
@@ -34,7 +40,16 @@ cudaError_t launch_permute(const int* ids, int T, int k, int E, int* counts, int
 cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdtype,
                               const ExpertList& list, int max_pairs_per_expert, const int* offsets,
                               const int* perm, float* h, float* y, cudaStream_t s,
-                              cudaEvent_t between = nullptr);
+                              cudaEvent_t between = nullptr, int* err = nullptr);
+// K3 (decode) with the weights streamed into shared memory by bulk copies (TMA);
+// same results as launch_ffn_decode.  Up to 8 pairs per entry.
+bool tma_gemv_supported(int H, int I, int wdtype);
+cudaError_t launch_ffn_decode_tma(const void* x, int T, int H, int I, int k, int wdtype, const ExpertList& list,
+                                  int nt, const int* offsets, const int* perm, float* h, float* y, int* err,
+                                  int num_sms, cudaStream_t s, cudaEvent_t between);
+// Decode GEMV selection (process-wide): 0 = bulk-copy kernel where supported, 1 = the
+// register-streaming kernel.
+void set_decode_gemv_mode(int mode);
 // K5: out[t] = sum_j gates[t][j] * y[inv[t*k+j]] (ascending j) + y[T*k+t] if has_shared.
 cudaError_t launch_combine(const float* y, const float* gates, const int* inv, int T, int H, int k,
                            bool has_shared, bool out_bf16, void* out, cudaStream_t s);
@@ -60,6 +75,8 @@ struct GemmMaps {
 };
 
 size_t gemm_smem_bytes();
+// One CTA waits (bounded by limit_ns) on an mbarrier nobody arrives on; sets *err = 199.
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, int* err, cudaStream_t s);
 // A[q] = x[perm[q] / k] for q < T*k; A[T*k + t] = x[t] when with_shared (bf16 rows of H).
 cudaError_t launch_gather_rows(const void* x, const int* perm, int T, int k, int H, bool with_shared,
                                void* A, cudaStream_t s);

@@ -187,6 +187,165 @@ router_logits_tiled_kernel(const XT* __restrict__ x, const float* __restrict__ w
     }
 }
 
+// Decode routing in one launch: the router CTAs of router_logits_kernel write
+// their logits; the last CTA to finish (a __threadfence + atomic ticket, no
+// waiting) then runs top-k + gates for every token and the stable permutation
+// of the T*k pairs, and resets the ticket for the next launch.
+template <typename XT>
+__global__ void __launch_bounds__(kRouterThreads)
+route_decode_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T, int H, int E, int k,
+                    int gating, float* __restrict__ z, int* __restrict__ ids, float* __restrict__ gates,
+                    int* __restrict__ counts, int* __restrict__ offsets, int* __restrict__ perm,
+                    int* __restrict__ inv, int* __restrict__ ticket) {
+  __shared__ float part[kRouterThreads / 32][kRouterEPB][kRouterTPB];
+  __shared__ int last;
+  __shared__ int s_cnt[256], s_base[256], s_wc[kRouterThreads / 32][256];
+  __shared__ int s_ids[64 * 16];
+  const int e0 = blockIdx.x * kRouterEPB, t0 = blockIdx.y * kRouterTPB;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  {  // ---- logits of this CTA's experts and tokens (as router_logits_kernel)
+    float acc[kRouterEPB][kRouterTPB];
+#pragma unroll
+    for (int i = 0; i < kRouterEPB; ++i)
+#pragma unroll
+      for (int t = 0; t < kRouterTPB; ++t) acc[i][t] = 0.f;
+    for (int hh = threadIdx.x * 4; hh < H; hh += kRouterThreads * 4) {
+      float wv[kRouterEPB][4];
+#pragma unroll
+      for (int i = 0; i < kRouterEPB; ++i) {
+        if (e0 + i < E) {
+          float4 a = *reinterpret_cast<const float4*>(w + (size_t)(e0 + i) * H + hh);
+          wv[i][0] = a.x; wv[i][1] = a.y; wv[i][2] = a.z; wv[i][3] = a.w;
+        } else {
+          wv[i][0] = wv[i][1] = wv[i][2] = wv[i][3] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < kRouterTPB; ++t) {
+        if (t0 + t < T) {
+          float xv[4];
+          load_x4<XT>(x + (size_t)(t0 + t) * H + hh, xv);
+#pragma unroll
+          for (int i = 0; i < kRouterEPB; ++i)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[i][t] = fmaf(wv[i][c], xv[c], acc[i][t]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kRouterEPB; ++i)
+#pragma unroll
+      for (int t = 0; t < kRouterTPB; ++t) {
+        float v = warp_sum(acc[i][t]);
+        if (lane == 0) part[warp][i][t] = v;
+      }
+    __syncthreads();
+    if (threadIdx.x < kRouterEPB * kRouterTPB) {
+      int i = threadIdx.x / kRouterTPB, t = threadIdx.x % kRouterTPB;
+      if (e0 + i < E && t0 + t < T) {
+        float sum = 0.f;
+        for (int wp = 0; wp < kRouterThreads / 32; ++wp) sum += part[wp][i][t];
+        z[(size_t)(t0 + t) * E + e0 + i] = sum;
+      }
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int nblocks = gridDim.x * gridDim.y;
+    last = atomicAdd(ticket, 1) == nblocks - 1;
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  // ---- top-k + gates: one warp per token, logits read through L2
+  for (int t = warp; t < T; t += kRouterThreads / 32) {
+    float v[8];
+    bool taken[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const int e = lane + 32 * m;
+      v[m] = e < E ? __ldcg(z + (size_t)t * E + e) : 0.f;
+      taken[m] = !(e < E);
+    }
+    float zsel[16];
+    int isel[16];
+    for (int r = 0; r < k; ++r) {
+      float best = 0.f;
+      int bi = 0x7FFFFFFF;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int e = lane + 32 * m;
+        if (!taken[m] && (bi == 0x7FFFFFFF || v[m] > best)) { best = v[m]; bi = e; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+        const bool better = (oi != 0x7FFFFFFF) && (bi == 0x7FFFFFFF || ob > best || (ob == best && oi < bi));
+        if (better) { best = ob; bi = oi; }
+      }
+      zsel[r] = best;
+      isel[r] = bi;
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        if (lane + 32 * m == bi) taken[m] = true;
+    }
+    if (lane == 0) {
+      float wsum = 0.f, wv[16];
+      for (int r = 0; r < k; ++r) {
+        const float a = gating == 0 ? expf(zsel[r] - zsel[0]) : 1.0f / (1.0f + expf(-zsel[r]));
+        wv[r] = a;
+        wsum += a;
+      }
+      for (int r = 0; r < k; ++r) {
+        ids[(size_t)t * k + r] = isel[r];
+        gates[(size_t)t * k + r] = wv[r] / wsum;
+        s_ids[t * k + r] = isel[r];
+      }
+    }
+  }
+  // ---- stable counting sort of the n = T*k pairs by expert (n <= 1024)
+  const int n = T * k;
+  for (int e = threadIdx.x; e < E; e += kRouterThreads) s_cnt[e] = 0;
+  __syncthreads();
+  for (int p = threadIdx.x; p < n; p += kRouterThreads) atomicAdd(&s_cnt[s_ids[p]], 1);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) { s_base[e] = run; run += s_cnt[e]; }
+    offsets[E] = run;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kRouterThreads) { counts[e] = s_cnt[e]; offsets[e] = s_base[e]; }
+  const unsigned lt = (1u << lane) - 1u;
+  for (int c = 0; c < n; c += kRouterThreads) {
+    for (int i = threadIdx.x; i < (kRouterThreads / 32) * E; i += kRouterThreads) s_wc[i / E][i % E] = 0;
+    __syncthreads();
+    const int p = c + threadIdx.x;
+    const int e = p < n ? s_ids[p] : -1;
+    const unsigned mask = __match_any_sync(0xFFFFFFFFu, e);
+    const int rank = __popc(mask & lt);
+    if (e >= 0 && rank == 0) s_wc[warp][e] = __popc(mask);
+    __syncthreads();
+    if (e >= 0) {
+      int before = 0;
+      for (int w2 = 0; w2 < warp; ++w2) before += s_wc[w2][e];
+      const int q = s_base[e] + before + rank;
+      perm[q] = p;
+      inv[p] = q;
+    }
+    __syncthreads();
+    for (int ee = threadIdx.x; ee < E; ee += kRouterThreads) {
+      int sum = 0;
+      for (int w2 = 0; w2 < kRouterThreads / 32; ++w2) sum += s_wc[w2][ee];
+      s_base[ee] += sum;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *ticket = 0;
+}
+
 }  // namespace
 
 cudaError_t launch_router_logits_tiled(const void* x, bool x_bf16, const float* w_router, int T, int H,
@@ -199,6 +358,23 @@ cudaError_t launch_router_logits_tiled(const void* x, bool x_bf16, const float* 
   else
     router_logits_tiled_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(x), w_router, T, H, E,
                                                            logits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_decode(const void* x, bool x_bf16, const float* w_router, int T, int H, int E, int k,
+                                int gating, float* logits, int* ids, float* gates, int* counts, int* offsets,
+                                int* perm, int* inv, int* ticket, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  if (T > 64 || E > 256 || k > 16) return cudaErrorInvalidValue;
+  dim3 grid((E + kRouterEPB - 1) / kRouterEPB, (T + kRouterTPB - 1) / kRouterTPB);
+  if (x_bf16)
+    route_decode_kernel<uint16_t><<<grid, kRouterThreads, 0, s>>>(static_cast<const uint16_t*>(x), w_router, T, H,
+                                                                  E, k, gating, logits, ids, gates, counts, offsets,
+                                                                  perm, inv, ticket);
+  else
+    route_decode_kernel<float><<<grid, kRouterThreads, 0, s>>>(static_cast<const float*>(x), w_router, T, H, E, k,
+                                                               gating, logits, ids, gates, counts, offsets, perm,
+                                                               inv, ticket);
   return cudaGetLastError();
 }
 

@@ -54,6 +54,72 @@ def test_router_topk_parity(T, H, E, k, gating, xbf16):
     assert np.max(np.abs(g.cpu().numpy()[ok] - gr[ok])) <= 2e-6
 
 
+@pytest.mark.parametrize("T,H,E,k,gating,xbf16", [
+    (1, 256, 16, 2, "softmax", False), (1, 2048, 128, 8, "softmax", True), (1, 4096, 256, 6, "sigmoid", True),
+    (8, 7168, 256, 8, "sigmoid", True), (32, 7168, 256, 8, "sigmoid", True), (64, 512, 256, 16, "softmax", True),
+    (3, 64, 8, 8, "softmax", False), (48, 256, 16, 2, "sigmoid", True), (64, 256, 16, 16, "sigmoid", True),
+])
+def test_fused_decode_routing_parity(T, H, E, k, gating, xbf16):
+    x = synth.normal_f32(5, 8, 0, 0, T * H).reshape(T, H)
+    w = synth.normal_f32(5, 4, 0, 0, E * H, 0.02).reshape(E, H)
+    xd, xv = _bf16_dev(x) if xbf16 else (torch.from_numpy(np.ascontiguousarray(x)).to(DEV), x)
+    wd = torch.from_numpy(w).to(DEV)
+    z = torch.empty((T, E), device=DEV)
+    ids = torch.full((T, k), -1, dtype=torch.int32, device=DEV)
+    g = torch.empty((T, k), device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offs = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    ticket = torch.zeros(1, dtype=torch.int32, device=DEV)
+    for rep in range(2):                      # the ticket is left at 0 for the next call
+        ft.ft_route_decode(xd, xbf16, wd, T, H, E, k, gating, z, ids, g, counts, offs, perm, inv, ticket)
+    torch.cuda.synchronize()
+    assert int(ticket.item()) == 0
+    zr = moe.router_logits(xv, w)
+    ir, gap = moe.topk(zr, k)
+    gi = ids.cpu().numpy()
+    div = first_divergence(gi, ir, gap)
+    ok = np.all(gi == ir, axis=1)
+    gr = moe.gates(np.take_along_axis(zr, ir.astype(np.int64), axis=1), gating)
+    assert np.max(np.abs(g.cpu().numpy()[ok] - gr[ok])) <= 2e-6
+    pp, iv = perm.cpu().numpy(), inv.cpu().numpy()
+    if div is None:                             # same selection: the oracle's permutation, bit for bit
+        c, o, p = moe.permute(ir, E)
+        assert np.array_equal(counts.cpu().numpy(), c) and np.array_equal(offs.cpu().numpy(), o)
+        assert np.array_equal(pp, p) and np.array_equal(iv, np.argsort(p))
+    else:                                       # a near-tie flip: check the sort's properties
+        flat = gi.reshape(-1)
+        assert sorted(pp.tolist()) == list(range(T * k)) and np.array_equal(pp[iv], np.arange(T * k))
+        keys = flat[pp] * (T * k) + pp
+        assert np.all(np.diff(keys) > 0)
+
+
+def test_fused_decode_routing_after_wider_call():
+    # a 256-expert call leaves every row of the kernel's per-warp counts dirty in
+    # shared memory; a following 16-expert call with many tokens must not read them
+    def run(T, H, E, k):
+        x = synth.normal_f32(T + E, 8, 0, 0, T * H).reshape(T, H)
+        w = synth.normal_f32(T + E, 4, 0, 0, E * H, 0.3).reshape(E, H)
+        xd, xv = _bf16_dev(x)
+        bufs = [torch.empty((T, E), device=DEV), torch.empty((T, k), dtype=torch.int32, device=DEV),
+                torch.empty((T, k), device=DEV), torch.empty(E, dtype=torch.int32, device=DEV),
+                torch.empty(E + 1, dtype=torch.int32, device=DEV), torch.empty(T * k, dtype=torch.int32, device=DEV),
+                torch.empty(T * k, dtype=torch.int32, device=DEV)]
+        ticket = torch.zeros(1, dtype=torch.int32, device=DEV)
+        ft.ft_route_decode(xd, True, torch.from_numpy(w).to(DEV), T, H, E, k, "softmax", *bufs, ticket)
+        torch.cuda.synchronize()
+        ir, gap = moe.topk(moe.router_logits(xv, w), k)
+        if first_divergence(bufs[1].cpu().numpy(), ir, gap) is None:
+            c, o, p = moe.permute(ir, E)
+            assert np.array_equal(bufs[4].cpu().numpy(), o)
+            assert np.array_equal(bufs[5].cpu().numpy(), p) and np.array_equal(bufs[6].cpu().numpy(), np.argsort(p))
+    for rep in range(4):
+        run(64, 512, 256, 16)
+        run(48, 256, 16, 2)
+        run(64, 256, 8, 4)
+
+
 @pytest.mark.parametrize("T,k,E", [(1, 2, 16), (7, 8, 128), (33, 6, 256), (300, 8, 256), (4096, 6, 256),
                                    (5, 16, 16), (0, 2, 16)])
 def test_permute_parity(T, k, E):
@@ -76,13 +142,22 @@ def test_permute_parity(T, k, E):
         assert np.array_equal(inv.cpu().numpy(), np.argsort(p))
 
 
+@pytest.mark.parametrize("gemv_mode", [0, 1])
 @pytest.mark.parametrize("wd,H,I,T,E,k,shared", [
     ("f32", 256, 128, 1, 16, 2, False), ("f32", 256, 128, 20, 4, 2, True),
     ("bf16", 2048, 768, 1, 128, 8, False), ("bf16", 2048, 768, 3, 16, 8, True),
     ("bf16", 1024, 512, 37, 6, 3, True), ("int4", 1024, 512, 1, 16, 4, False),
     ("int4", 7168, 2048, 2, 8, 8, False), ("int4", 1024, 256, 19, 5, 2, True),
 ])
-def test_expert_ffn_and_combine_parity(wd, H, I, T, E, k, shared):
+def test_expert_ffn_and_combine_parity(wd, H, I, T, E, k, shared, gemv_mode):
+    ft.ft_set_decode_gemv(gemv_mode)      # bulk-copy kernel (where supported) or register kernel
+    try:
+        _ffn_and_combine_case(wd, H, I, T, E, k, shared)
+    finally:
+        ft.ft_set_decode_gemv(ft.FT_DECODE_GEMV_REGISTER)
+
+
+def _ffn_and_combine_case(wd, H, I, T, E, k, shared):
     cfg = synth.MoeConfig("t", 1, E, H, I, k, "sigmoid", wd, shared, E, T, (T,), "iid", "decode")
     rng = np.random.default_rng(H + T)
     ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
