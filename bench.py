@@ -311,9 +311,9 @@ def run_ours(args):
     torch.cuda.set_device(dev)
     cfg = synth.CONFIGS[CONFIG_ID]
     W, K = args.warmup, args.steps
-    vals, bits = token_chain(cfg, rank, W + 2 * K)      # device leg, then e2e leg
+    vals, bits = token_chain(cfg, rank, W + 3 * K)      # device leg, stage leg, e2e leg
     stack = GpuStack(cfg, device=dev)
-    x_dev = torch.from_numpy(bits).view(torch.bfloat16).to(dev).view(W + 2 * K, 1, cfg.H)
+    x_dev = torch.from_numpy(bits).view(torch.bfloat16).to(dev).view(W + 3 * K, 1, cfg.H)
     out = torch.empty((cfg.L, 1, cfg.H), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -322,10 +322,9 @@ def run_ours(args):
         stack.step(x_dev[s], out, stream)
     torch.cuda.synchronize(dev)
 
-    # ---- device-timed leg: inputs resident in HBM
+    # ---- device-timed leg: inputs resident in HBM, no instrumentation
     stack.reset_stats()
     ft.ft_moe_reset_perf(stack.h)
-    ft.ft_moe_set_stage_timing(stack.h, 1)
     clocks = ClockSampler(local)
     clocks.start()
     barrier(dev)
@@ -339,14 +338,23 @@ def run_ours(args):
     barrier(dev)
     clk = clocks.stop()
     dt = e0.elapsed_time(e1) * 1e-3
-    perf = ft.ft_moe_perf(stack.h)
+    launches = ft.ft_moe_perf(stack.h)["kernel_launches"]
     st = stack.stats()
-    ft.ft_moe_set_stage_timing(stack.h, 0)
     tokens, t_max = aggregate(K * cfg.batches[0], dt, dev)
+
+    # ---- stage leg: the same number of steps (the chain continued) with CUDA events
+    # around every stage on the forward's stream; gives each kernel's device time
+    ft.ft_moe_reset_perf(stack.h)
+    ft.ft_moe_set_stage_timing(stack.h, 1)
+    for s in range(W + K, W + 2 * K):
+        stack.step(x_dev[s], out, stream)
+    torch.cuda.synchronize(dev)
+    perf = ft.ft_moe_perf(stack.h)
+    ft.ft_moe_set_stage_timing(stack.h, 0)
 
     # ---- end-to-end leg through host buffers (pinned): H2D of the step's token and
     # D2H of the step's layer outputs inside the timed region, read back every step
-    x_host = torch.from_numpy(bits[W + K:W + 2 * K]).view(torch.bfloat16).view(K, 1, cfg.H).pin_memory()
+    x_host = torch.from_numpy(bits[W + 2 * K:W + 3 * K]).view(torch.bfloat16).view(K, 1, cfg.H).pin_memory()
     out_host = torch.empty((K, cfg.L, 1, cfg.H), dtype=torch.bfloat16).pin_memory()
     x_in = torch.empty((1, cfg.H), dtype=torch.bfloat16, device=dev)
     barrier(dev)
@@ -388,7 +396,7 @@ def run_ours(args):
             "e2e": {"value": e2e_tokens / e2e_max, "unit": "tokens/s",
                     "h2d_bytes_per_step": int(cfg.H * 2 * cfg.batches[0]),
                     "d2h_bytes_per_step": int(cfg.L * cfg.H * 2 * cfg.batches[0])},
-            "gpu_launches": int(perf["kernel_launches"]),
+            "gpu_launches": int(launches),
             "clocks": clk,
             "cache": {"miss_rate": st["misses"] / max(st["routed"], 1), "routed": st["routed"],
                       "misses": st["misses"], "h2d_bytes": st["h2d_bytes"],
@@ -419,7 +427,7 @@ def run_ours(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=160)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)

@@ -60,7 +60,7 @@ enum ft_status {
   FT_ERR_DEVICE_CHECK = 7  /* a kernel's own bounds check failed (the kernel skipped the access) */
 };
 
-enum ft_wdtype { FT_W_F32 = 0, FT_W_BF16 = 1, FT_W_INT4_G128 = 2 };
+enum ft_wdtype { FT_W_F32 = 0, FT_W_BF16 = 1, FT_W_INT4_G128 = 2, FT_W_NVFP4 = 3 };
 enum ft_gating { FT_GATE_SOFTMAX = 0, FT_GATE_SIGMOID = 1 };
 enum ft_access_kind { FT_ROUTED = 0, FT_PREFETCH = 1 };
 
@@ -103,7 +103,8 @@ typedef struct {
 /* Creates a stack description with `cache_slots` expert slots of one blob each.
  *   num_experts E (1..FT_MAX_EXPERTS), top_k k (1..min(E, FT_MAX_TOPK)),
  *   hidden H and inter I (SwiGLU intermediate): multiples of 8.  For
- *   FT_W_INT4_G128 they must be multiples of 128.  wdtype is an ft_wdtype.
+ *   FT_W_INT4_G128 they must be multiples of 128, for FT_W_NVFP4 of 32.  wdtype is an
+ *   ft_wdtype.
  * The stack starts with 1 layer, softmax gating and no shared expert.  Call
  * ft_moe_set_layers before filling the pool.  Allocates the slot arena on the
  * current device; the pinned pool is allocated by ft_moe_set_layers.
@@ -131,7 +132,14 @@ FT_API size_t ft_moe_blob_bytes(const ft_moe* h);
  *               of a row holds element 2b in its low nibble and 2b+1 in its high
  *               nibble, two's complement in [-8, 7].  Then the bf16 scales
  *               S_gate [I][H/128], S_up [I][H/128], S_down [H][I/128], one per 128
- *               consecutive K elements of a row.  w = q * s. */
+ *               consecutive K elements of a row.  w = q * s.
+ *   nvfp4:      packed e2m1 W_gate [I][H/2], W_up [I][H/2], W_down [H][I/2] (same nibble
+ *               order; code bit 3 sign, bits 2-1 exponent bias 1, bit 0 mantissa), then
+ *               e4m3 block scales S_gate [I][H/16], S_up [I][H/16], S_down [H][I/16] (one
+ *               byte per 16 consecutive K elements), then the fp32 global scales g_gate,
+ *               g_up, g_down and 4 zero bytes.  w = e2m1(q) * e4m3(s) * g.  H and I must
+ *               be multiples of 32.  Decode only: nvfp4 stacks use the streaming GEMV for
+ *               every batch size. */
 FT_API void* ft_moe_pool_ptr(ft_moe* h, int layer, int expert);
 
 /* Copies the shared expert of `layer` (a host blob in the same layout) into resident
@@ -164,7 +172,10 @@ FT_API int ft_moe_reserve(ft_moe* h, int max_tokens);
  * the k outputs in ascending k order, plus the shared expert.
  * Returns FT_ERR_CAPACITY, before any state changes, if the distinct experts of
  * the call exceed the cache slots.  All forwards of a handle are ordered: a
- * forward on another stream first waits for the previous forward's kernels. */
+ * forward on another stream first waits for the previous forward's kernels.  A forward
+ * that fails after its first launch drains `stream` before returning, except on
+ * FT_ERR_TIMEOUT, after which the caller should call ft_moe_sync before using the
+ * handle on another stream. */
 FT_API int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const float* router_w,
                    void* out, void* stream);
 
@@ -183,16 +194,6 @@ FT_API int ft_moe_set_gemm_threshold(ft_moe* h, int min_avg_pairs);
 /* Routing launch shape for calls of up to 64 tokens: 1 (default) = one fused kernel
  * (ft_route_decode), 0 = router, top-k and permutation as three launches.  Same results. */
 FT_API int ft_moe_set_fused_routing(ft_moe* h, int enabled);
-
-/* Decode GEMV kernel (process-wide; same results, different speed):
- *   FT_DECODE_GEMV_REGISTER (default): 16-byte loads straight to registers, one CTA per
- *     block of rows.
- *   FT_DECODE_GEMV_BULK: weights streamed into shared memory by bulk copies, one
- *     persistent CTA per SM, packed int4 dequant; used for up to 8 tokens per expert when
- *     rows allow it (bf16/f32: H, I multiples of 8; int4: multiples of 1024), else the
- *     register kernel. */
-enum ft_decode_gemv { FT_DECODE_GEMV_BULK = 0, FT_DECODE_GEMV_REGISTER = 1 };
-FT_API int ft_set_decode_gemv(int mode);
 
 /* Host-side fault injection for tests of failure handling (no GPU fault is made).
  *   FT_INJECT_COPY_FAIL: the countdown-th slot fill from now is reported failed instead
@@ -223,6 +224,10 @@ FT_API int ft_moe_last_routing(const ft_moe* h, int* ids, float* gates, int* n_t
  * it, keeping recency).  Reallocates the arena and copies resident slots on the
  * device.  FT_ERR_BUSY if a forward is in flight on another thread. */
 FT_API int ft_cache_resize(ft_moe* h, int slots);
+
+/* Empties the cache at a safe point (waits for the handle's work): every slot becomes
+ * free, capacity, counters and trace are kept. */
+FT_API int ft_cache_clear(ft_moe* h);
 
 /* Reads the counters (waits for the copy stream so h2d_seconds is complete). */
 FT_API int ft_cache_stats(const ft_moe* h, ft_cache_stats_t* out);

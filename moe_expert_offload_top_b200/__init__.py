@@ -22,14 +22,13 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 FT_OK, FT_ERR_INVALID, FT_ERR_OOM, FT_ERR_CUDA, FT_ERR_CAPACITY, FT_ERR_BUSY, FT_ERR_TIMEOUT, \
     FT_ERR_DEVICE_CHECK = range(8)
-FT_W_F32, FT_W_BF16, FT_W_INT4_G128 = 0, 1, 2
+FT_W_F32, FT_W_BF16, FT_W_INT4_G128, FT_W_NVFP4 = 0, 1, 2, 3
 FT_GATE_SOFTMAX, FT_GATE_SIGMOID = 0, 1
 FT_ROUTED, FT_PREFETCH = 0, 1
 FT_INJECT_COPY_FAIL, FT_INJECT_ROUTE_TIMEOUT = 1, 2
 FT_POLICY_LRU, FT_POLICY_STATIC = 0, 1
-FT_DECODE_GEMV_BULK, FT_DECODE_GEMV_REGISTER = 0, 1
 FT_MAX_EXPERTS, FT_MAX_TOPK = 256, 16
-WDTYPE = {"f32": FT_W_F32, "bf16": FT_W_BF16, "int4": FT_W_INT4_G128}
+WDTYPE = {"f32": FT_W_F32, "bf16": FT_W_BF16, "int4": FT_W_INT4_G128, "nvfp4": FT_W_NVFP4}
 GATING = {"softmax": FT_GATE_SOFTMAX, "sigmoid": FT_GATE_SIGMOID}
 
 
@@ -75,6 +74,7 @@ _SIGS = {
     "ft_moe_last_routing": ([_vp, _vp, _vp, ctypes.POINTER(_i)], _i),
     "ft_cache_resize": ([_vp, _i], _i),
     "ft_cache_stats": ([_vp, ctypes.POINTER(ft_cache_stats_t)], _i),
+    "ft_cache_clear": ([_vp], _i),
     "ft_cache_reset_stats": ([_vp], _i),
     "ft_cache_trace": ([_vp, _vp, _i, ctypes.POINTER(_i)], _i),
     "ft_cache_set_trace": ([_vp, _i], _i),
@@ -95,7 +95,6 @@ _SIGS = {
     "ft_moe_sync": ([_vp], _i),
     "ft_moe_set_gemm_threshold": ([_vp, _i], _i),
     "ft_moe_debug_inject": ([_vp, _i, _i], _i),
-    "ft_set_decode_gemv": ([_i], _i),
     "ft_moe_set_fused_routing": ([_vp, _i], _i),
     "ft_debug_device_wait_selftest": ([_i, _vp], _i),
     "ft_moe_perf": ([_vp, ctypes.POINTER(ft_perf_t)], _i),
@@ -201,6 +200,10 @@ def ft_cache_resize(h, slots):
     return _check(h, _lib.ft_cache_resize(h, slots))
 
 
+def ft_cache_clear(h):
+    return _check(h, _lib.ft_cache_clear(h))
+
+
 def ft_cache_stats(h):
     st = ft_cache_stats_t()
     _check(h, _lib.ft_cache_stats(h, ctypes.byref(st)))
@@ -245,10 +248,6 @@ def ft_moe_set_gemm_threshold(h, min_avg_pairs):
 
 def ft_moe_set_fused_routing(h, enabled):
     return _check(h, _lib.ft_moe_set_fused_routing(h, int(enabled)))
-
-
-def ft_set_decode_gemv(mode):
-    return _check(None, _lib.ft_set_decode_gemv(mode))
 
 
 def ft_moe_debug_inject(h, what, countdown):

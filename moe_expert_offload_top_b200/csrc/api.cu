@@ -395,7 +395,7 @@ ft_moe* ft_moe_create(int num_experts, int top_k, int hidden, int inter, int wdt
                       int cache_slots) {
   if (num_experts < 1 || num_experts > FT_MAX_EXPERTS || top_k < 1 || top_k > num_experts ||
       top_k > FT_MAX_TOPK || hidden < 8 || inter < 8 || hidden % 8 || inter % 8 ||
-      wdtype < FT_W_F32 || wdtype > FT_W_INT4_G128 || cache_slots < 1) {
+      wdtype < FT_W_F32 || wdtype > FT_W_NVFP4 || cache_slots < 1) {
     g_create_error = "ft_moe_create: invalid argument";
     return nullptr;
   }
@@ -403,12 +403,17 @@ ft_moe* ft_moe_create(int num_experts, int top_k, int hidden, int inter, int wdt
     g_create_error = "ft_moe_create: int4 needs hidden and inter multiples of 128";
     return nullptr;
   }
+  if (wdtype == FT_W_NVFP4 && (hidden % 32 || inter % 32)) {
+    g_create_error = "ft_moe_create: nvfp4 needs hidden and inter multiples of 32";
+    return nullptr;
+  }
   ft_moe* h = new ft_moe();
   cudaGetDevice(&h->device);
   h->E = num_experts; h->k = top_k; h->H = hidden; h->I = inter; h->wdtype = wdtype;
   h->C = cache_slots;
   const size_t n = 3ull * hidden * inter;
-  h->blob = wdtype == FT_W_F32 ? 4 * n : wdtype == FT_W_BF16 ? 2 * n : n / 2 + 2 * (n / 128);
+  h->blob = wdtype == FT_W_F32 ? 4 * n : wdtype == FT_W_BF16 ? 2 * n
+            : wdtype == FT_W_NVFP4 ? n / 2 + n / 16 + 16 : n / 2 + 2 * (n / 128);
   if (cudaMalloc(&h->arena, (size_t)cache_slots * h->blob) != cudaSuccess) {
     cudaGetLastError();
     g_create_error = "ft_moe_create: slot arena allocation failed";
@@ -575,11 +580,17 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   }
   if (rc) return rc;
   h->last_T = T;
+  // A failure from here on leaves no kernel of this call running: the caller's stream is
+  // drained first, so a following forward on another stream cannot race on the scratch.
+  auto bail = [&](int code, const std::string& msg) {
+    cudaStreamSynchronize(s);
+    return fail(h, code, msg);
+  };
   if (*h->h_err) {
     const int code = *h->h_err;
     *h->h_err = 0;
     cudaMemsetAsync(h->d_err, 0, sizeof(int), s);
-    return fail(h, FT_ERR_DEVICE_CHECK,
+    return bail(FT_ERR_DEVICE_CHECK,
                 "a previous forward's kernel gave up waiting (code " + std::to_string(code) + ")");
   }
 
@@ -587,7 +598,7 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   std::vector<int> cnt(E, 0);
   for (int i = 0; i < T * k; ++i) {
     const int e = h->h_ids[i];
-    if (e < 0 || e >= E) return fail(h, FT_ERR_DEVICE_CHECK, "router produced an invalid expert id");
+    if (e < 0 || e >= E) return bail(FT_ERR_DEVICE_CHECK, "router produced an invalid expert id");
     cnt[e]++;
   }
   std::vector<int> S, keys;
@@ -601,7 +612,7 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   const bool pre0 = h->prefill && layer == 0;
   const bool pre_next = h->prefill && layer + 1 < h->L;
   if ((int)S.size() > h->C || ((pre0 || pre_next) && E > h->C))
-    return fail(h, FT_ERR_CAPACITY, "cache has fewer slots than one step needs");
+    return bail(FT_ERR_CAPACITY, "cache has fewer slots than one step needs");
 
   const long long call = h->call;
   std::vector<ftc::Access> recs;
@@ -609,13 +620,13 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
     h->lru.access_set(all_keys(h, 0), E, (int)call, FT_PREFETCH, recs);
     rc = issue_fills(h, recs, 0);
     account(h, recs, 0);
-    if (rc) return rc;
+    if (rc) return bail(rc, h->err);
   }
   const size_t first_routed = recs.size();
   h->lru.access_set(keys, E, (int)call, FT_ROUTED, recs);
   rc = issue_fills(h, recs, first_routed);
   account(h, recs, first_routed);
-  if (rc) return rc;
+  if (rc) return bail(rc, h->err);
 
   // the kernels read the slots of S: wait for their newest fill
   ftk::ExpertList list;
@@ -642,8 +653,9 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
     // algorithmic bytes: every weight of the listed experts once, their inputs and outputs
     const double xb = xbf16 ? 2.0 : 4.0;
     const size_t mat = (size_t)h->H * h->I;
-    const double wmat = h->wdtype == FT_W_INT4_G128 ? mat / 2.0 + 2.0 * (mat / 128) :
-                        (double)mat * (h->wdtype == FT_W_F32 ? 4 : 2);
+    const double wmat = h->wdtype == FT_W_INT4_G128 ? mat / 2.0 + 2.0 * (mat / 128)
+                        : h->wdtype == FT_W_NVFP4 ? mat / 2.0 + mat / 16.0
+                                                  : (double)mat * (h->wdtype == FT_W_F32 ? 4 : 2);
     const double pairs = (double)T * k + (h->has_shared ? T : 0);
     se->gu_bytes = list.n * 2.0 * wmat + pairs * (h->H * xb + h->I * 4.0);
     se->d_bytes = list.n * wmat + pairs * (h->I * 4.0 + h->H * 4.0);
@@ -718,12 +730,6 @@ int ft_moe_sync(ft_moe* h) {
 int ft_moe_set_fused_routing(ft_moe* h, int enabled) {
   if (!h) return FT_ERR_INVALID;
   h->fused_routing = enabled != 0;
-  return FT_OK;
-}
-
-int ft_set_decode_gemv(int mode) {
-  if (mode != FT_DECODE_GEMV_BULK && mode != FT_DECODE_GEMV_REGISTER) return FT_ERR_INVALID;
-  ftk::set_decode_gemv_mode(mode);
   return FT_OK;
 }
 
@@ -834,6 +840,16 @@ int ft_cache_resize(ft_moe* h, int slots) {
   h->st.evictions += (long long)evicted.size();
   h->slot_last_use.assign(slots, -1);
   h->slot_fill_batch.assign(slots, -1);
+  return FT_OK;
+}
+
+int ft_cache_clear(ft_moe* h) {
+  if (!h) return FT_ERR_INVALID;
+  BusyGuard g(h);
+  if (!g.ok) return fail(h, FT_ERR_BUSY, "ft_cache_clear: forward in flight");
+  FT_CUDA(h, cudaStreamSynchronize(h->copy));
+  if (h->has_last_stream) FT_CUDA(h, cudaStreamSynchronize(h->last_stream));
+  reset_cache_state(h);
   return FT_OK;
 }
 
@@ -1116,8 +1132,8 @@ int ft_expert_ffn_decode(const void* x, int T, int H, int I, int top_k, int wdty
                          int max_pairs_per_expert, const int* offsets, const int* perm, float* h,
                          float* y, void* stream) {
   if (T < 0 || H < 8 || I < 8 || H % 8 || I % 8 || top_k < 1 || n_list < 0 ||
-      n_list > ftk::kMaxList || wdtype < FT_W_F32 || wdtype > FT_W_INT4_G128 ||
-      (wdtype == FT_W_INT4_G128 && (H % 128 || I % 128)) ||
+      n_list > ftk::kMaxList || wdtype < FT_W_F32 || wdtype > FT_W_NVFP4 ||
+      (wdtype == FT_W_INT4_G128 && (H % 128 || I % 128)) || (wdtype == FT_W_NVFP4 && (H % 32 || I % 32)) ||
       (n_list > 0 && (!blobs || !experts || !offsets || !perm || !h || !y || !x)))
     return FT_ERR_INVALID;
   ftk::ExpertList list;

@@ -10,6 +10,8 @@
 // matrix-vector products bound by HBM bandwidth: every weight byte is read
 // exactly once per launch with 16-byte streaming loads, and the few token
 // vectors of an expert are staged once per CTA in shared memory.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "kernels.hpp"
 
@@ -17,10 +19,22 @@ namespace ftk {
 
 namespace {
 
-enum { WT_F32 = 0, WT_BF16 = 1, WT_INT4 = 2 };
+enum { WT_F32 = 0, WT_BF16 = 1, WT_INT4 = 2, WT_NVFP4 = 3 };
 enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
 
-constexpr int kWarps = 4;               // warps per CTA
+#ifndef FT_GEMV_WARPS
+#define FT_GEMV_WARPS 4
+#endif
+#ifndef FT_GEMV_GU_RPW
+#define FT_GEMV_GU_RPW 2
+#endif
+#ifndef FT_GEMV_D_RPW
+#define FT_GEMV_D_RPW 4
+#endif
+#ifndef FT_GEMV_NT_MAX
+#define FT_GEMV_NT_MAX 8
+#endif
+constexpr int kWarps = FT_GEMV_WARPS;   // warps per CTA
 constexpr int kThreads = kWarps * 32;
 
 // Elements held by one 16-byte weight load.
@@ -28,10 +42,27 @@ template <int WT> struct WTraits;
 template <> struct WTraits<WT_F32>  { static constexpr int EL = 4; };
 template <> struct WTraits<WT_BF16> { static constexpr int EL = 8; };
 template <> struct WTraits<WT_INT4> { static constexpr int EL = 32; };
+template <> struct WTraits<WT_NVFP4> { static constexpr int EL = 32; };
+
+// Two e2m1 values of one byte -> fp32 (hardware conversion to f16x2, then widened).
+FT_DEVICE void e2m1x2_to_f32(uint32_t byte, float& lo, float& hi) {
+  uint32_t h2;
+  asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h2) : "r"(byte));
+  lo = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+  hi = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+}
+// Two e4m3 values of a 16-bit word -> fp32.
+FT_DEVICE void e4m3x2_to_f32(uint32_t two, float& lo, float& hi) {
+  uint32_t h2;
+  asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h2) : "r"(two));
+  lo = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+  hi = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+}
 
 // 16-byte weight load, read once per launch: evict-first in the caches.  Not
 // volatile, so the compiler may hoist the loads of later iterations.
 FT_DEVICE uint4 ldw(const uint8_t* p) { return __ldcs(reinterpret_cast<const uint4*>(p)); }
+
 
 // Weights of one 16-byte chunk, group g of 8 elements (f32: 4 elements) -> fp32
 // (int4: the raw integers; the group scale multiplies the chunk's partial sum).
@@ -94,19 +125,30 @@ grouped_gemv_kernel(const void* __restrict__ xin, int T, int H, int I, int k,
   const int entry = blockIdx.y;
   const int e = list.expert[entry];
   const uint8_t* blob = list.blob[entry];
-  const int q0 = e >= 0 ? offsets[e] : T * k;
-  const int q1 = e >= 0 ? offsets[e + 1] : T * k + T;
-  if (q1 <= q0) return;
   const int K = GU ? H : I;
   const int rows = GU ? I : H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rbase = (blockIdx.x * kWarps + warp) * RPW;
+  // Programmatic dependent launch: the down projection may be launched while this
+  // gate/up grid runs; it waits for this grid's completion before it reads h.
+  if (GU) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  else asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int q0 = e >= 0 ? offsets[e] : T * k;
+  const int q1 = e >= 0 ? offsets[e + 1] : T * k + T;
+  if (q1 <= q0) return;
   if (rbase >= rows) return;
 
   const size_t mat = (size_t)H * I;
   const uint8_t* wmat[2];
   const uint16_t* smat[2] = {nullptr, nullptr};
-  if (WT == WT_INT4) {
+  const uint8_t* fmat[2] = {nullptr, nullptr};   // nvfp4 e4m3 block scales
+  float gmat[2] = {1.f, 1.f};                    // nvfp4 fp32 global scales
+  if (WT == WT_NVFP4) {
+    const uint8_t* sc = blob + 3 * mat / 2;
+    const float* gl = reinterpret_cast<const float*>(blob + 3 * mat / 2 + 3 * mat / 16);
+    if (GU) { wmat[0] = blob; wmat[1] = blob + mat / 2; fmat[0] = sc; fmat[1] = sc + mat / 16; gmat[0] = gl[0]; gmat[1] = gl[1]; }
+    else { wmat[0] = blob + mat; wmat[1] = nullptr; fmat[0] = sc + 2 * (mat / 16); gmat[0] = gl[2]; }
+  } else if (WT == WT_INT4) {
     const uint16_t* sc = reinterpret_cast<const uint16_t*>(blob + 3 * mat / 2);
     if (GU) { wmat[0] = blob; wmat[1] = blob + mat / 2; smat[0] = sc; smat[1] = sc + mat / 128; }
     else { wmat[0] = blob + mat; wmat[1] = nullptr; smat[0] = sc + 2 * (mat / 128); }
@@ -115,7 +157,7 @@ grouped_gemv_kernel(const void* __restrict__ xin, int T, int H, int I, int k,
     if (GU) { wmat[0] = blob; wmat[1] = blob + mat * es; }
     else { wmat[0] = blob + 2 * mat * es; wmat[1] = nullptr; }
   }
-  const size_t row_bytes = WT == WT_INT4 ? (size_t)K / 2 : (size_t)K * (WT == WT_F32 ? 4 : 2);
+  const size_t row_bytes = (WT == WT_INT4 || WT == WT_NVFP4) ? (size_t)K / 2 : (size_t)K * (WT == WT_F32 ? 4 : 2);
   bool rok[RPW];
 #pragma unroll
   for (int r = 0; r < RPW; ++r) rok[r] = rbase + r < rows;
@@ -152,8 +194,12 @@ grouped_gemv_kernel(const void* __restrict__ xin, int T, int H, int I, int k,
         for (int m = 0; m < NM; ++m) {
           const int rr = rok[r] ? rbase + r : rbase;
           wc[r][m] = ldw(wmat[m] + (size_t)rr * row_bytes +
-                         (WT == WT_INT4 ? kk / 2 : kk * (WT == WT_F32 ? 4 : 2)));
+                         ((WT == WT_INT4 || WT == WT_NVFP4) ? kk / 2 : kk * (WT == WT_F32 ? 4 : 2)));
           if (WT == WT_INT4) sc[r][m] = bf16_to_f32(__ldg(smat[m] + (size_t)rr * (K / 128) + kk / 128));
+          if (WT == WT_NVFP4) {   // the chunk's two block scales, packed in sc as raw bits
+            const uint16_t two = __ldg(reinterpret_cast<const unsigned short*>(fmat[m] + (size_t)rr * (K / 16) + kk / 16));
+            sc[r][m] = __uint_as_float((uint32_t)two);
+          }
         }
       float part[RPW][NM][NT];
 #pragma unroll
@@ -162,6 +208,95 @@ grouped_gemv_kernel(const void* __restrict__ xin, int T, int H, int I, int k,
         for (int m = 0; m < NM; ++m)
 #pragma unroll
           for (int t = 0; t < NT; ++t) part[r][m][t] = 0.f;
+      if constexpr (WT == WT_NVFP4) {
+        // e2m1 bytes -> f16x2 by the hardware conversion -> fp32; partial sums per
+        // 16-element block are scaled by that block's e4m3 scale.
+        float pb[RPW][NM][NT][2];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r)
+#pragma unroll
+          for (int m = 0; m < NM; ++m)
+#pragma unroll
+            for (int t = 0; t < NT; ++t) pb[r][m][t][0] = pb[r][m][t][1] = 0.f;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float xv[NT][8];
+#pragma unroll
+          for (int t = 0; t < NT; ++t)
+            if (t < nt) ldin<8, BF16IN>(in[t], kk + 8 * g, xv[t]);
+#pragma unroll
+          for (int r = 0; r < RPW; ++r)
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+              const uint32_t w = g == 0 ? wc[r][m].x : g == 1 ? wc[r][m].y : g == 2 ? wc[r][m].z : wc[r][m].w;
+              float wv[8];
+#pragma unroll
+              for (int b = 0; b < 4; ++b) e2m1x2_to_f32((w >> (8 * b)) & 0xFFu, wv[2 * b], wv[2 * b + 1]);
+#pragma unroll
+              for (int t = 0; t < NT; ++t)
+                if (t < nt) {
+#pragma unroll
+                  for (int j = 0; j < 8; ++j) pb[r][m][t][g >> 1] = fmaf(wv[j], xv[t][j], pb[r][m][t][g >> 1]);
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < RPW; ++r)
+#pragma unroll
+          for (int m = 0; m < NM; ++m) {
+            float s0, s1;
+            e4m3x2_to_f32(__float_as_uint(sc[r][m]), s0, s1);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) part[r][m][t] = s0 * pb[r][m][t][0] + s1 * pb[r][m][t][1];
+          }
+      } else if constexpr (WT == WT_INT4) {
+        // Packed dequant.  Nibbles n and n+4 of a word sit in the two 16-bit halves of
+        // (w >> 4n) & 0x000F000F; xor with 0x4308 per half makes the bf16 128 + (q + 8)
+        // (0x4300 is 128.0 in bf16, its last mantissa bit 1.0; xor 8 maps a 4-bit
+        // two's-complement q to q + 8).  Widening to fp32 and one packed add of -136
+        // give the pair (q_n, q_{n+4}) exactly; packed fp32 FMAs meet the matching x
+        // pairs.  About 3 lane instructions per weight instead of 5.
+        float2 acc2[RPW][NM][NT];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r)
+#pragma unroll
+          for (int m = 0; m < NM; ++m)
+#pragma unroll
+            for (int t = 0; t < NT; ++t) acc2[r][m][t] = make_float2(0.f, 0.f);
+        const float2 bias = make_float2(-136.f, -136.f);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float2 xp[NT][4];
+#pragma unroll
+          for (int t = 0; t < NT; ++t)
+            if (t < nt) {
+              float xv[8];
+              ldin<8, BF16IN>(in[t], kk + 8 * g, xv);
+#pragma unroll
+              for (int n = 0; n < 4; ++n) xp[t][n] = make_float2(xv[n], xv[n + 4]);
+            }
+#pragma unroll
+          for (int r = 0; r < RPW; ++r)
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+              const uint32_t w = g == 0 ? wc[r][m].x : g == 1 ? wc[r][m].y : g == 2 ? wc[r][m].z : wc[r][m].w;
+#pragma unroll
+              for (int n = 0; n < 4; ++n) {
+                const uint32_t v = ((w >> (4 * n)) & 0x000F000Fu) ^ 0x43084308u;
+                const float2 q2 = __fadd2_rn(make_float2(bf16lo(v), bf16hi(v)), bias);
+#pragma unroll
+                for (int t = 0; t < NT; ++t)
+                  if (t < nt) acc2[r][m][t] = __ffma2_rn(q2, xp[t][n], acc2[r][m][t]);
+              }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < RPW; ++r)
+#pragma unroll
+          for (int m = 0; m < NM; ++m)
+#pragma unroll
+            for (int t = 0; t < NT; ++t) part[r][m][t] = acc2[r][m][t].x + acc2[r][m][t].y;
+      } else {
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
         float wv[RPW][NM][GE];
@@ -183,6 +318,7 @@ grouped_gemv_kernel(const void* __restrict__ xin, int T, int H, int I, int k,
           }
         }
       }
+      }
 #pragma unroll
       for (int r = 0; r < RPW; ++r)
 #pragma unroll
@@ -196,8 +332,8 @@ grouped_gemv_kernel(const void* __restrict__ xin, int T, int H, int I, int k,
     for (int r = 0; r < RPW; ++r)
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
-        float a0 = warp_sum(acc[r][0][t]);
-        float a1 = GU ? warp_sum(acc[r][NM - 1][t]) : 0.f;
+        const float a0 = warp_sum(acc[r][0][t]) * gmat[0];
+        const float a1 = GU ? warp_sum(acc[r][NM - 1][t]) * gmat[NM - 1] : 0.f;
         if (lane == 0 && rok[r] && t < nt) {
           const int q = c + t;
           if (GU) hbuf[(size_t)q * I + rbase + r] = silu(a0) * a1;
@@ -207,18 +343,36 @@ grouped_gemv_kernel(const void* __restrict__ xin, int T, int H, int I, int k,
   }
 }
 
+// Launches `kern`; with `dependent`, as a programmatic dependent launch of the
+// previous kernel on the stream (it may start before that kernel completes and must
+// order itself with griddepcontrol.wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, cudaStream_t s, bool dependent,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 template <int MODE, int WT, int RPW>
 cudaError_t launch_gemv(int nt_max, dim3 grid, cudaStream_t s, const void* x, int T, int H, int I, int k,
                         const ExpertList& list, const int* offsets, const int* perm, float* h, float* y) {
 #define FT_GEMV_CASE(NTV)                                                                  \
   {                                                                                        \
-    grouped_gemv_kernel<MODE, WT, NTV, RPW><<<grid, kThreads, 0, s>>>(x, T, H, I, k, list, \
-                                                                     offsets, perm, h, y); \
-    return cudaGetLastError();                                                             \
+    return launch_pdl(grouped_gemv_kernel<MODE, WT, NTV, RPW>, grid, dim3(kThreads), s,    \
+                      MODE == MODE_DOWN, x, T, H, I, k, list, offsets, perm, h, y);        \
   }
   if (nt_max <= 1) FT_GEMV_CASE(1)
-  if (nt_max <= 2) FT_GEMV_CASE(2)
-  if (nt_max <= 4) FT_GEMV_CASE(4)
+  if (nt_max <= 2 || FT_GEMV_NT_MAX <= 2) FT_GEMV_CASE(2)
+  if (nt_max <= 4 || FT_GEMV_NT_MAX <= 4) FT_GEMV_CASE(4)
   FT_GEMV_CASE(8)
 #undef FT_GEMV_CASE
 }
@@ -228,6 +382,7 @@ template <bool OUT_BF16>
 __global__ void combine_kernel(const float* __restrict__ y, const float* __restrict__ gates,
                                const int* __restrict__ inv, int T, int H, int k, int has_shared,
                                void* __restrict__ out) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int per_tok = H / 4;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long long)T * per_tok) return;
@@ -253,12 +408,7 @@ __global__ void combine_kernel(const float* __restrict__ y, const float* __restr
   }
 }
 
-int g_decode_mode = 1;   // FT_DECODE_GEMV_REGISTER: faster on the measured decode shapes
-int g_num_sms = 0;
-
 }  // namespace
-
-void set_decode_gemv_mode(int mode) { g_decode_mode = mode; }
 
 cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdtype,
                               const ExpertList& list, int max_pairs_per_expert, const int* offsets,
@@ -267,30 +417,29 @@ cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdt
   if (list.n <= 0 || T <= 0) return cudaSuccess;
   int nt = max_pairs_per_expert < T ? max_pairs_per_expert : T;
   if (nt < 1) nt = 1;
-  int nt_all = nt;                        // the shared expert's entry owns all T tokens
-  for (int i = 0; i < list.n; ++i)
-    if (list.expert[i] < 0 && T > nt_all) nt_all = T;
-  if (g_decode_mode == 0 && nt_all <= 8 && tma_gemv_supported(H, I, wdtype)) {
-    if (g_num_sms <= 0) {
-      int dev = 0;
-      cudaGetDevice(&dev);
-      cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    }
-    return launch_ffn_decode_tma(x, T, H, I, k, wdtype, list, nt_all, offsets, perm, h, y, err, g_num_sms, s,
-                                 between);
-  }
-  constexpr int RPW_GU = 2, RPW_D = 4;
+  (void)err;
+  // rows per warp: two gate/up row pairs or four down rows (int4: half, for registers)
+  const bool i4 = wdtype == WT_INT4;
+  constexpr int RPW_GU = FT_GEMV_GU_RPW, RPW_D = FT_GEMV_D_RPW;
   dim3 g1((I + kWarps * RPW_GU - 1) / (kWarps * RPW_GU), list.n);
   dim3 g2((H + kWarps * RPW_D - 1) / (kWarps * RPW_D), list.n);
   cudaError_t e;
-#define FT_FFN(WTV)                                                                                   \
-  e = launch_gemv<MODE_GATE_UP, WTV, RPW_GU>(nt, g1, s, x, T, H, I, k, list, offsets, perm, h, y);    \
-  if (e != cudaSuccess) return e;                                                                     \
-  if (between) cudaEventRecord(between, s);                                                          \
-  return launch_gemv<MODE_DOWN, WTV, RPW_D>(nt, g2, s, x, T, H, I, k, list, offsets, perm, h, y);
-  if (wdtype == WT_F32) { FT_FFN(WT_F32) }
-  if (wdtype == WT_BF16) { FT_FFN(WT_BF16) }
-  FT_FFN(WT_INT4)
+#define FT_FFN(WTV, GUR, DR)                                                                          \
+  {                                                                                                   \
+    dim3 ga((I + kWarps * GUR - 1) / (kWarps * GUR), list.n);                                          \
+    dim3 gb((H + kWarps * DR - 1) / (kWarps * DR), list.n);                                            \
+    e = launch_gemv<MODE_GATE_UP, WTV, GUR>(nt, ga, s, x, T, H, I, k, list, offsets, perm, h, y);     \
+    if (e != cudaSuccess) return e;                                                                   \
+    if (between) cudaEventRecord(between, s);                                                        \
+    return launch_gemv<MODE_DOWN, WTV, DR>(nt, gb, s, x, T, H, I, k, list, offsets, perm, h, y);      \
+  }
+  (void)i4;
+  (void)g1;
+  (void)g2;
+  if (wdtype == WT_F32) FT_FFN(WT_F32, RPW_GU, RPW_D)
+  if (wdtype == WT_BF16) FT_FFN(WT_BF16, RPW_GU, RPW_D)
+  if (wdtype == WT_NVFP4) FT_FFN(WT_NVFP4, 1, 2)
+  FT_FFN(WT_INT4, 1, 2)
 #undef FT_FFN
 }
 
@@ -301,9 +450,11 @@ cudaError_t launch_combine(const float* y, const float* gates, const int* inv, i
   const int threads = 256;
   const unsigned blocks = (unsigned)((n + threads - 1) / threads);
   if (out_bf16)
-    combine_kernel<true><<<blocks, threads, 0, s>>>(y, gates, inv, T, H, k, has_shared, out);
+    return launch_pdl(combine_kernel<true>, dim3(blocks), dim3(threads), s, true, y, gates, inv, T, H, k,
+                      (int)has_shared, out);
   else
-    combine_kernel<false><<<blocks, threads, 0, s>>>(y, gates, inv, T, H, k, has_shared, out);
+    return launch_pdl(combine_kernel<false>, dim3(blocks), dim3(threads), s, true, y, gates, inv, T, H, k,
+                      (int)has_shared, out);
   return cudaGetLastError();
 }
 

@@ -41,15 +41,6 @@ cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdt
                               const ExpertList& list, int max_pairs_per_expert, const int* offsets,
                               const int* perm, float* h, float* y, cudaStream_t s,
                               cudaEvent_t between = nullptr, int* err = nullptr);
-// K3 (decode) with the weights streamed into shared memory by bulk copies (TMA);
-// same results as launch_ffn_decode.  Up to 8 pairs per entry.
-bool tma_gemv_supported(int H, int I, int wdtype);
-cudaError_t launch_ffn_decode_tma(const void* x, int T, int H, int I, int k, int wdtype, const ExpertList& list,
-                                  int nt, const int* offsets, const int* perm, float* h, float* y, int* err,
-                                  int num_sms, cudaStream_t s, cudaEvent_t between);
-// Decode GEMV selection (process-wide): 0 = bulk-copy kernel where supported, 1 = the
-// register-streaming kernel.
-void set_decode_gemv_mode(int mode);
 // K5: out[t] = sum_j gates[t][j] * y[inv[t*k+j]] (ascending j) + y[T*k+t] if has_shared.
 cudaError_t launch_combine(const float* y, const float* gates, const int* inv, int T, int H, int k,
                            bool has_shared, bool out_bf16, void* out, cudaStream_t s);

@@ -51,8 +51,8 @@ extern "C" int ft_expert_ffn_decode_noalloc(const void* x, int T, int H, int I, 
                                             const float* gates, const int* inv, int has_shared, void* out,
                                             void* stream) {
   if (T < 0 || H < 8 || I < 8 || H % 8 || I % 8 || top_k < 1 || n_list < 0 ||
-      n_list > ftk::kMaxList || wdtype < FT_W_F32 || wdtype > FT_W_INT4_G128 ||
-      (wdtype == FT_W_INT4_G128 && (H % 128 || I % 128)) ||
+      n_list > ftk::kMaxList || wdtype < FT_W_F32 || wdtype > FT_W_NVFP4 ||
+      (wdtype == FT_W_INT4_G128 && (H % 128 || I % 128)) || (wdtype == FT_W_NVFP4 && (H % 32 || I % 32)) ||
       (T > 0 && (!x || !offsets || !perm || !gates || !inv || !out)) ||
       (n_list > 0 && (!blobs || !experts))) {
     ftk::set_step_error("ft_expert_ffn_decode_noalloc: invalid argument");

@@ -45,6 +45,41 @@ def dequant_int4(packed: np.ndarray, scale_bits: np.ndarray) -> np.ndarray:
     return q * np.repeat(s, 128, axis=1)
 
 
+def decode_e2m1(codes: np.ndarray) -> np.ndarray:
+    """FP4 E2M1 codes (0..15) -> float64.  Bit 3 sign, bits 2-1 exponent (bias 1), bit 0
+    mantissa; exponent 0 is subnormal: m * 0.5.  (The OCP microscaling FP4 element.)"""
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where(c & 8, -1.0, 1.0)
+    e = (c >> 1) & 3
+    m = c & 1
+    mag = np.where(e == 0, m * 0.5, (1.0 + m * 0.5) * np.power(2.0, e - 1))
+    return sign * mag
+
+
+def decode_e4m3(codes: np.ndarray) -> np.ndarray:
+    """FP8 E4M3 codes -> float64.  Bit 7 sign, bits 6-3 exponent (bias 7), bits 2-0
+    mantissa; exponent 0 is subnormal: m/8 * 2^-6; no infinities (0x7F/0xFF are NaN)."""
+    c = np.asarray(codes, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 15
+    m = c & 7
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.power(2.0, e - 7))
+    mag = np.where((c & 0x7F) == 0x7F, np.nan, mag)
+    return sign * mag
+
+
+def dequant_nvfp4(packed: np.ndarray, scale_codes: np.ndarray, g: float) -> np.ndarray:
+    """w = e2m1(q) * e4m3(s) * g, s shared by 16 consecutive reduction-axis elements
+    of a row (READING of the pages' NVFP4 release: the 16-element micro-block with an
+    E4M3 scale and an FP32 tensor scale; element 2b in the low nibble of byte b)."""
+    p = np.asarray(packed, dtype=np.uint8)
+    codes = np.empty((p.shape[0], p.shape[1] * 2), dtype=np.int64)
+    codes[:, 0::2] = p & 0x0F
+    codes[:, 1::2] = p >> 4
+    s = decode_e4m3(scale_codes)
+    return decode_e2m1(codes) * np.repeat(s, 16, axis=1) * float(g)
+
+
 def expert_weights(blob: np.ndarray, wdtype: str, H: int, I: int):
     """Decode one expert blob into (W_gate [I,H], W_up [I,H], W_down [H,I]) float64.
 
@@ -52,7 +87,8 @@ def expert_weights(blob: np.ndarray, wdtype: str, H: int, I: int):
     stores experts "in runtime layout" without giving it - FreeToken linux,
     setup, "prepare the model weights"): the three matrices row-major, gate,
     up, down; for int4, the three packed matrices and then their three scale
-    arrays.
+    arrays; for nvfp4, the three packed e2m1 matrices, their three e4m3 block-scale
+    arrays and the three fp32 global scales.
     """
     blob = np.asarray(blob, dtype=np.uint8).reshape(-1)
     m = H * I
@@ -62,6 +98,15 @@ def expert_weights(blob: np.ndarray, wdtype: str, H: int, I: int):
     if wdtype == "bf16":
         w = widen_bf16(blob.view(np.uint16))
         return w[:m].reshape(I, H), w[m:2 * m].reshape(I, H), w[2 * m:3 * m].reshape(H, I)
+    if wdtype == "nvfp4":
+        q = blob[:3 * m // 2]
+        s = blob[3 * m // 2:3 * m // 2 + 3 * m // 16]
+        g = blob[3 * m // 2 + 3 * m // 16:3 * m // 2 + 3 * m // 16 + 12].view(np.float32).astype(np.float64)
+        n = m // 16
+        wg = dequant_nvfp4(q[:m // 2].reshape(I, H // 2), s[:n].reshape(I, H // 16), g[0])
+        wu = dequant_nvfp4(q[m // 2:m].reshape(I, H // 2), s[n:2 * n].reshape(I, H // 16), g[1])
+        wd = dequant_nvfp4(q[m:3 * m // 2].reshape(H, I // 2), s[2 * n:3 * n].reshape(H, I // 16), g[2])
+        return wg, wu, wd
     if wdtype == "int4":
         q = blob[:3 * m // 2]
         s = blob[3 * m // 2:].view(np.uint16)

@@ -32,7 +32,8 @@ def run_workload(*, L: int, E: int, H: int, I: int, k: int, gating: str, wdtype:
     filled on each miss instead of from the pool (same result by construction of
     the method - a check that the trace's slots hold the right experts).
 
-    Returns dict(ids [steps,L,B,k], gates, gap, trace, stats, out {(s,l): [B,H]}).
+    Returns dict(ids [steps,L,B,k], gates, gap, zsel (the selected logits, in id order),
+    trace, stats, out {(s,l): [B,H]}).
     """
     steps, B, _ = x_steps.shape
     lru = SharedLru(capacity)
@@ -40,6 +41,7 @@ def run_workload(*, L: int, E: int, H: int, I: int, k: int, gating: str, wdtype:
     ids_all = np.zeros((steps, L, B, k), dtype=np.int32)
     g_all = np.zeros((steps, L, B, k))
     gap_all = np.zeros((steps, L, B))
+    zsel_all = np.zeros((steps, L, B, k))
     outs = {}
     routers = {l: router_of(l) for l in range(L)}
     arena = {}
@@ -61,6 +63,7 @@ def run_workload(*, L: int, E: int, H: int, I: int, k: int, gating: str, wdtype:
             call = s * L + l
             r = moe.route(x, routers[l], k, gating)
             ids_all[s, l], g_all[s, l], gap_all[s, l] = r["ids"], r["gates"], r["gap"]
+            zsel_all[s, l] = np.take_along_axis(r["z"], r["ids"].astype(np.int64), axis=1)
             if prefill and l == 0:
                 fill(lru.access_set(call, 0, range(E), PREFETCH))
             fill(lru.access_set(call, l, moe.selected_set(r["ids"]), ROUTED))
@@ -74,5 +77,5 @@ def run_workload(*, L: int, E: int, H: int, I: int, k: int, gating: str, wdtype:
                 sh = shared_of(l) if shared_of is not None else None
                 outs[(s, l)] = moe.experts_and_combine(x, r["ids"], r["gates"], E, wdtype, H, I,
                                                        get, sh)
-    return {"ids": ids_all, "gates": g_all, "gap": gap_all, "trace": lru.trace,
+    return {"ids": ids_all, "gates": g_all, "gap": gap_all, "zsel": zsel_all, "trace": lru.trace,
             "stats": lru.stats, "out": outs, "lru": lru}

@@ -19,7 +19,7 @@ _LIB = os.path.join(_HERE, "libsynth.so")
 _lock = threading.Lock()
 _lib = None
 
-W_CODE = {"f32": 0, "bf16": 1, "int4": 2}
+W_CODE = {"f32": 0, "bf16": 1, "int4": 2, "nvfp4": 3}
 T_TOKENS, T_AR1, T_ROUTER = 8, 9, 4
 
 
@@ -43,6 +43,7 @@ def lib():
             L.synth_normal_f32.argtypes = [u64, i32, i32, i32, u64, u64, f32, vp]
             L.synth_round_bf16.argtypes = [vp, u64, vp]
             L.synth_quantise_int4.argtypes = [vp, i32, i32, vp, vp]
+            L.synth_quantise_nvfp4_rows.argtypes = [vp, i32, i32, f32, vp, vp]
             L.synth_blob_bytes.argtypes = [i32, i32, i32]
             L.synth_blob_bytes.restype = u64
             L.synth_expert_blob.argtypes = [u64, i32, i32, i32, i32, i32, i32, f32, vp]
@@ -79,6 +80,17 @@ def quantise_int4(w: np.ndarray):
     q = np.empty((R, K // 2), dtype=np.uint8)
     s = np.empty((R, K // 128), dtype=np.uint16)
     lib().synth_quantise_int4(_ptr(w), R, K, _ptr(q), _ptr(s))
+    return q, s
+
+
+def quantise_nvfp4(w: np.ndarray, g: float):
+    """nvfp4 quantiser for rows of w with global scale g: (packed e2m1 [R, K/2], e4m3 codes [R, K/16])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    R, K = w.shape
+    assert K % 16 == 0
+    q = np.empty((R, K // 2), dtype=np.uint8)
+    s = np.empty((R, K // 16), dtype=np.uint8)
+    lib().synth_quantise_nvfp4_rows(_ptr(w), R, K, g, _ptr(q), _ptr(s))
     return q, s
 
 
@@ -147,5 +159,5 @@ def tokens(cfg: MoeConfig, batch: int):
     return x, None
 
 
-__all__ = ["MoeConfig", "CONFIGS", "build", "lib", "normal_f32", "round_bf16", "quantise_int4",
+__all__ = ["MoeConfig", "CONFIGS", "build", "lib", "normal_f32", "round_bf16", "quantise_int4", "quantise_nvfp4",
            "expert_weights_f32", "expert_blob", "fill_pool", "router_weights", "ar1_chain", "tokens"]

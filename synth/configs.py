@@ -21,7 +21,7 @@ class MoeConfig:
     I: int            # SwiGLU intermediate size
     k: int            # top-k
     gating: str       # "softmax" (renormalised over the k selected) or "sigmoid" (normalised over the k)
-    wdtype: str       # "f32", "bf16" or "int4" (g128, bf16 scales)
+    wdtype: str       # "f32", "bf16", "int4" (g128, bf16 scales) or "nvfp4" (e2m1, e4m3 per 16, fp32 global)
     shared: bool      # one always-on shared expert per layer, gate weight 1
     C: int            # cache slots (shared across all layers)
     tokens: int       # tokens in the whole run
@@ -43,6 +43,8 @@ class MoeConfig:
             return 4 * n
         if self.wdtype == "bf16":
             return 2 * n
+        if self.wdtype == "nvfp4":
+            return n // 2 + n // 16 + 16
         return n // 2 + 2 * (n // 128)
 
     @property

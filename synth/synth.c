@@ -21,6 +21,14 @@
  *                128 consecutive reduction-axis elements of a row.
  *   The int4 quantiser (data preparation, run once): s = bf16_rne(max|w|/7),
  *   q = 0 if s == 0 else clamp(rint(w/s), -8, 7) with ties to even.
+ *   nvfp4      : Q_gate [I][H/2], Q_up [I][H/2], Q_down [H][I/2] (e2m1 nibbles, element
+ *                2b in the low nibble of byte b), then e4m3 block scales S_gate [I][H/16],
+ *                S_up [I][H/16], S_down [H][I/16] (one byte per 16 consecutive reduction-
+ *                axis elements), then the fp32 global scales g_gate, g_up, g_down and 4
+ *                zero bytes.  w = e2m1(q) * e4m3(s) * g.
+ *   The nvfp4 quantiser: g = max|W| / (448 * 6) (1 if W is zero); per block of 16,
+ *   s = e4m3_rne(max|w| / 6 / g); q = e2m1_rne(w / (s * g)) (0 if s = 0), both with
+ *   ties to even and saturation (448, 6).
  */
 #define _GNU_SOURCE
 #include <math.h>
@@ -34,7 +42,7 @@
 
 #define SYNTH_API __attribute__((visibility("default")))
 
-enum { SYN_W_F32 = 0, SYN_W_BF16 = 1, SYN_W_INT4 = 2 };
+enum { SYN_W_F32 = 0, SYN_W_BF16 = 1, SYN_W_INT4 = 2, SYN_W_NVFP4 = 3 };
 enum {
   SYN_T_WGATE = 1, SYN_T_WUP = 2, SYN_T_WDOWN = 3, SYN_T_ROUTER = 4,
   SYN_T_SH_GATE = 5, SYN_T_SH_UP = 6, SYN_T_SH_DOWN = 7,
@@ -212,6 +220,62 @@ SYNTH_API void synth_quantise_int4(const float* w, int rows, int K, uint8_t* q, 
   }
 }
 
+/* e2m1 (FP4) code of a real value: nearest of {0,.5,1,1.5,2,3,4,6} (ties to the even
+ * mantissa), saturating at 6; bit 3 is the sign. */
+static uint8_t e2m1_rne(float v) {
+  static const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+  uint8_t sgn = v < 0.f ? 8 : 0;
+  float a = fabsf(v);
+  int best = 0;
+  for (int c = 1; c < 8; ++c) {
+    float d = fabsf(a - mag[c]), db = fabsf(a - mag[best]);
+    if (d < db || (d == db && (c & 1) == 0)) best = c;
+  }
+  return (uint8_t)(sgn | best);
+}
+
+/* e4m3 (FP8, bias 7, no infinities, max 448) code of a non-negative value, round to
+ * nearest even, saturating at 448. */
+static uint8_t e4m3_rne(float v) {
+  if (!(v > 0.f)) return 0;
+  if (v >= 448.f) return 0x7E;
+  int best = 0;
+  float bestd = v;
+  for (int c = 1; c <= 0x7E; ++c) {
+    int e = c >> 3, m = c & 7;
+    float val = e == 0 ? ldexpf((float)m, -9) : ldexpf(1.f + m / 8.f, e - 7);
+    float d = fabsf(v - val);
+    if (d < bestd || (d == bestd && (c & 1) == 0)) { best = c; bestd = d; }
+  }
+  return (uint8_t)best;
+}
+
+static float e4m3_value(uint8_t c) {
+  int e = (c >> 3) & 15, m = c & 7;
+  return e == 0 ? ldexpf((float)m, -9) : ldexpf(1.f + m / 8.f, e - 7);
+}
+
+/* nvfp4 quantiser for one matrix [rows][K] (K % 16 == 0) given its global scale g. */
+SYNTH_API void synth_quantise_nvfp4_rows(const float* w, int rows, int K, float g, uint8_t* q, uint8_t* scales) {
+  const float e2m1_mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+  (void)e2m1_mag;
+  for (int r = 0; r < rows; ++r) {
+    const float* wr = w + (size_t)r * K;
+    for (int b = 0; b < K / 16; ++b) {
+      float amax = 0.f;
+      for (int j = 0; j < 16; ++j) { float a = fabsf(wr[b * 16 + j]); if (a > amax) amax = a; }
+      uint8_t sc = e4m3_rne(amax / 6.0f / g);
+      scales[(size_t)r * (K / 16) + b] = sc;
+      float s = e4m3_value(sc) * g;
+      for (int j = 0; j < 16; j += 2) {
+        uint8_t c0 = s > 0.f ? e2m1_rne(wr[b * 16 + j] / s) : 0;
+        uint8_t c1 = s > 0.f ? e2m1_rne(wr[b * 16 + j + 1] / s) : 0;
+        q[(size_t)r * (K / 2) + (b * 16 + j) / 2] = (uint8_t)(c0 | (c1 << 4));
+      }
+    }
+  }
+}
+
 /* One matrix [rows][cols] of tensor id `tensor` in the blob's element format. */
 static void write_matrix(uint64_t seed, int tensor, int layer, int expert, int rows, int cols,
                          int wdtype, float sigma, uint8_t* dst_w, uint16_t* dst_s, float* scratch) {
@@ -235,7 +299,24 @@ SYNTH_API uint64_t synth_blob_bytes(int H, int I, int wdtype) {
   uint64_t n = 3ull * H * I;
   if (wdtype == SYN_W_F32) return n * 4;
   if (wdtype == SYN_W_BF16) return n * 2;
+  if (wdtype == SYN_W_NVFP4) return n / 2 + n / 16 + 16;
   return n / 2 + (n / 128) * 2;
+}
+
+/* nvfp4 matrix: two passes over the draws (the global scale needs the matrix maximum). */
+static void write_matrix_nvfp4(uint64_t seed, int tensor, int layer, int expert, int rows, int cols, float sigma,
+                               uint8_t* q, uint8_t* sc, float* g_out, float* scratch) {
+  float amax = 0.f;
+  for (int r = 0; r < rows; ++r) {
+    synth_normal_f32(seed, tensor, layer, expert, (uint64_t)r * cols, cols, sigma, scratch);
+    for (int c = 0; c < cols; ++c) { float a = fabsf(scratch[c]); if (a > amax) amax = a; }
+  }
+  float g = amax > 0.f ? amax / (448.0f * 6.0f) : 1.0f;
+  *g_out = g;
+  for (int r = 0; r < rows; ++r) {
+    synth_normal_f32(seed, tensor, layer, expert, (uint64_t)r * cols, cols, sigma, scratch);
+    synth_quantise_nvfp4_rows(scratch, 1, cols, g, q + (size_t)r * (cols / 2), sc + (size_t)r * (cols / 16));
+  }
 }
 
 /* Writes one expert blob.  shared != 0 selects the always-on shared expert of `layer`. */
@@ -245,9 +326,21 @@ SYNTH_API int synth_expert_blob(uint64_t seed, int layer, int expert, int shared
       td = shared ? SYN_T_SH_DOWN : SYN_T_WDOWN;
   int ex = shared ? 0 : expert;
   if (wdtype == SYN_W_INT4 && ((H % 128) || (I % 128))) return -1;
+  if (wdtype == SYN_W_NVFP4 && ((H % 32) || (I % 32))) return -1;
   float* scratch = (float*)malloc(sizeof(float) * (size_t)(H > I ? H : I));
   if (!scratch) return -2;
   uint64_t mat = (uint64_t)H * I;
+  if (wdtype == SYN_W_NVFP4) {
+    uint8_t* q = dst;
+    uint8_t* sc = dst + 3 * mat / 2;
+    float g[4] = {0.f, 0.f, 0.f, 0.f};
+    write_matrix_nvfp4(seed, tg, layer, ex, I, H, sigma, q, sc, &g[0], scratch);
+    write_matrix_nvfp4(seed, tu, layer, ex, I, H, sigma, q + mat / 2, sc + mat / 16, &g[1], scratch);
+    write_matrix_nvfp4(seed, td, layer, ex, H, I, sigma, q + mat, sc + 2 * (mat / 16), &g[2], scratch);
+    memcpy(dst + 3 * mat / 2 + 3 * mat / 16, g, 16);
+    free(scratch);
+    return 0;
+  }
   if (wdtype == SYN_W_INT4) {
     uint8_t* q = dst;
     uint16_t* s = (uint16_t*)(dst + 3 * mat / 2);

@@ -142,22 +142,14 @@ def test_permute_parity(T, k, E):
         assert np.array_equal(inv.cpu().numpy(), np.argsort(p))
 
 
-@pytest.mark.parametrize("gemv_mode", [0, 1])
 @pytest.mark.parametrize("wd,H,I,T,E,k,shared", [
     ("f32", 256, 128, 1, 16, 2, False), ("f32", 256, 128, 20, 4, 2, True),
     ("bf16", 2048, 768, 1, 128, 8, False), ("bf16", 2048, 768, 3, 16, 8, True),
     ("bf16", 1024, 512, 37, 6, 3, True), ("int4", 1024, 512, 1, 16, 4, False),
     ("int4", 7168, 2048, 2, 8, 8, False), ("int4", 1024, 256, 19, 5, 2, True),
+    ("nvfp4", 2048, 768, 1, 16, 8, False), ("nvfp4", 1024, 512, 3, 8, 4, True), ("nvfp4", 256, 96, 12, 4, 2, True),
 ])
-def test_expert_ffn_and_combine_parity(wd, H, I, T, E, k, shared, gemv_mode):
-    ft.ft_set_decode_gemv(gemv_mode)      # bulk-copy kernel (where supported) or register kernel
-    try:
-        _ffn_and_combine_case(wd, H, I, T, E, k, shared)
-    finally:
-        ft.ft_set_decode_gemv(ft.FT_DECODE_GEMV_REGISTER)
-
-
-def _ffn_and_combine_case(wd, H, I, T, E, k, shared):
+def test_expert_ffn_and_combine_parity(wd, H, I, T, E, k, shared):
     cfg = synth.MoeConfig("t", 1, E, H, I, k, "sigmoid", wd, shared, E, T, (T,), "iid", "decode")
     rng = np.random.default_rng(H + T)
     ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
@@ -225,7 +217,7 @@ def _run_gpu(stack, x, steps, sample=None, stream=None, routing=True, resize_at=
 
 
 def _check_run(cfg, stack, vals, outs, ids, ref, steps):
-    div = first_divergence(ids, ref["ids"][:steps], ref["gap"][:steps])
+    div = first_divergence(ids, ref["ids"][:steps], ref["gap"][:steps], ref.get("zsel"))
     last = steps if div is None else div // (cfg.L * vals.shape[1])
     tr = stack.trace()
     want = trace_tuples(ref["trace"])
@@ -349,6 +341,16 @@ def test_prefill_policy_small():
         _check_run(cfg, st, vals, outs, ids, ref, 1)
         s = st.stats()
         assert s["misses"] == 0 and s["prefetch_misses"] == 3 * 16
+
+
+def test_nvfp4_stack_decode_forward_parity():
+    cfg = synth.MoeConfig("nvfp4-small", L=2, E=32, H=1024, I=512, k=4, gating="softmax", wdtype="nvfp4",
+                          shared=False, C=24, tokens=16, batches=(1,), process="ar1", mode="decode")
+    with GpuStack(cfg) as st:
+        vals, x = st.tokens(1)
+        outs, ids = _run_gpu(st, x, cfg.tokens)
+        ref = oracle_run(cfg, st, vals)
+        _check_run(cfg, st, vals, outs, ids, ref, cfg.tokens)
 
 
 def test_forwards_on_alternating_streams():

@@ -214,6 +214,7 @@ def _dense_brute_force(x, Wr, k, gating, weights):
     (8, 8, 6, 3, "sigmoid", "bf16"),
     (4, 6, 2, 4, "softmax", "bf16"),
     (4, 128, 128, 2, "sigmoid", "int4"),
+    (4, 64, 32, 2, "softmax", "nvfp4"),
 ])
 def test_sparse_layer_equals_dense_brute_force(E, H, I, k, gating, wd):
     cfg = synth.MoeConfig("t", 1, E, H, I, k, gating, wd, False, E, 5, (5,), "iid", "decode")
@@ -226,10 +227,10 @@ def test_sparse_layer_equals_dense_brute_force(E, H, I, k, gating, wd):
         if wd == "bf16":
             widen = lambda a: (synth.round_bf16(a).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
             fg, fu, fd = widen(fg), widen(fu), widen(fd)
-        elif wd == "int4":
+        elif wd in ("int4", "nvfp4"):
             fg, fu, fd = moe.expert_weights(blobs[e], wd, H, I)   # dequant pinned separately
         weights.append((np.asarray(fg, np.float64), np.asarray(fu, np.float64), np.asarray(fd, np.float64)))
-    if wd == "int4":
+    if wd in ("int4", "nvfp4"):
         x = x[:2]
     r = moe.moe_layer(x, Wr, k, gating, wd, H, I, lambda e: blobs[e])
     ref = _dense_brute_force(x, Wr, k, gating, weights)
@@ -381,3 +382,58 @@ def test_shared_expert_adds_with_weight_one():
     shared_direct = (u * scipy.special.expit(u) * v) @ fd.T
     assert np.allclose(with_sh - without, shared_direct, rtol=1e-10, atol=1e-14)
     assert not np.array_equal(sh, blobs[0])
+
+
+def test_fp4_fp8_decoders_golden():
+    n4 = n8 = 0
+    for f in _golden_lines("int4_bf16_formats.txt"):
+        if f[0] == "e2m1":
+            v = moe.decode_e2m1(np.array([int(f[1])]))[0]
+            assert v == float(f[2]) and np.signbit(v) == f[2].startswith("-")
+            n4 += 1
+        elif f[0] == "e4m3":
+            assert moe.decode_e4m3(np.array([int(f[1], 16)]))[0] == float(f[2])
+            n8 += 1
+    assert n4 == 16 and n8 >= 8
+    assert np.isnan(moe.decode_e4m3(np.array([0x7F]))[0])
+
+
+def test_nvfp4_roundtrip_is_nearest_grid_point():
+    # brute force: every dequantised element is the grid value e2m1 * (block scale) nearest
+    # to the draw (saturating at 6 * scale), the block scale is the e4m3 value nearest to
+    # max|w| / 6 / g
+    rng = np.random.default_rng(12)
+    w = (rng.standard_normal((8, 64)) * 0.02).astype(np.float32)
+    w[2, :16] = 0.0
+    g = float(np.float32(np.abs(w).max() / (448 * 6)))
+    q, s = synth.quantise_nvfp4(w, g)
+    deq = moe.dequant_nvfp4(q, s, g)
+    grid = moe.decode_e2m1(np.arange(16))
+    e4 = moe.decode_e4m3(np.arange(0x7F))
+    for r in range(8):
+        for b in range(4):
+            blk = w[r, 16 * b:16 * b + 16].astype(np.float64)
+            want_s = e4[np.argmin(np.abs(e4 - np.float32(np.abs(blk).max() / 6.0 / np.float32(g))))]
+            sc = moe.decode_e4m3(s[r, b:b + 1])[0]
+            assert sc == want_s
+            step = sc * g
+            for j in range(16):
+                if step == 0:
+                    assert deq[r, 16 * b + j] == 0.0
+                    continue
+                dist = np.abs(blk[j] / np.float32(step) - grid)
+                assert abs(deq[r, 16 * b + j] / step - grid[np.argmin(dist)]) < 1e-12 or \
+                    abs(dist[np.argmin(dist)] - np.sort(dist)[1]) < 1e-6     # a tie: either neighbour
+
+
+def test_nvfp4_blob_layout_matches_draws():
+    cfg = synth.MoeConfig("t", 1, 2, 64, 32, 1, "softmax", "nvfp4", False, 1, 1, (1,), "iid", "decode")
+    blob = synth.expert_blob(cfg, 0, 1)
+    assert blob.nbytes == cfg.blob_bytes
+    wg, wu, wd = moe.expert_weights(blob, "nvfp4", 64, 32)
+    fg, fu, fd = synth.expert_weights_f32(cfg, 0, 1)
+    for a, b in ((wg, fg), (wu, fu), (wd, fd)):
+        assert a.shape == b.shape
+        # within half the largest grid step (2 * block scale * g) of the draw
+        assert np.max(np.abs(a - b)) <= np.abs(b).max() / 6 * 1.1
+        assert np.corrcoef(a.reshape(-1), b.reshape(-1))[0, 1] > 0.98
