@@ -410,36 +410,58 @@ __global__ void combine_kernel(const float* __restrict__ y, const float* __restr
 
 }  // namespace
 
+// Rows per warp for one matrix pass: enough rows that a warp streams about
+// FT_GEMV_WARP_BYTES of weights (short rows need several), at most 8.
+#ifndef FT_GEMV_WARP_BYTES
+#define FT_GEMV_WARP_BYTES 16384
+#endif
+static int rows_per_warp(size_t row_bytes_all_matrices, int cap) {
+  int r = 1;
+  while (r < cap && (size_t)(2 * r) * row_bytes_all_matrices <= FT_GEMV_WARP_BYTES) r *= 2;
+  return r;
+}
+
+template <int MODE, int WT>
+static cudaError_t launch_pass(int nt, int rpw, int rows, cudaStream_t s, const void* x, int T, int H, int I, int k,
+                               const ExpertList& list, const int* offsets, const int* perm, float* h, float* y) {
+  auto grid = [&](int r) { return dim3((rows + kWarps * r - 1) / (kWarps * r), list.n); };
+  switch (rpw) {
+    case 1: return launch_gemv<MODE, WT, 1>(nt, grid(1), s, x, T, H, I, k, list, offsets, perm, h, y);
+    case 2: return launch_gemv<MODE, WT, 2>(nt, grid(2), s, x, T, H, I, k, list, offsets, perm, h, y);
+    case 4: return launch_gemv<MODE, WT, 4>(nt, grid(4), s, x, T, H, I, k, list, offsets, perm, h, y);
+    default:
+      // packed formats stop at 4 rows per warp (their dequant needs the registers)
+      if constexpr (WT == WT_INT4 || WT == WT_NVFP4)
+        return launch_gemv<MODE, WT, 4>(nt, grid(4), s, x, T, H, I, k, list, offsets, perm, h, y);
+      else
+        return launch_gemv<MODE, WT, 8>(nt, grid(8), s, x, T, H, I, k, list, offsets, perm, h, y);
+  }
+}
+
 cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdtype,
                               const ExpertList& list, int max_pairs_per_expert, const int* offsets,
                               const int* perm, float* h, float* y, cudaStream_t s,
                               cudaEvent_t between, int* err) {
+  (void)err;
   if (list.n <= 0 || T <= 0) return cudaSuccess;
   int nt = max_pairs_per_expert < T ? max_pairs_per_expert : T;
   if (nt < 1) nt = 1;
-  (void)err;
-  // rows per warp: two gate/up row pairs or four down rows (int4: half, for registers)
-  const bool i4 = wdtype == WT_INT4;
-  constexpr int RPW_GU = FT_GEMV_GU_RPW, RPW_D = FT_GEMV_D_RPW;
-  dim3 g1((I + kWarps * RPW_GU - 1) / (kWarps * RPW_GU), list.n);
-  dim3 g2((H + kWarps * RPW_D - 1) / (kWarps * RPW_D), list.n);
+  auto bytes_of = [&](int K) -> size_t {
+    return wdtype == WT_F32 ? (size_t)K * 4 : wdtype == WT_BF16 ? (size_t)K * 2 : (size_t)K / 2;
+  };
+  const int cap = (wdtype == WT_INT4 || wdtype == WT_NVFP4) ? 4 : 8;
+  const int r_gu = rows_per_warp(2 * bytes_of(H), cap);   // a gate row and an up row
+  const int r_d = rows_per_warp(bytes_of(I), cap);
   cudaError_t e;
-#define FT_FFN(WTV, GUR, DR)                                                                          \
-  {                                                                                                   \
-    dim3 ga((I + kWarps * GUR - 1) / (kWarps * GUR), list.n);                                          \
-    dim3 gb((H + kWarps * DR - 1) / (kWarps * DR), list.n);                                            \
-    e = launch_gemv<MODE_GATE_UP, WTV, GUR>(nt, ga, s, x, T, H, I, k, list, offsets, perm, h, y);     \
-    if (e != cudaSuccess) return e;                                                                   \
-    if (between) cudaEventRecord(between, s);                                                        \
-    return launch_gemv<MODE_DOWN, WTV, DR>(nt, gb, s, x, T, H, I, k, list, offsets, perm, h, y);      \
-  }
-  (void)i4;
-  (void)g1;
-  (void)g2;
-  if (wdtype == WT_F32) FT_FFN(WT_F32, RPW_GU, RPW_D)
-  if (wdtype == WT_BF16) FT_FFN(WT_BF16, RPW_GU, RPW_D)
-  if (wdtype == WT_NVFP4) FT_FFN(WT_NVFP4, 1, 2)
-  FT_FFN(WT_INT4, 1, 2)
+#define FT_FFN(WTV)                                                                                        \
+  e = launch_pass<MODE_GATE_UP, WTV>(nt, r_gu, I, s, x, T, H, I, k, list, offsets, perm, h, y);            \
+  if (e != cudaSuccess) return e;                                                                          \
+  if (between) cudaEventRecord(between, s);                                                               \
+  return launch_pass<MODE_DOWN, WTV>(nt, r_d, H, s, x, T, H, I, k, list, offsets, perm, h, y);
+  if (wdtype == WT_F32) { FT_FFN(WT_F32) }
+  if (wdtype == WT_BF16) { FT_FFN(WT_BF16) }
+  if (wdtype == WT_NVFP4) { FT_FFN(WT_NVFP4) }
+  FT_FFN(WT_INT4)
 #undef FT_FFN
 }
 

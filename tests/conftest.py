@@ -11,6 +11,14 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: large full-size workload")
+    # The library is built in-tree (nvcc cross-compiles without a GPU); the build is
+    # incremental, so this is a no-op when libftmoe.so is current.
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_ftmoe_build", os.path.join(ROOT, "moe_expert_offload_top_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
 
 
 def pytest_collection_modifyitems(config, items):
