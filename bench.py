@@ -13,7 +13,7 @@ FreeToken pages.
 
 Reports (one JSON line, rank 0): decode tokens/s timed on the device with
 CUDA events (max over ranks), an end-to-end figure through host buffers, the
-roofline of the dominant kernel (the gate/up expert GEMV, HBM-bound) from
+roofline of the dominant kernel (the fused decode expert FFN, HBM-bound) from
 live CUDA events, cache miss rate and H2D fill bandwidth, SM clocks sampled
 during the timed region, and the CPU oracle timed on a bounded sample.
 N > 1 runs independent replicas (one stack per GPU, its own token chain):
@@ -52,6 +52,26 @@ def workload_desc(cfg):
         "l2": "not flushed: each step streams ~%d MB of expert weights, above the 126 MB L2"
               % round(cfg.L * (cfg.k * cfg.blob_bytes + cfg.E * cfg.H * 4) / 1e6),
     }
+
+
+# DRAM traffic of the dominant kernel (the decode gate/up GEMV) from one ncu capture of
+# this workload: dram__bytes_read.sum + dram__bytes_write.sum of its launches divided by
+# their algorithmic bytes.  Valid only while the kernel's sources hash to `sha256`;
+# otherwise the JSON line carries traffic null.
+GEMV_TRAFFIC = {"sources": ["moe_expert_offload_top_b200/csrc/decode_gemv.cuh",
+                            "moe_expert_offload_top_b200/csrc/expert_decode.cu"],
+                "sha256": None, "ratio": None, "capture": None}
+
+
+def kernel_traffic(bytes_per_launch):
+    import hashlib
+    h = hashlib.sha256()
+    for rel in GEMV_TRAFFIC["sources"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if GEMV_TRAFFIC["ratio"] is None or h.hexdigest() != GEMV_TRAFFIC["sha256"]:
+        return None, h.hexdigest()
+    return GEMV_TRAFFIC["ratio"] * bytes_per_launch, h.hexdigest()
 
 
 def measured_peaks():
@@ -374,25 +394,36 @@ def run_ours(args):
 
     if rank == 0:
         peak, peak_src = measured_peaks()
-        gu_launches = max(perf["timed_forwards"], 1)
-        gu_s = perf["ffn_gate_up_ms"] * 1e-3
-        achieved = perf["ffn_gate_up_bytes"] / gu_s / 1e9 if gu_s > 0 else None
+        fwd = max(perf["timed_forwards"], 1)
+        fl = perf["ffn_fused_launches"]
+        if fl > 0:
+            # the fused decode FFN (gate/up + SwiGLU + down + combine in one launch)
+            f_s = perf["ffn_fused_ms"] * 1e-3
+            achieved = perf["ffn_fused_bytes"] / f_s / 1e9 if f_s > 0 else None
+            roof = {"kernel": "ffn_decode_fused_kernel (expert gate/up + SwiGLU + down + combine, decode)",
+                    "bytes_per_launch": perf["ffn_fused_bytes"] / fl, "avg_launch_us": 1e6 * f_s / fl,
+                    "launches_per_forward": fl / fwd}
+        else:
+            gu_s = perf["ffn_gate_up_ms"] * 1e-3
+            gl = max(perf["ffn_gate_up_launches"], 1)
+            achieved = perf["ffn_gate_up_bytes"] / gu_s / 1e9 if gu_s > 0 else None
+            traffic, src_hash = kernel_traffic(perf["ffn_gate_up_bytes"] / gl)
+            roof = {"kernel": "grouped_gemv_kernel (expert gate/up + SwiGLU, decode)",
+                    "bytes_per_launch": perf["ffn_gate_up_bytes"] / gl, "avg_launch_us": 1e6 * gu_s / gl,
+                    "launches_per_forward": gl / fwd, "traffic": traffic,
+                    "traffic_source": GEMV_TRAFFIC["capture"] if traffic is not None else
+                    "no ncu capture of these kernel sources (sha256 %s)" % src_hash[:12],
+                    "down_proj_gbs": perf["ffn_down_bytes"] / (perf["ffn_down_ms"] * 1e-3) / 1e9
+                    if perf["ffn_down_ms"] > 0 else None}
         line = {
             "metric": METRIC, "value": tokens / t_max, "unit": "tokens/s", "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": 1e3 * t_max / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,0.02) weights, AR(1) hidden states)",
             "config": dict(workload_desc(cfg), parallelism="replicas x%d" % world),
-            "roofline": {
-                "kernel": "grouped_gemv_kernel (expert gate/up + SwiGLU, decode)",
-                "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak if achieved else None, "peak_source": peak_src,
-                "traffic": None,
-                "bytes_per_launch": perf["ffn_gate_up_bytes"] / gu_launches,
-                "avg_launch_us": 1e6 * gu_s / gu_launches,
-                "down_proj_gbs": perf["ffn_down_bytes"] / (perf["ffn_down_ms"] * 1e-3) / 1e9
-                if perf["ffn_down_ms"] > 0 else None,
-            },
+            "roofline": dict({"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                              "frac": achieved / peak if achieved else None, "peak_source": peak_src,
+                              "traffic": None}, **roof),
             "e2e": {"value": e2e_tokens / e2e_max, "unit": "tokens/s",
                     "h2d_bytes_per_step": int(cfg.H * 2 * cfg.batches[0]),
                     "d2h_bytes_per_step": int(cfg.L * cfg.H * 2 * cfg.batches[0])},
@@ -404,8 +435,8 @@ def run_ours(args):
                       "link_h2d_gbs_measured": link_h2d, "link_d2h_gbs_measured": link_d2h,
                       "h2d_frac_of_link": (st["h2d_bytes"] / st["h2d_seconds"] / 1e9) / link_h2d
                       if st["h2d_seconds"] > 0 and link_h2d else None},
-            "stages_us_per_forward": {k2: 1e3 * perf[k2 + "_ms"] / gu_launches for k2 in
-                                      ("router", "permute", "ffn_gate_up", "ffn_down", "combine")},
+            "stages_us_per_forward": {k2: 1e3 * perf[k2 + "_ms"] / fwd for k2 in
+                                      ("router", "permute", "ffn_gate_up", "ffn_down", "combine", "ffn_fused")},
             "host_wait_us_per_forward": 1e3 * perf["host_wait_ms"] / max(perf["forwards"], 1),
         }
         if world == 1 and args.prefill:

@@ -195,6 +195,13 @@ FT_API int ft_moe_set_gemm_threshold(ft_moe* h, int min_avg_pairs);
  * (ft_route_decode), 0 = router, top-k and permutation as three launches.  Same results. */
 FT_API int ft_moe_set_fused_routing(ft_moe* h, int enabled);
 
+/* Decode FFN launch shape (the GEMV path).  Either way the experts whose slots this
+ * stream has already waited for run before the wait for this call's misses, and the rest
+ * after it.  0 (default) = per group a gate/up and a down launch, then one combine;
+ * 1 = per group one fused kernel that runs gate/up + SwiGLU, down and (in the last group)
+ * the combine.  The per-output arithmetic is the same, so the outputs are bit-identical. */
+FT_API int ft_moe_set_fused_ffn(ft_moe* h, int enabled);
+
 /* Host-side fault injection for tests of failure handling (no GPU fault is made).
  *   FT_INJECT_COPY_FAIL: the countdown-th slot fill from now is reported failed instead
  *     of being issued.  The forward returns FT_ERR_CUDA before launching its FFN; the
@@ -202,8 +209,12 @@ FT_API int ft_moe_set_fused_routing(ft_moe* h, int enabled);
  *     (their accesses stay in the trace).  The next forward works normally.
  *   FT_INJECT_ROUTE_TIMEOUT: the countdown-th routing wait reports FT_ERR_TIMEOUT (after
  *     the GPU work completes); the cache is unchanged.
+ *   FT_INJECT_FUSED_WAIT: in the countdown-th fused decode FFN launch every down item
+ *     waits for one gate/up item more than exist, so each of those device waits gives
+ *     up after 1 ms and writes code 111 to the error word; the kernel still completes,
+ *     and the next forward (or ft_moe_sync) reports FT_ERR_DEVICE_CHECK.
  * countdown 0 disarms. */
-enum ft_inject { FT_INJECT_COPY_FAIL = 1, FT_INJECT_ROUTE_TIMEOUT = 2 };
+enum ft_inject { FT_INJECT_COPY_FAIL = 1, FT_INJECT_ROUTE_TIMEOUT = 2, FT_INJECT_FUSED_WAIT = 3 };
 FT_API int ft_moe_debug_inject(ft_moe* h, int what, int countdown);
 
 /* Runs one CTA that waits, with the same bounded wait the prefill GEMM kernels use, on a
@@ -264,8 +275,19 @@ typedef struct {
   double ffn_down_bytes;
   double ffn_flops;        /* 2 * (3 * H * I) per (token, expert) pair */
   double host_wait_ms;     /* host time spent waiting for the routing ids */
+  /* Fused decode FFN (gate/up + SwiGLU + down + combine in one launch, the default for
+   * the GEMV path): kernel time, algorithmic bytes (the weights of every listed expert,
+   * x in and out back) and launches.  A forward whose experts are partly still being
+   * copied runs two launches (the resident experts first), so launches >= forwards. */
+  double ffn_fused_ms;
+  double ffn_fused_bytes;
+  long long ffn_fused_launches;
+  long long ffn_gate_up_launches;   /* per-pass gate/up launches (two where a forward is split) */
 } ft_perf_t;
 
+/* Stage timing holds the forward's stream with a one-thread kernel while the host queues
+ * each stage, so the CUDA events around a launch time the kernel, not the host issuing
+ * it.  For measurement only: it serialises the host and the GPU. */
 FT_API int ft_moe_set_stage_timing(ft_moe* h, int enabled);
 /* Waits for the timed forwards and reads the counters. */
 FT_API int ft_moe_perf(ft_moe* h, ft_perf_t* out);

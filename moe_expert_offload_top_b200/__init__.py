@@ -25,7 +25,7 @@ FT_OK, FT_ERR_INVALID, FT_ERR_OOM, FT_ERR_CUDA, FT_ERR_CAPACITY, FT_ERR_BUSY, FT
 FT_W_F32, FT_W_BF16, FT_W_INT4_G128, FT_W_NVFP4 = 0, 1, 2, 3
 FT_GATE_SOFTMAX, FT_GATE_SIGMOID = 0, 1
 FT_ROUTED, FT_PREFETCH = 0, 1
-FT_INJECT_COPY_FAIL, FT_INJECT_ROUTE_TIMEOUT = 1, 2
+FT_INJECT_COPY_FAIL, FT_INJECT_ROUTE_TIMEOUT, FT_INJECT_FUSED_WAIT = 1, 2, 3
 FT_POLICY_LRU, FT_POLICY_STATIC = 0, 1
 FT_MAX_EXPERTS, FT_MAX_TOPK = 256, 16
 WDTYPE = {"f32": FT_W_F32, "bf16": FT_W_BF16, "int4": FT_W_INT4_G128, "nvfp4": FT_W_NVFP4}
@@ -50,7 +50,9 @@ class ft_perf_t(ctypes.Structure):
                 ("permute_ms", ctypes.c_double), ("ffn_gate_up_ms", ctypes.c_double),
                 ("ffn_down_ms", ctypes.c_double), ("combine_ms", ctypes.c_double),
                 ("ffn_gate_up_bytes", ctypes.c_double), ("ffn_down_bytes", ctypes.c_double),
-                ("ffn_flops", ctypes.c_double), ("host_wait_ms", ctypes.c_double)]
+                ("ffn_flops", ctypes.c_double), ("host_wait_ms", ctypes.c_double),
+                ("ffn_fused_ms", ctypes.c_double), ("ffn_fused_bytes", ctypes.c_double),
+                ("ffn_fused_launches", ctypes.c_longlong), ("ffn_gate_up_launches", ctypes.c_longlong)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -96,6 +98,7 @@ _SIGS = {
     "ft_moe_set_gemm_threshold": ([_vp, _i], _i),
     "ft_moe_debug_inject": ([_vp, _i, _i], _i),
     "ft_moe_set_fused_routing": ([_vp, _i], _i),
+    "ft_moe_set_fused_ffn": ([_vp, _i], _i),
     "ft_debug_device_wait_selftest": ([_i, _vp], _i),
     "ft_moe_perf": ([_vp, ctypes.POINTER(ft_perf_t)], _i),
     "ft_moe_reset_perf": ([_vp], _i),
@@ -248,6 +251,10 @@ def ft_moe_set_gemm_threshold(h, min_avg_pairs):
 
 def ft_moe_set_fused_routing(h, enabled):
     return _check(h, _lib.ft_moe_set_fused_routing(h, int(enabled)))
+
+
+def ft_moe_set_fused_ffn(h, enabled):
+    return _check(h, _lib.ft_moe_set_fused_ffn(h, int(enabled)))
 
 
 def ft_moe_debug_inject(h, what, countdown):

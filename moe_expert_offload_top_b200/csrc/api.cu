@@ -49,10 +49,17 @@ struct FillTiming {
 };
 
 // Stage boundaries of one timed forward, on its stream.
-enum { SE_R0, SE_R1, SE_P0, SE_P1, SE_G0, SE_G1, SE_D1, SE_C1, SE_N };
+// Per-pass FFN: G0 | gate/up | G1 | down | D1 | combine | C1.  Fused FFN: F0 | launch | F1
+// and, when split around the fill wait, F2 | launch | F3; C1 closes the forward.
+// Split per-pass FFN (resident experts first): G0 | gate/up | G1 | down | DA, the fill wait,
+// G2 | gate/up | G3 | down | D1 | combine | C1.
+enum { SE_R0, SE_R1, SE_P0, SE_P1, SE_G0, SE_G1, SE_D1, SE_C1, SE_F0, SE_F1, SE_F2, SE_F3,
+       SE_DA, SE_G2, SE_G3, SE_N };
 struct StageEvents {
   cudaEvent_t ev[SE_N];
-  double gu_bytes, d_bytes, flops;
+  double gu_bytes, d_bytes, flops, fused_bytes;
+  int fused_launches;   // 0: per-pass kernels
+  int split;            // per-pass kernels in two groups around the fill wait
 };
 
 }  // namespace
@@ -96,7 +103,10 @@ struct ft_moe {
   int* d_inv = nullptr;
   float* d_h = nullptr;
   float* d_y = nullptr;
-  int* h_ids = nullptr;
+  int* h_ids = nullptr;            // routing ids on the host: h_box + 2
+  int* h_box = nullptr;            // mapped pinned {seq, device error word, ids[T*k]}
+  int* d_box = nullptr;
+  int route_seq = 0;
   int* d_err = nullptr;           // device-side error word (bounded waits that gave up)
   int* d_ticket = nullptr;        // arrival counter of the fused decode routing kernel
   int* h_err = nullptr;
@@ -108,8 +118,14 @@ struct ft_moe {
   int fused_routing = 1;          // one-launch routing for decode-sized calls
   int inject_copy_fail = 0;       // countdown to a simulated failed slot fill (0 = off)
   int inject_route_timeout = 0;   // countdown to a simulated routing-wait timeout
+  int inject_fused_wait = 0;      // countdown to a fused decode FFN launch whose waits run out
   cudaEvent_t route_ev = nullptr;
   int last_T = 0;
+  int fused_ffn = 0;              // decode FFN + combine as one launch (ffn_decode_fused_kernel)
+  int* d_ctl = nullptr;           // work counters of the fused decode FFN
+  int* h_hold = nullptr;          // mapped pinned flag that releases hold_kernel (stage timing)
+  int* d_hold = nullptr;
+  int hold_seq = 0;
 
   ft_cache_stats_t st{};
   ft_perf_t perf{};
@@ -161,6 +177,30 @@ int wait_event(ft_moe* h, cudaEvent_t ev, const char* what) {
   }
 }
 
+// Host wait for the fused routing kernel's mailbox (mapped pinned memory): returns once
+// box[0] == seq.  Polls the routing event now and then to catch a failed kernel, and
+// gives up after the handle's deadline.
+int wait_box(ft_moe* h, int seq) {
+  const volatile int* flag = h->h_box;
+  auto t0 = std::chrono::steady_clock::now();
+  for (unsigned it = 1;; ++it) {
+    if (*flag == seq) break;
+    if ((it & 255) == 0) {
+      const cudaError_t q = cudaEventQuery(h->route_ev);
+      if (q == cudaSuccess) {
+        if (*flag == seq) break;
+        return fail(h, FT_ERR_CUDA, "routing kernel finished without publishing its ids");
+      }
+      if (q != cudaErrorNotReady) return cuda_fail(h, q, "routing ids");
+      auto dt = std::chrono::steady_clock::now() - t0;
+      if (std::chrono::duration_cast<std::chrono::milliseconds>(dt).count() > h->timeout_ms)
+        return fail(h, FT_ERR_TIMEOUT, "timed out waiting for routing ids");
+    }
+  }
+  std::atomic_thread_fence(std::memory_order_acquire);
+  return FT_OK;
+}
+
 void free_scratch(ft_moe* h) {
   cudaFree(h->d_logits); cudaFree(h->d_ids); cudaFree(h->d_gates); cudaFree(h->d_counts);
   cudaFree(h->d_offsets); cudaFree(h->d_perm); cudaFree(h->d_inv); cudaFree(h->d_h);
@@ -168,10 +208,10 @@ void free_scratch(ft_moe* h) {
   cudaFree(h->d_ax);
   h->d_ax = nullptr;
   h->maps_dirty = true;
-  if (h->h_ids) cudaFreeHost(h->h_ids);
+  if (h->h_box) cudaFreeHost(h->h_box);
   h->d_logits = nullptr; h->d_ids = nullptr; h->d_gates = nullptr; h->d_counts = nullptr;
   h->d_offsets = nullptr; h->d_perm = nullptr; h->d_inv = nullptr; h->d_h = nullptr;
-  h->d_y = nullptr; h->h_ids = nullptr;
+  h->d_y = nullptr; h->h_ids = nullptr; h->h_box = nullptr; h->d_box = nullptr;
   h->cap_tokens = 0;
 }
 
@@ -190,7 +230,8 @@ int ensure_scratch(ft_moe* h, int T) {
             cudaMalloc(&h->d_inv, sizeof(int) * pairs) == cudaSuccess &&
             cudaMalloc(&h->d_h, sizeof(float) * rows * h->I) == cudaSuccess &&
             cudaMalloc(&h->d_y, sizeof(float) * rows * h->H) == cudaSuccess &&
-            cudaHostAlloc(&h->h_ids, sizeof(int) * pairs, cudaHostAllocDefault) == cudaSuccess &&
+            cudaHostAlloc(&h->h_box, sizeof(int) * (2 + pairs), cudaHostAllocMapped) == cudaSuccess &&
+            cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->d_box), h->h_box, 0) == cudaSuccess &&
             (h->wdtype != FT_W_BF16 ||
              cudaMalloc(&h->d_ax, sizeof(uint16_t) * rows * h->H) == cudaSuccess);
   if (!ok) {
@@ -198,6 +239,8 @@ int ensure_scratch(ft_moe* h, int T) {
     free_scratch(h);
     return fail(h, FT_ERR_OOM, "scratch allocation failed");
   }
+  h->h_box[0] = h->h_box[1] = 0;
+  h->h_ids = h->h_box + 2;
   h->cap_tokens = T;
   return FT_OK;
 }
@@ -329,9 +372,29 @@ StageEvents* stage_begin(ft_moe* h) {
   h->stage_pending.push_back(h->stage_free.back());
   h->stage_free.pop_back();
   StageEvents* se = &h->stage_pending.back();
-  se->gu_bytes = se->d_bytes = se->flops = 0.0;
+  se->gu_bytes = se->d_bytes = se->flops = se->fused_bytes = 0.0;
+  se->fused_launches = 0;
+  se->split = 0;
   return se;
 }
+
+// While stage timing is on, the forward's stream is held by a one-thread kernel until
+// the host has queued the launches of a stage, so the events around each launch time
+// the kernel rather than the host issuing it.  The guard releases the hold on every path.
+struct StageHold {
+  ft_moe* h = nullptr;
+  void begin(ft_moe* hh, StageEvents* se, cudaStream_t s) {
+    if (!se || !hh->d_hold) return;
+    h = hh;
+    ++h->hold_seq;
+    ftk::launch_hold(h->d_hold, h->hold_seq, 200000000ull, s);
+  }
+  void release() {
+    if (h) *reinterpret_cast<volatile int*>(h->h_hold) = h->hold_seq;
+    h = nullptr;
+  }
+  ~StageHold() { release(); }
+};
 
 void stage_mark(StageEvents* se, int which, cudaStream_t s) {
   if (se) cudaEventRecord(se->ev[which], s);
@@ -352,11 +415,23 @@ void harvest_stages(ft_moe* h, bool block) {
     };
     h->perf.router_ms += ms(SE_R0, SE_R1);
     h->perf.permute_ms += ms(SE_P0, SE_P1);
-    h->perf.ffn_gate_up_ms += ms(SE_G0, SE_G1);
-    h->perf.ffn_down_ms += ms(SE_G1, SE_D1);
-    h->perf.combine_ms += ms(SE_D1, SE_C1);
-    h->perf.ffn_gate_up_bytes += se.gu_bytes;
-    h->perf.ffn_down_bytes += se.d_bytes;
+    if (se.fused_launches > 0) {
+      h->perf.ffn_fused_ms += ms(SE_F0, SE_F1) + (se.fused_launches > 1 ? ms(SE_F2, SE_F3) : 0.0);
+      h->perf.ffn_fused_bytes += se.fused_bytes;
+      h->perf.ffn_fused_launches += se.fused_launches;
+    } else {
+      h->perf.ffn_gate_up_launches += se.split ? 2 : 1;
+      if (se.split) {
+        h->perf.ffn_gate_up_ms += ms(SE_G0, SE_G1) + ms(SE_G2, SE_G3);
+        h->perf.ffn_down_ms += ms(SE_G1, SE_DA) + ms(SE_G3, SE_D1);
+      } else {
+        h->perf.ffn_gate_up_ms += ms(SE_G0, SE_G1);
+        h->perf.ffn_down_ms += ms(SE_G1, SE_D1);
+      }
+      h->perf.combine_ms += ms(SE_D1, SE_C1);
+      h->perf.ffn_gate_up_bytes += se.gu_bytes;
+      h->perf.ffn_down_bytes += se.d_bytes;
+    }
     h->perf.ffn_flops += se.flops;
     h->perf.timed_forwards++;
     h->stage_free.push_back(se);
@@ -434,6 +509,13 @@ ft_moe* ft_moe_create(int num_experts, int top_k, int hidden, int inter, int wdt
   cudaMemset(h->d_ticket, 0, sizeof(int));
   cudaHostAlloc(&h->h_err, sizeof(int), cudaHostAllocDefault);
   if (h->h_err) *h->h_err = 0;
+  const size_t ctl_bytes = sizeof(int) * (size_t)ftk::ffn_fused_ctl_ints(hidden);
+  cudaMalloc(&h->d_ctl, ctl_bytes);
+  cudaMemset(h->d_ctl, 0, ctl_bytes);
+  if (cudaHostAlloc(&h->h_hold, sizeof(int), cudaHostAllocMapped) == cudaSuccess) {
+    *h->h_hold = 0;
+    cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->d_hold), h->h_hold, 0);
+  }
   cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
   reset_cache_state(h);
   if (cudaGetLastError() != cudaSuccess) {
@@ -535,17 +617,17 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   const bool xbf16 = h->wdtype != FT_W_F32;
   if (h->stage_pending.size() > 256) harvest_stages(h, false);
   StageEvents* se = stage_begin(h);
+  StageHold hold;
+  hold.begin(h, se, s);
   stage_mark(se, SE_R0, s);
   const bool fused_route = h->fused_routing && T <= 64 && E <= 256 && k <= 16;
   if (fused_route) {
     // logits, top-k/gates and the permutation in one launch
+    // the kernel also publishes the ids and the error word to the host mailbox
     FT_CUDA(h, ftk::launch_route_decode(x, xbf16, router_w, T, h->H, E, k, h->gating, h->d_logits, h->d_ids,
                                         h->d_gates, h->d_counts, h->d_offsets, h->d_perm, h->d_inv,
-                                        h->d_ticket, s));
+                                        h->d_ticket, s, h->d_box, ++h->route_seq, h->d_err));
     stage_mark(se, SE_R1, s);
-    FT_CUDA(h, cudaMemcpyAsync(h->h_ids, h->d_ids, sizeof(int) * (size_t)T * k,
-                               cudaMemcpyDeviceToHost, s));
-    FT_CUDA(h, cudaMemcpyAsync(h->h_err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost, s));
     FT_CUDA(h, cudaEventRecord(h->route_ev, s));
     stage_mark(se, SE_P0, s);
     stage_mark(se, SE_P1, s);
@@ -568,13 +650,14 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
     h->perf.kernel_launches += 3;
   }
   h->perf.forwards++;
+  hold.release();
   {
     auto w0 = std::chrono::steady_clock::now();
     if (h->inject_route_timeout > 0 && --h->inject_route_timeout == 0) {
       cudaEventSynchronize(h->route_ev);   // the work itself completes; only the report is injected
       return fail(h, FT_ERR_TIMEOUT, "timed out waiting for routing ids (injected)");
     }
-    rc = wait_event(h, h->route_ev, "routing ids");
+    rc = fused_route ? wait_box(h, h->route_seq) : wait_event(h, h->route_ev, "routing ids");
     h->perf.host_wait_ms +=
         std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - w0).count();
   }
@@ -583,12 +666,14 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   // A failure from here on leaves no kernel of this call running: the caller's stream is
   // drained first, so a following forward on another stream cannot race on the scratch.
   auto bail = [&](int code, const std::string& msg) {
+    hold.release();
     cudaStreamSynchronize(s);
     return fail(h, code, msg);
   };
-  if (*h->h_err) {
-    const int code = *h->h_err;
-    *h->h_err = 0;
+  int* dev_err = fused_route ? h->h_box + 1 : h->h_err;
+  if (*dev_err) {
+    const int code = *dev_err;
+    *dev_err = 0;
     cudaMemsetAsync(h->d_err, 0, sizeof(int), s);
     return bail(FT_ERR_DEVICE_CHECK,
                 "a previous forward's kernel gave up waiting (code " + std::to_string(code) + ")");
@@ -631,69 +716,153 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   // the kernels read the slots of S: wait for their newest fill
   ftk::ExpertList list;
   list.n = 0;
+  long long entry_fill[ftk::kMaxList];
   long long need_fill = -1;
   for (size_t i = 0; i < S.size(); ++i) {
     const int slot = h->lru.slot_of(keys[i]);
     list.expert[list.n] = S[i];
     list.blob[list.n] = h->arena + (size_t)slot * h->blob;
+    entry_fill[list.n] = h->slot_fill_batch[slot];
     list.n++;
     need_fill = std::max(need_fill, h->slot_fill_batch[slot]);
   }
   if (h->has_shared) {
     list.expert[list.n] = -1;
     list.blob[list.n] = h->shared + (size_t)layer * h->blob;
+    entry_fill[list.n] = -1;
     list.n++;
   }
-  if (need_fill > h->compute_waited_fill || (need_fill >= 0 && s != h->last_stream)) {
+  const bool same_stream = h->has_last_stream && s == h->last_stream;
+  const bool must_wait = need_fill > h->compute_waited_fill || (need_fill >= 0 && !same_stream);
+  auto wait_fills = [&]() -> int {
     const int r = (int)(need_fill % kRing);
     FT_CUDA(h, cudaStreamWaitEvent(s, h->fill_ev[r], 0));
     h->compute_waited_fill = h->fill_ev_batch[r];
-  }
+    return FT_OK;
+  };
+  const double xb = xbf16 ? 2.0 : 4.0;
+  const size_t mat = (size_t)h->H * h->I;
+  const double wmat = h->wdtype == FT_W_INT4_G128 ? mat / 2.0 + 2.0 * (mat / 128)
+                      : h->wdtype == FT_W_NVFP4 ? mat / 2.0 + mat / 16.0
+                                                : (double)mat * (h->wdtype == FT_W_F32 ? 4 : 2);
+  const double pairs = (double)T * k + (h->has_shared ? T : 0);
   if (se) {
     // algorithmic bytes: every weight of the listed experts once, their inputs and outputs
-    const double xb = xbf16 ? 2.0 : 4.0;
-    const size_t mat = (size_t)h->H * h->I;
-    const double wmat = h->wdtype == FT_W_INT4_G128 ? mat / 2.0 + 2.0 * (mat / 128)
-                        : h->wdtype == FT_W_NVFP4 ? mat / 2.0 + mat / 16.0
-                                                  : (double)mat * (h->wdtype == FT_W_F32 ? 4 : 2);
-    const double pairs = (double)T * k + (h->has_shared ? T : 0);
     se->gu_bytes = list.n * 2.0 * wmat + pairs * (h->H * xb + h->I * 4.0);
     se->d_bytes = list.n * wmat + pairs * (h->I * 4.0 + h->H * 4.0);
     se->flops = pairs * 6.0 * mat;
   }
+  hold.begin(h, se, s);
   const bool use_gemm = gemm_shapes_ok(h) && (long long)T * k >= (long long)h->gemm_min_avg_pairs * (long long)S.size();
-  if (use_gemm) {
-    rc = ensure_maps(h);
-    if (rc) return rc;
-    ftk::GemmGroups groups;
-    groups.n = list.n;
-    for (int i = 0; i < list.n; ++i) {
-      groups.expert[i] = list.expert[i];
-      groups.z[i] = list.expert[i] >= 0 ? h->lru.slot_of(layer * E + list.expert[i]) : layer;
-    }
-    FT_CUDA(h, ftk::launch_gather_rows(x, h->d_perm, T, k, h->H, h->has_shared != 0, h->d_ax, s));
-    h->perf.kernel_launches += 1;
-    stage_mark(se, SE_G0, s);
-    FT_CUDA(h, ftk::launch_grouped_gemm(0, h->maps, groups, h->d_offsets, T, k, h->I, h->H, h->d_h,
-                                        h->d_err, h->num_sms, s));
-    stage_mark(se, SE_G1, s);
-    FT_CUDA(h, ftk::launch_grouped_gemm(1, h->maps, groups, h->d_offsets, T, k, h->I, h->H, h->d_y,
-                                        h->d_err, h->num_sms, s));
-    if (se) {   // bf16 h, and the weights of each listed expert read once
-      const double pairs = (double)T * k + (h->has_shared ? T : 0);
-      se->gu_bytes = list.n * 2.0 * h->H * h->I * 2 + pairs * (h->H * 2.0 + h->I * 2.0);
-      se->d_bytes = list.n * 1.0 * h->H * h->I * 2 + pairs * (h->I * 2.0 + h->H * 4.0);
-    }
-  } else {
-    stage_mark(se, SE_G0, s);
-    FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, list, max_pairs, h->d_offsets,
-                                      h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr, h->d_err));
+  // Decode path: entries whose slots this stream has already waited for (and the shared
+  // expert) run while this call's misses are still being copied; the rest run after the
+  // wait for the fills, followed by the combine.
+  ftk::ExpertList ready, later;
+  ready.n = later.n = 0;
+  for (int i = 0; i < list.n; ++i) {
+    const bool is_ready = entry_fill[i] < 0 || (same_stream && entry_fill[i] <= h->compute_waited_fill);
+    ftk::ExpertList& dst = is_ready ? ready : later;
+    dst.expert[dst.n] = list.expert[i];
+    dst.blob[dst.n] = list.blob[i];
+    dst.n++;
   }
-  stage_mark(se, SE_D1, s);
-  FT_CUDA(h, ftk::launch_combine(h->d_y, h->d_gates, h->d_inv, T, h->H, k, h->has_shared != 0,
-                                 xbf16, out, s));
-  stage_mark(se, SE_C1, s);
-  h->perf.kernel_launches += 3;
+  const bool split = !use_gemm && ready.n > 0 && later.n > 0;
+  if (!use_gemm && h->fused_ffn) {
+    // one fused launch per group; the last one also runs the combine
+    ftk::FusedParams fp{};
+    fp.x = x; fp.offsets = h->d_offsets; fp.perm = h->d_perm; fp.h = h->d_h; fp.y = h->d_y;
+    fp.gates = h->d_gates; fp.inv = h->d_inv; fp.out = out; fp.ctl = h->d_ctl; fp.err = h->d_err;
+    fp.T = T; fp.H = h->H; fp.I = h->I; fp.k = k;
+    fp.has_shared = h->has_shared != 0; fp.out_bf16 = xbf16 ? 1 : 0;
+    fp.limit_ns = 2000000000ull;
+    if (h->inject_fused_wait > 0 && --h->inject_fused_wait == 0) {
+      fp.wait_extra = 1;          // a count nothing reaches: every down item's wait runs out
+      fp.limit_ns = 1000000ull;   // after 1 ms, with code 111 in the error word
+    }
+    if (se) {   // weights of every listed expert once, x in, out back (h, y stay in L2)
+      se->fused_bytes = list.n * 3.0 * wmat + (double)T * h->H * xb * 2.0;
+    }
+    if (split) {
+      fp.combine = 0;
+      stage_mark(se, SE_F0, s);
+      FT_CUDA(h, ftk::launch_ffn_fused(fp, h->wdtype, ready, max_pairs, h->num_sms, s));
+      stage_mark(se, SE_F1, s);
+      rc = wait_fills();
+      if (rc) return bail(rc, h->err);
+      fp.combine = 1;
+      stage_mark(se, SE_F2, s);
+      FT_CUDA(h, ftk::launch_ffn_fused(fp, h->wdtype, later, max_pairs, h->num_sms, s));
+      stage_mark(se, SE_F3, s);
+      if (se) se->fused_launches = 2;
+      h->perf.kernel_launches += 2;
+    } else {
+      if (must_wait) {
+        rc = wait_fills();
+        if (rc) return bail(rc, h->err);
+      }
+      fp.combine = 1;
+      stage_mark(se, SE_F0, s);
+      FT_CUDA(h, ftk::launch_ffn_fused(fp, h->wdtype, list, max_pairs, h->num_sms, s));
+      stage_mark(se, SE_F1, s);
+      if (se) se->fused_launches = 1;
+      h->perf.kernel_launches += 1;
+    }
+    stage_mark(se, SE_C1, s);
+  } else {
+    if (use_gemm) {
+      if (must_wait) {
+        rc = wait_fills();
+        if (rc) return bail(rc, h->err);
+      }
+      rc = ensure_maps(h);
+      if (rc) return rc;
+      ftk::GemmGroups groups;
+      groups.n = list.n;
+      for (int i = 0; i < list.n; ++i) {
+        groups.expert[i] = list.expert[i];
+        groups.z[i] = list.expert[i] >= 0 ? h->lru.slot_of(layer * E + list.expert[i]) : layer;
+      }
+      FT_CUDA(h, ftk::launch_gather_rows(x, h->d_perm, T, k, h->H, h->has_shared != 0, h->d_ax, s));
+      h->perf.kernel_launches += 1;
+      stage_mark(se, SE_G0, s);
+      FT_CUDA(h, ftk::launch_grouped_gemm(0, h->maps, groups, h->d_offsets, T, k, h->I, h->H, h->d_h,
+                                          h->d_err, h->num_sms, s));
+      stage_mark(se, SE_G1, s);
+      FT_CUDA(h, ftk::launch_grouped_gemm(1, h->maps, groups, h->d_offsets, T, k, h->I, h->H, h->d_y,
+                                          h->d_err, h->num_sms, s));
+      if (se) {   // bf16 h, and the weights of each listed expert read once
+        se->gu_bytes = list.n * 2.0 * h->H * h->I * 2 + pairs * (h->H * 2.0 + h->I * 2.0);
+        se->d_bytes = list.n * 1.0 * h->H * h->I * 2 + pairs * (h->I * 2.0 + h->H * 4.0);
+      }
+    } else if (split) {
+      // gate/up | G1 | down of the ready group, the wait, then gate/up | G3 | down of the rest
+      stage_mark(se, SE_G0, s);
+      FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, ready, max_pairs, h->d_offsets,
+                                        h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr, h->d_err));
+      stage_mark(se, SE_DA, s);
+      rc = wait_fills();
+      if (rc) return bail(rc, h->err);
+      stage_mark(se, SE_G2, s);
+      FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, later, max_pairs, h->d_offsets,
+                                        h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G3] : nullptr, h->d_err));
+      if (se) se->split = 1;
+      h->perf.kernel_launches += 2;
+    } else {
+      if (must_wait) {
+        rc = wait_fills();
+        if (rc) return bail(rc, h->err);
+      }
+      stage_mark(se, SE_G0, s);
+      FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, list, max_pairs, h->d_offsets,
+                                        h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr, h->d_err));
+    }
+    stage_mark(se, SE_D1, s);
+    FT_CUDA(h, ftk::launch_combine(h->d_y, h->d_gates, h->d_inv, T, h->H, k, h->has_shared != 0,
+                                   xbf16, out, s));
+    stage_mark(se, SE_C1, s);
+    h->perf.kernel_launches += 3;
+  }
+  hold.release();
   {
     const int r = (int)(call % kRing);
     FT_CUDA(h, cudaEventRecord(h->use_ev[r], s));
@@ -727,6 +896,12 @@ int ft_moe_sync(ft_moe* h) {
   return FT_OK;
 }
 
+int ft_moe_set_fused_ffn(ft_moe* h, int enabled) {
+  if (!h) return FT_ERR_INVALID;
+  h->fused_ffn = enabled != 0;
+  return FT_OK;
+}
+
 int ft_moe_set_fused_routing(ft_moe* h, int enabled) {
   if (!h) return FT_ERR_INVALID;
   h->fused_routing = enabled != 0;
@@ -737,6 +912,7 @@ int ft_moe_debug_inject(ft_moe* h, int what, int countdown) {
   if (!h || countdown < 0) return FT_ERR_INVALID;
   if (what == FT_INJECT_COPY_FAIL) h->inject_copy_fail = countdown;
   else if (what == FT_INJECT_ROUTE_TIMEOUT) h->inject_route_timeout = countdown;
+  else if (what == FT_INJECT_FUSED_WAIT) h->inject_fused_wait = countdown;
   else return fail(h, FT_ERR_INVALID, "ft_moe_debug_inject: unknown fault");
   return FT_OK;
 }
@@ -923,7 +1099,9 @@ void ft_moe_destroy(ft_moe* h) {
   free_scratch(h);
   cudaFree(h->d_err);
   cudaFree(h->d_ticket);
+  cudaFree(h->d_ctl);
   if (h->h_err) cudaFreeHost(h->h_err);
+  if (h->h_hold) cudaFreeHost(h->h_hold);
   if (h->copy) cudaStreamDestroy(h->copy);
   cudaFree(h->arena);
   cudaFree(h->shared);

@@ -25,10 +25,14 @@ cudaError_t launch_topk_gates(const float* logits, int T, int E, int k, int gati
                               float* gates, cudaStream_t s);
 // K1+K2 for decode (T <= 64, E <= 256, k <= 16) in one launch: logits, top-k + gates and
 // the stable permutation (the last router CTA does the second part).  *ticket must be 0
-// before the launch; the kernel leaves it 0.
+// before the launch; the kernel leaves it 0.  box (optional, mapped pinned host memory of
+// 2 + T*k ints): the last CTA also writes the ids to box[2..], *err to box[1] and then,
+// after a system-scope fence, seq to box[0], so the host can take the routing as soon as
+// it exists.
 cudaError_t launch_route_decode(const void* x, bool x_bf16, const float* w_router, int T, int H, int E, int k,
                                 int gating, float* logits, int* ids, float* gates, int* counts, int* offsets,
-                                int* perm, int* inv, int* ticket, cudaStream_t s);
+                                int* perm, int* inv, int* ticket, cudaStream_t s, int* box = nullptr,
+                                int seq = 0, const int* err = nullptr);
 // K2: stable counting sort of the T*k pairs by expert.
 // inv (optional): inv[t*k+j] = position of pair (t,j) in perm.
 cudaError_t launch_permute(const int* ids, int T, int k, int E, int* counts, int* offsets,
@@ -41,6 +45,46 @@ cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdt
                               const ExpertList& list, int max_pairs_per_expert, const int* offsets,
                               const int* perm, float* h, float* y, cudaStream_t s,
                               cudaEvent_t between = nullptr, int* err = nullptr);
+// K3 + K5 (decode) in one launch (ffn_fused.cuh): gate/up + SwiGLU into h, down into y
+// and, with `combine`, out[t] = sum_j gates[t][j] * y[inv[t*k+j]] (+ shared) for the
+// entries of `list`.  The combine of a launch covers every pair of the forward, so
+// entries not in `list` must have written their y rows earlier on the stream.
+// ctl: ffn_fused_ctl_ints(H) ints of device memory, zero before the first launch
+// (every launch leaves them zero); launches that use one ctl must not overlap.
+// A down item waits at most limit_ns for its entry's gate/up items and otherwise
+// writes 111 to *err.
+struct FusedParams {
+  const void* x;
+  const int* offsets;
+  const int* perm;
+  float* h;
+  float* y;
+  const float* gates;
+  const int* inv;
+  void* out;
+  int* ctl;
+  int* err;
+  int T, H, I, k;
+  int has_shared, combine, out_bf16;
+  int wait_extra;   // tests only: down items wait for this many gate/up items more than exist
+  unsigned long long limit_ns;
+};
+int ffn_fused_ctl_ints(int H);
+cudaError_t launch_ffn_fused(const FusedParams& p, int wdtype, const ExpertList& list, int max_pairs_per_expert,
+                             int num_sms, cudaStream_t s);
+cudaError_t launch_ffn_fused_f32(int nt, int rg, int rd, const FusedParams& p, const ExpertList& list, int num_sms,
+                                 cudaStream_t s);
+cudaError_t launch_ffn_fused_bf16(int nt, int rg, int rd, const FusedParams& p, const ExpertList& list, int num_sms,
+                                  cudaStream_t s);
+cudaError_t launch_ffn_fused_int4(int nt, int rg, int rd, const FusedParams& p, const ExpertList& list, int num_sms,
+                                  cudaStream_t s);
+cudaError_t launch_ffn_fused_nvfp4(int nt, int rg, int rd, const FusedParams& p, const ExpertList& list,
+                                   int num_sms, cudaStream_t s);
+// One thread waits until *flag >= want (the host writes the flag through mapped pinned
+// memory), at most limit_ns.  Holds the stream while the host queues the launches of
+// a timed stage, so that CUDA events around them time the kernels and not the host.
+cudaError_t launch_hold(const volatile int* flag, int want, unsigned long long limit_ns, cudaStream_t s);
+
 // K5: out[t] = sum_j gates[t][j] * y[inv[t*k+j]] (ascending j) + y[T*k+t] if has_shared.
 cudaError_t launch_combine(const float* y, const float* gates, const int* inv, int T, int H, int k,
                            bool has_shared, bool out_bf16, void* out, cudaStream_t s);

@@ -45,7 +45,8 @@ router_logits_kernel(const XT* __restrict__ x, const float* __restrict__ w, int 
   for (int i = 0; i < kRouterEPB; ++i)
 #pragma unroll
     for (int t = 0; t < kRouterTPB; ++t) acc[i][t] = 0.f;
-  for (int hh = threadIdx.x * 4; hh < H; hh += kRouterThreads * 4) {
+#pragma unroll 4
+  for (int hh = threadIdx.x * 4; hh < H; hh += kRouterThreads * 4) {   // unrolled: loads in flight together
     float wv[kRouterEPB][4];
 #pragma unroll
     for (int i = 0; i < kRouterEPB; ++i) {
@@ -196,10 +197,11 @@ __global__ void __launch_bounds__(kRouterThreads)
 route_decode_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T, int H, int E, int k,
                     int gating, float* __restrict__ z, int* __restrict__ ids, float* __restrict__ gates,
                     int* __restrict__ counts, int* __restrict__ offsets, int* __restrict__ perm,
-                    int* __restrict__ inv, int* __restrict__ ticket) {
+                    int* __restrict__ inv, int* __restrict__ ticket, int* __restrict__ box, int seq,
+                    const int* __restrict__ err) {
   __shared__ float part[kRouterThreads / 32][kRouterEPB][kRouterTPB];
   __shared__ int last;
-  __shared__ int s_cnt[256], s_base[256], s_wc[kRouterThreads / 32][256];
+  __shared__ int s_cnt[256], s_base[256], s_wc[kRouterThreads / 32][256], s_wsum[kRouterThreads / 32];
   __shared__ int s_ids[64 * 16];
   const int e0 = blockIdx.x * kRouterEPB, t0 = blockIdx.y * kRouterTPB;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -209,7 +211,8 @@ route_decode_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T
     for (int i = 0; i < kRouterEPB; ++i)
 #pragma unroll
       for (int t = 0; t < kRouterTPB; ++t) acc[i][t] = 0.f;
-    for (int hh = threadIdx.x * 4; hh < H; hh += kRouterThreads * 4) {
+#pragma unroll 4
+    for (int hh = threadIdx.x * 4; hh < H; hh += kRouterThreads * 4) {   // unrolled: loads in flight together
       float wv[kRouterEPB][4];
 #pragma unroll
       for (int i = 0; i < kRouterEPB; ++i) {
@@ -236,8 +239,10 @@ route_decode_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T
     for (int i = 0; i < kRouterEPB; ++i)
 #pragma unroll
       for (int t = 0; t < kRouterTPB; ++t) {
-        float v = warp_sum(acc[i][t]);
-        if (lane == 0) part[warp][i][t] = v;
+        if (t0 + t < T) {   // the same for the whole CTA: the shuffles stay warp-uniform
+          float v = warp_sum(acc[i][t]);
+          if (lane == 0) part[warp][i][t] = v;
+        }
       }
     __syncthreads();
     if (threadIdx.x < kRouterEPB * kRouterTPB) {
@@ -311,37 +316,72 @@ route_decode_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T
   __syncthreads();
   for (int p = threadIdx.x; p < n; p += kRouterThreads) atomicAdd(&s_cnt[s_ids[p]], 1);
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int e = 0; e < E; ++e) { s_base[e] = run; run += s_cnt[e]; }
-    offsets[E] = run;
+  {  // exclusive scan of the E <= 256 counts: one per thread, warp scans, then warp totals
+    const int c = threadIdx.x < E ? s_cnt[threadIdx.x] : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w2 = 0; w2 < warp; ++w2) before += s_wsum[w2];
+    if (threadIdx.x < E) {
+      s_base[threadIdx.x] = before + incl - c;
+      counts[threadIdx.x] = c;
+      offsets[threadIdx.x] = before + incl - c;
+    }
+    if (threadIdx.x == 0) offsets[E] = n;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kRouterThreads) { counts[e] = s_cnt[e]; offsets[e] = s_base[e]; }
   const unsigned lt = (1u << lane) - 1u;
-  for (int c = 0; c < n; c += kRouterThreads) {
-    for (int i = threadIdx.x; i < (kRouterThreads / 32) * E; i += kRouterThreads) s_wc[i / E][i % E] = 0;
-    __syncthreads();
-    const int p = c + threadIdx.x;
-    const int e = p < n ? s_ids[p] : -1;
-    const unsigned mask = __match_any_sync(0xFFFFFFFFu, e);
-    const int rank = __popc(mask & lt);
-    if (e >= 0 && rank == 0) s_wc[warp][e] = __popc(mask);
-    __syncthreads();
-    if (e >= 0) {
-      int before = 0;
-      for (int w2 = 0; w2 < warp; ++w2) before += s_wc[w2][e];
-      const int q = s_base[e] + before + rank;
-      perm[q] = p;
-      inv[p] = q;
+  if (n <= 32) {
+    // one warp: a pair's place is its expert's base + its rank among equal keys
+    if (warp == 0) {
+      const int e = lane < n ? s_ids[lane] : -1;
+      const unsigned mask = __match_any_sync(0xFFFFFFFFu, e);
+      if (e >= 0) {
+        const int q = s_base[e] + __popc(mask & lt);
+        perm[q] = lane;
+        inv[lane] = q;
+      }
     }
-    __syncthreads();
-    for (int ee = threadIdx.x; ee < E; ee += kRouterThreads) {
-      int sum = 0;
-      for (int w2 = 0; w2 < kRouterThreads / 32; ++w2) sum += s_wc[w2][ee];
-      s_base[ee] += sum;
+  } else {
+    for (int c = 0; c < n; c += kRouterThreads) {
+      for (int i = threadIdx.x; i < (kRouterThreads / 32) * E; i += kRouterThreads) s_wc[i / E][i % E] = 0;
+      __syncthreads();
+      const int p = c + threadIdx.x;
+      const int e = p < n ? s_ids[p] : -1;
+      const unsigned mask = __match_any_sync(0xFFFFFFFFu, e);
+      const int rank = __popc(mask & lt);
+      if (e >= 0 && rank == 0) s_wc[warp][e] = __popc(mask);
+      __syncthreads();
+      if (e >= 0) {
+        int before = 0;
+        for (int w2 = 0; w2 < warp; ++w2) before += s_wc[w2][e];
+        const int q = s_base[e] + before + rank;
+        perm[q] = p;
+        inv[p] = q;
+      }
+      __syncthreads();
+      for (int ee = threadIdx.x; ee < E; ee += kRouterThreads) {
+        int sum = 0;
+        for (int w2 = 0; w2 < kRouterThreads / 32; ++w2) sum += s_wc[w2][ee];
+        s_base[ee] += sum;
+      }
+      __syncthreads();
     }
+  }
+  if (box) {
+    // publish to the host through mapped pinned memory: ids and the device error word,
+    // then (after a system-scope fence) the sequence number the host waits for
+    for (int p = threadIdx.x; p < n; p += kRouterThreads) box[2 + p] = s_ids[p];
+    if (threadIdx.x == 0) box[1] = *reinterpret_cast<const volatile int*>(err);
+    __threadfence_system();
     __syncthreads();
+    if (threadIdx.x == 0) *reinterpret_cast<volatile int*>(box) = seq;
   }
   if (threadIdx.x == 0) *ticket = 0;
 }
@@ -363,18 +403,19 @@ cudaError_t launch_router_logits_tiled(const void* x, bool x_bf16, const float* 
 
 cudaError_t launch_route_decode(const void* x, bool x_bf16, const float* w_router, int T, int H, int E, int k,
                                 int gating, float* logits, int* ids, float* gates, int* counts, int* offsets,
-                                int* perm, int* inv, int* ticket, cudaStream_t s) {
+                                int* perm, int* inv, int* ticket, cudaStream_t s, int* box, int seq,
+                                const int* err) {
   if (T <= 0) return cudaSuccess;
   if (T > 64 || E > 256 || k > 16) return cudaErrorInvalidValue;
   dim3 grid((E + kRouterEPB - 1) / kRouterEPB, (T + kRouterTPB - 1) / kRouterTPB);
   if (x_bf16)
     route_decode_kernel<uint16_t><<<grid, kRouterThreads, 0, s>>>(static_cast<const uint16_t*>(x), w_router, T, H,
                                                                   E, k, gating, logits, ids, gates, counts, offsets,
-                                                                  perm, inv, ticket);
+                                                                  perm, inv, ticket, box, seq, err);
   else
     route_decode_kernel<float><<<grid, kRouterThreads, 0, s>>>(static_cast<const float*>(x), w_router, T, H, E, k,
                                                                gating, logits, ids, gates, counts, offsets, perm,
-                                                               inv, ticket);
+                                                               inv, ticket, box, seq, err);
   return cudaGetLastError();
 }
 

@@ -88,3 +88,35 @@ def test_step_larger_than_cache_is_rejected_first():
             st.forward(0, x[0], out)
         assert ei.value.code == ft.FT_ERR_CAPACITY
         assert st.trace() == [] and st.stats()["resident"] == 0
+
+
+def test_fused_ffn_wait_gives_up_and_is_reported():
+    """A fused decode FFN launch whose down items wait for a count nothing reaches: each
+    wait gives up after 1 ms, the kernel completes, the error word is reported at the next
+    synchronisation, and the following forwards are correct again."""
+    cfg = _cfg()
+    with GpuStack(cfg) as st:
+        ft.ft_moe_set_fused_ffn(st.h, 1)
+        vals, x = st.tokens(1)
+        out = torch.empty((cfg.L, 1, cfg.H), dtype=torch.bfloat16, device=DEV)
+        st.step(x[0], out)
+        ft.ft_moe_sync(st.h)
+        ft.ft_moe_debug_inject(st.h, ft.FT_INJECT_FUSED_WAIT, 1)
+        st.forward(0, x[1], out[0])              # the kernel's waits run out; the call returns
+        with pytest.raises(ft.FtError) as ei:
+            ft.ft_moe_sync(st.h)
+        assert ei.value.code == ft.FT_ERR_DEVICE_CHECK and "111" in str(ei.value)
+        a = torch.ones(1024, device=DEV)
+        assert float((a * 2).sum()) == 2048.0    # the context still runs work
+        got = {}
+        for s in range(2, 6):
+            st.step(x[s], out)
+            got[s] = out.float().cpu().numpy().copy()
+        ft.ft_moe_sync(st.h)
+        from oracle import moe
+        for s in range(2, 6):
+            for l in range(cfg.L):
+                r = moe.route(vals[s], synth.router_weights(cfg, l), cfg.k, cfg.gating)
+                ref = moe.experts_and_combine(vals[s], r["ids"], r["gates"], cfg.E, cfg.wdtype, cfg.H, cfg.I,
+                                              lambda e, l=l: st.pool_blob(l, e))
+                assert_close(got[s][l], ref, "bf16", "step %d layer %d" % (s, l))

@@ -1,0 +1,117 @@
+"""The fused decode FFN (gate/up + SwiGLU, down and combine in one launch, resident
+experts launched before the wait for this call's misses) against the per-pass kernels
+and the oracle: the same inputs through two stacks, one per launch shape, give the
+same trace and bit-identical outputs, and the oracle's outputs within the bound."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import moe_expert_offload_top_b200 as ft
+import synth
+from moe_expert_offload_top_b200.workload import GpuStack
+from gpu_util import assert_close, first_divergence, oracle_run
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _run(cfg, fused, batch=1, steps=None, gemm_threshold=None, stage_timing=False, oracle=False):
+    steps = cfg.tokens // batch if steps is None else steps
+    with GpuStack(cfg) as st:
+        ft.ft_moe_set_fused_ffn(st.h, int(fused))
+        if gemm_threshold is not None:
+            ft.ft_moe_set_gemm_threshold(st.h, gemm_threshold)
+        if stage_timing:
+            ft.ft_moe_set_stage_timing(st.h, 1)
+        vals, x = st.tokens(batch)
+        out = torch.empty((cfg.L, batch, cfg.H), dtype=st.xdt, device=DEV)
+        outs, ids = [], np.zeros((steps, cfg.L, batch, cfg.k), dtype=np.int32)
+        for s in range(steps):
+            for l in range(cfg.L):
+                st.forward(l, x[s], out[l])
+                ids[s, l] = st.last_routing(batch)[0]
+            outs.append(out.float().cpu().numpy().copy())
+        torch.cuda.synchronize()
+        res = {"outs": outs, "ids": ids, "trace": st.trace(), "stats": st.stats(), "vals": vals,
+               "perf": ft.ft_moe_perf(st.h)}
+        if oracle:
+            res["ref"] = oracle_run(cfg, st, vals[:steps])
+    return res
+
+
+CASES = {
+    # name: (config, batch)
+    "bf16-misses": (dataclasses.replace(synth.CONFIGS[2], L=2, tokens=24, C=40), 1),
+    "bf16-batch8": (dataclasses.replace(synth.CONFIGS[2], L=2, tokens=48, C=160), 8),
+    "bf16-shared": (synth.MoeConfig("shared-small", L=2, E=32, H=1024, I=512, k=6, gating="sigmoid",
+                                    wdtype="bf16", shared=True, C=20, tokens=12, batches=(1,),
+                                    process="ar1", mode="decode"), 1),
+    "f32-tiny": (synth.CONFIGS[1], 1),
+    "int4": (synth.MoeConfig("int4-small", L=2, E=32, H=1024, I=512, k=8, gating="sigmoid", wdtype="int4",
+                             shared=False, C=24, tokens=12, batches=(1,), process="ar1", mode="decode"), 1),
+    "nvfp4": (synth.MoeConfig("nvfp4-small", L=2, E=32, H=1024, I=512, k=4, gating="softmax", wdtype="nvfp4",
+                              shared=False, C=16, tokens=12, batches=(1,), process="ar1", mode="decode"), 1),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_fused_matches_per_pass_bitwise_and_oracle(name):
+    cfg, batch = CASES[name]
+    if batch > 1:
+        cfg = dataclasses.replace(cfg, batches=(batch,))
+    a = _run(cfg, fused=True, batch=batch, oracle=True)
+    b = _run(cfg, fused=False, batch=batch)
+    assert np.array_equal(a["ids"], b["ids"])
+    assert a["trace"] == b["trace"]
+    assert a["stats"]["misses"] > 0
+    for s, (oa, ob) in enumerate(zip(a["outs"], b["outs"])):
+        assert np.array_equal(oa, ob), "step %d: fused and per-pass outputs differ" % s
+    ref = a["ref"]
+    steps = len(a["outs"])
+    div = first_divergence(a["ids"], ref["ids"][:steps], ref["gap"][:steps], ref.get("zsel"))
+    last = steps if div is None else div // (cfg.L * batch)
+    for s in range(last):
+        for l in range(cfg.L):
+            assert_close(a["outs"][s][l], ref["out"][(s, l)], cfg.wdtype, "%s step %d layer %d" % (name, s, l))
+
+
+def test_many_tokens_gemv_path_fused():
+    # 80 tokens at once on the GEMV path (the tcgen05 GEMMs switched off): three-launch
+    # routing, then the fused FFN with up to 8 pairs per weight pass
+    cfg = synth.MoeConfig("wide-gemv", L=1, E=16, H=1024, I=512, k=4, gating="softmax", wdtype="bf16",
+                          shared=True, C=16, tokens=160, batches=(80,), process="iid", mode="decode")
+    a = _run(cfg, fused=True, batch=80, gemm_threshold=1 << 30, oracle=True)
+    b = _run(cfg, fused=False, batch=80, gemm_threshold=1 << 30)
+    for oa, ob in zip(a["outs"], b["outs"]):
+        assert np.array_equal(oa, ob)
+    ref = a["ref"]
+    div = first_divergence(a["ids"], ref["ids"], ref["gap"], ref.get("zsel"))
+    last = 2 if div is None else div // 80
+    for s in range(last):
+        assert_close(a["outs"][s][0], ref["out"][(s, 0)], "bf16", "step %d" % s)
+
+
+def test_resident_experts_run_before_the_fill_wait():
+    # with misses in most forwards, stage timing sees two fused launches for those
+    # forwards: the resident experts, then the copied ones with the combine
+    cfg = dataclasses.replace(synth.CONFIGS[2], L=2, tokens=24, C=40)
+    a = _run(cfg, fused=True, stage_timing=True)
+    p = a["perf"]
+    assert p["timed_forwards"] == cfg.L * cfg.tokens
+    assert p["timed_forwards"] < p["ffn_fused_launches"] < 2 * p["timed_forwards"]
+    assert p["ffn_fused_ms"] > 0 and p["ffn_fused_bytes"] > 0
+    assert p["ffn_gate_up_ms"] == 0 and p["combine_ms"] == 0
+
+
+def test_per_pass_kernels_split_around_the_fill_wait():
+    # the default launch shape: forwards with both resident and copied experts run two
+    # gate/up + down pairs (five FFN launches with the combine), the others one pair
+    cfg = dataclasses.replace(synth.CONFIGS[2], L=2, tokens=24, C=40)
+    a = _run(cfg, fused=False, stage_timing=True)
+    p = a["perf"]
+    fwd = cfg.L * cfg.tokens
+    assert p["forwards"] == fwd and p["ffn_fused_launches"] == 0
+    assert 4 * fwd < p["kernel_launches"] < 6 * fwd      # routing + 3, + 2 where split
+    assert p["ffn_gate_up_ms"] > 0 and p["ffn_down_ms"] > 0 and p["combine_ms"] > 0
