@@ -202,6 +202,13 @@ FT_API int ft_moe_set_fused_routing(ft_moe* h, int enabled);
  * the combine.  The per-output arithmetic is the same, so the outputs are bit-identical. */
 FT_API int ft_moe_set_fused_ffn(ft_moe* h, int enabled);
 
+/* int4 decode GEMV (per-pass launch shape): 1 (default) = on the tensor cores
+ * (mma.sync with bf16 operands and fp32 accumulation; the down projection's input h is
+ * carried as two bf16 halves, 16 mantissa bits), 0 = fp32 multiply-adds on the CUDA
+ * cores.  Both are within the stated bound of the oracle; their outputs differ in the
+ * last bits (summation order).  ft_expert_ffn_decode always uses the tensor cores. */
+FT_API int ft_moe_set_int4_tensor_cores(ft_moe* h, int enabled);
+
 /* Host-side fault injection for tests of failure handling (no GPU fault is made).
  *   FT_INJECT_COPY_FAIL: the countdown-th slot fill from now is reported failed instead
  *     of being issued.  The forward returns FT_ERR_CUDA before launching its FFN; the
@@ -287,7 +294,9 @@ typedef struct {
 
 /* Stage timing holds the forward's stream with a one-thread kernel while the host queues
  * each stage, so the CUDA events around a launch time the kernel, not the host issuing
- * it.  For measurement only: it serialises the host and the GPU. */
+ * it; and every forward's FFN then runs after the wait for its fills (no split into
+ * resident and copied experts), so each launch covers the forward's whole list.  For
+ * measurement only: it serialises the host and the GPU. */
 FT_API int ft_moe_set_stage_timing(ft_moe* h, int enabled);
 /* Waits for the timed forwards and reads the counters. */
 FT_API int ft_moe_perf(ft_moe* h, ft_perf_t* out);

@@ -99,6 +99,7 @@ _SIGS = {
     "ft_moe_debug_inject": ([_vp, _i, _i], _i),
     "ft_moe_set_fused_routing": ([_vp, _i], _i),
     "ft_moe_set_fused_ffn": ([_vp, _i], _i),
+    "ft_moe_set_int4_tensor_cores": ([_vp, _i], _i),
     "ft_debug_device_wait_selftest": ([_i, _vp], _i),
     "ft_moe_perf": ([_vp, ctypes.POINTER(ft_perf_t)], _i),
     "ft_moe_reset_perf": ([_vp], _i),
@@ -255,6 +256,10 @@ def ft_moe_set_fused_routing(h, enabled):
 
 def ft_moe_set_fused_ffn(h, enabled):
     return _check(h, _lib.ft_moe_set_fused_ffn(h, int(enabled)))
+
+
+def ft_moe_set_int4_tensor_cores(h, enabled):
+    return _check(h, _lib.ft_moe_set_int4_tensor_cores(h, int(enabled)))
 
 
 def ft_moe_debug_inject(h, what, countdown):

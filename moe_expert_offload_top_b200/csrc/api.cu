@@ -122,6 +122,7 @@ struct ft_moe {
   cudaEvent_t route_ev = nullptr;
   int last_T = 0;
   int fused_ffn = 0;              // decode FFN + combine as one launch (ffn_decode_fused_kernel)
+  int int4_tensor = 1;            // int4 decode GEMV on the tensor cores (mma.sync)
   int* d_ctl = nullptr;           // work counters of the fused decode FFN
   int* h_hold = nullptr;          // mapped pinned flag that releases hold_kernel (stage timing)
   int* d_hold = nullptr;
@@ -766,7 +767,8 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
     dst.blob[dst.n] = list.blob[i];
     dst.n++;
   }
-  const bool split = !use_gemm && ready.n > 0 && later.n > 0;
+  // (not while stage timing: its events then time each launch over the forward's whole list)
+  const bool split = !use_gemm && ready.n > 0 && later.n > 0 && !se;
   if (!use_gemm && h->fused_ffn) {
     // one fused launch per group; the last one also runs the combine
     ftk::FusedParams fp{};
@@ -838,13 +840,15 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
       // gate/up | G1 | down of the ready group, the wait, then gate/up | G3 | down of the rest
       stage_mark(se, SE_G0, s);
       FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, ready, max_pairs, h->d_offsets,
-                                        h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr, h->d_err));
+                                        h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr, h->d_err,
+                                        h->int4_tensor != 0));
       stage_mark(se, SE_DA, s);
       rc = wait_fills();
       if (rc) return bail(rc, h->err);
       stage_mark(se, SE_G2, s);
       FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, later, max_pairs, h->d_offsets,
-                                        h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G3] : nullptr, h->d_err));
+                                        h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G3] : nullptr, h->d_err,
+                                        h->int4_tensor != 0));
       if (se) se->split = 1;
       h->perf.kernel_launches += 2;
     } else {
@@ -854,7 +858,8 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
       }
       stage_mark(se, SE_G0, s);
       FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, list, max_pairs, h->d_offsets,
-                                        h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr, h->d_err));
+                                        h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr, h->d_err,
+                                        h->int4_tensor != 0));
     }
     stage_mark(se, SE_D1, s);
     FT_CUDA(h, ftk::launch_combine(h->d_y, h->d_gates, h->d_inv, T, h->H, k, h->has_shared != 0,
@@ -893,6 +898,12 @@ int ft_moe_sync(ft_moe* h) {
     cudaMemset(h->d_err, 0, sizeof(int));
     return fail(h, FT_ERR_DEVICE_CHECK, "a kernel gave up waiting (code " + std::to_string(code) + ")");
   }
+  return FT_OK;
+}
+
+int ft_moe_set_int4_tensor_cores(ft_moe* h, int enabled) {
+  if (!h) return FT_ERR_INVALID;
+  h->int4_tensor = enabled != 0;
   return FT_OK;
 }
 

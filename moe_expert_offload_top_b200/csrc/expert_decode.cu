@@ -35,25 +35,6 @@ grouped_gemv_kernel(const void* __restrict__ xin, int T, int H, int I, int k,
                                       blockIdx.x, offsets, perm, hbuf, ybuf);
 }
 
-// Launches `kern`; with `dependent`, as a programmatic dependent launch of the
-// previous kernel on the stream (it may start before that kernel completes and must
-// order itself with griddepcontrol.wait).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, cudaStream_t s, bool dependent,
-                       Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = dependent ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
-}
-
 template <int MODE, int WT, int RPW>
 cudaError_t launch_gemv(int nt_max, dim3 grid, cudaStream_t s, const void* x, int T, int H, int I, int k,
                         const ExpertList& list, const int* offsets, const int* perm, float* h, float* y) {
@@ -133,9 +114,11 @@ static cudaError_t launch_pass(int nt, int rpw, int rows, cudaStream_t s, const 
 cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdtype,
                               const ExpertList& list, int max_pairs_per_expert, const int* offsets,
                               const int* perm, float* h, float* y, cudaStream_t s,
-                              cudaEvent_t between, int* err) {
+                              cudaEvent_t between, int* err, bool int4_tensor) {
   (void)err;
   if (list.n <= 0 || T <= 0) return cudaSuccess;
+  if (wdtype == WT_INT4 && int4_tensor)
+    return launch_ffn_int4_mma(x, T, H, I, k, list, offsets, perm, h, y, s, between);
   int nt = max_pairs_per_expert < T ? max_pairs_per_expert : T;
   if (nt < 1) nt = 1;
   auto bytes_of = [&](int K) -> size_t {

@@ -41,10 +41,15 @@ cudaError_t launch_permute(const int* ids, int T, int k, int E, int* counts, int
 // then the down projection into y [pairs][H] fp32.  Pairs are positions in the
 // permutation (routed) or T*k + t (shared expert).  `between` (optional) is recorded
 // on s between the two launches.
+// int4 weights run on the tensor cores (launch_ffn_int4_mma) unless int4_tensor is false;
+// h then holds each value as bf16 hi and lo halves (the row's first and second I uint16).
 cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdtype,
                               const ExpertList& list, int max_pairs_per_expert, const int* offsets,
                               const int* perm, float* h, float* y, cudaStream_t s,
-                              cudaEvent_t between = nullptr, int* err = nullptr);
+                              cudaEvent_t between = nullptr, int* err = nullptr, bool int4_tensor = true);
+// K3 (decode) for int4 group-128 weights with mma.sync (gemv_int4_mma.cu); x bf16.
+cudaError_t launch_ffn_int4_mma(const void* x, int T, int H, int I, int k, const ExpertList& list, const int* offsets,
+                                const int* perm, float* h, float* y, cudaStream_t s, cudaEvent_t between);
 // K3 + K5 (decode) in one launch (ffn_fused.cuh): gate/up + SwiGLU into h, down into y
 // and, with `combine`, out[t] = sum_j gates[t][j] * y[inv[t*k+j]] (+ shared) for the
 // entries of `list`.  The combine of a launch covers every pair of the forward, so
