@@ -113,6 +113,11 @@ struct ft_moe {
   uint16_t* d_ax = nullptr;       // gathered token rows for the prefill GEMMs
   ftk::GemmMaps maps;
   bool maps_dirty = true;
+  // NVFP4 prefill: the selected experts expanded to bf16 for the tcgen05 GEMMs
+  uint8_t* stage = nullptr;       // stage_cap bf16 expert blobs (3*H*I*2 bytes each)
+  int stage_cap = 0;
+  float* d_stage_gs = nullptr;    // 3 fp32 matrix scales per stage slot
+  ftk::GemmMaps smaps;            // a_x, a_h as maps; B maps over the stage
   int num_sms = 148;
   int gemm_min_avg_pairs = 32;    // tcgen05 path when bf16 and T*k/|S| >= this
   int fused_routing = 1;          // one-launch routing for decode-sized calls
@@ -233,7 +238,7 @@ int ensure_scratch(ft_moe* h, int T) {
             cudaMalloc(&h->d_y, sizeof(float) * rows * h->H) == cudaSuccess &&
             cudaHostAlloc(&h->h_box, sizeof(int) * (2 + pairs), cudaHostAllocMapped) == cudaSuccess &&
             cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->d_box), h->h_box, 0) == cudaSuccess &&
-            (h->wdtype != FT_W_BF16 ||
+            ((h->wdtype != FT_W_BF16 && h->wdtype != FT_W_NVFP4) ||
              cudaMalloc(&h->d_ax, sizeof(uint16_t) * rows * h->H) == cudaSuccess);
   if (!ok) {
     cudaGetLastError();
@@ -340,7 +345,28 @@ int issue_fills(ft_moe* h, std::vector<ftc::Access>& recs, size_t first) {
 }
 
 bool gemm_shapes_ok(const ft_moe* h) {
-  return h->wdtype == FT_W_BF16 && h->H % 256 == 0 && h->I % 128 == 0;
+  return (h->wdtype == FT_W_BF16 || h->wdtype == FT_W_NVFP4) && h->H % 256 == 0 && h->I % 128 == 0;
+}
+
+// Room for n bf16 expert blobs in the NVFP4 staging arena (grows only).
+int ensure_stage(ft_moe* h, int n) {
+  if (n <= h->stage_cap) return FT_OK;
+  if (h->has_last_stream) FT_CUDA(h, cudaStreamSynchronize(h->last_stream));
+  cudaFree(h->stage);
+  cudaFree(h->d_stage_gs);
+  h->stage = nullptr;
+  h->d_stage_gs = nullptr;
+  h->stage_cap = 0;
+  const size_t bytes = (size_t)n * 3 * h->H * h->I * 2;
+  if (cudaMalloc(&h->stage, bytes) != cudaSuccess || cudaMalloc(&h->d_stage_gs, sizeof(float) * 3 * n) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(h->stage);
+    h->stage = nullptr;
+    return fail(h, FT_ERR_OOM, "NVFP4 staging arena allocation failed");
+  }
+  h->stage_cap = n;
+  h->maps_dirty = true;
+  return FT_OK;
 }
 
 int ensure_maps(ft_moe* h) {
@@ -348,15 +374,26 @@ int ensure_maps(ft_moe* h) {
   const uint64_t rows = (uint64_t)h->cap_tokens * (h->k + 1);
   const uint64_t H = h->H, I = h->I;
   bool ok = ftk::encode_map_2d(&h->maps.a_x, h->d_ax, H, rows, H * 2, 128) &&
-            ftk::encode_map_2d(&h->maps.a_h, h->d_h, I, rows, I * 2, 128) &&
-            ftk::encode_map_3d(&h->maps.b1_routed, h->arena, H, 2 * I, h->C, H * 2, h->blob, 128) &&
-            ftk::encode_map_3d(&h->maps.b2_routed, h->arena + 2 * I * H * 2, I, H, h->C, I * 2, h->blob, 256);
-  if (ok && h->shared) {
+            ftk::encode_map_2d(&h->maps.a_h, h->d_h, I, rows, I * 2, 128);
+  // slot maps only where the slots hold bf16 blobs (NVFP4 stacks use the staged copies)
+  if (ok && h->wdtype == FT_W_BF16)
+    ok = ftk::encode_map_3d(&h->maps.b1_routed, h->arena, H, 2 * I, h->C, H * 2, h->blob, 128) &&
+         ftk::encode_map_3d(&h->maps.b2_routed, h->arena + 2 * I * H * 2, I, H, h->C, I * 2, h->blob, 256);
+  if (ok && h->shared && h->wdtype == FT_W_BF16) {
     ok = ftk::encode_map_3d(&h->maps.b1_shared, h->shared, H, 2 * I, h->L, H * 2, h->blob, 128) &&
          ftk::encode_map_3d(&h->maps.b2_shared, h->shared + 2 * I * H * 2, I, H, h->L, I * 2, h->blob, 256);
   } else {
     h->maps.b1_shared = h->maps.b1_routed;
     h->maps.b2_shared = h->maps.b2_routed;
+  }
+  if (ok && h->stage) {   // staged NVFP4 experts: routed and shared alike, slot z = list index
+    const uint64_t sblob = 3 * H * I * 2;
+    h->smaps.a_x = h->maps.a_x;
+    h->smaps.a_h = h->maps.a_h;
+    ok = ftk::encode_map_3d(&h->smaps.b1_routed, h->stage, H, 2 * I, h->stage_cap, H * 2, sblob, 128) &&
+         ftk::encode_map_3d(&h->smaps.b2_routed, h->stage + 2 * I * H * 2, I, H, h->stage_cap, I * 2, sblob, 256);
+    h->smaps.b1_shared = h->smaps.b1_routed;
+    h->smaps.b2_shared = h->smaps.b2_routed;
   }
   if (!ok) return fail(h, FT_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   h->maps_dirty = false;
@@ -816,22 +853,33 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
         rc = wait_fills();
         if (rc) return bail(rc, h->err);
       }
+      const bool staged = h->wdtype == FT_W_NVFP4;   // expanded to bf16 for the tensor cores
+      if (staged) {
+        rc = ensure_stage(h, list.n);
+        if (rc) return bail(rc, h->err);
+      }
       rc = ensure_maps(h);
       if (rc) return rc;
       ftk::GemmGroups groups;
       groups.n = list.n;
       for (int i = 0; i < list.n; ++i) {
         groups.expert[i] = list.expert[i];
-        groups.z[i] = list.expert[i] >= 0 ? h->lru.slot_of(layer * E + list.expert[i]) : layer;
+        groups.z[i] = staged ? i : list.expert[i] >= 0 ? h->lru.slot_of(layer * E + list.expert[i]) : layer;
       }
+      if (staged) {
+        FT_CUDA(h, ftk::launch_dequant_nvfp4_stage(list, h->H, h->I, h->stage, h->d_stage_gs, h->num_sms, s));
+        h->perf.kernel_launches += 1;
+      }
+      const ftk::GemmMaps& gm = staged ? h->smaps : h->maps;
+      const float* gsc = staged ? h->d_stage_gs : nullptr;
       FT_CUDA(h, ftk::launch_gather_rows(x, h->d_perm, T, k, h->H, h->has_shared != 0, h->d_ax, s));
       h->perf.kernel_launches += 1;
       stage_mark(se, SE_G0, s);
-      FT_CUDA(h, ftk::launch_grouped_gemm(0, h->maps, groups, h->d_offsets, T, k, h->I, h->H, h->d_h,
-                                          h->d_err, h->num_sms, s));
+      FT_CUDA(h, ftk::launch_grouped_gemm(0, gm, groups, h->d_offsets, T, k, h->I, h->H, h->d_h,
+                                          h->d_err, h->num_sms, s, gsc));
       stage_mark(se, SE_G1, s);
-      FT_CUDA(h, ftk::launch_grouped_gemm(1, h->maps, groups, h->d_offsets, T, k, h->I, h->H, h->d_y,
-                                          h->d_err, h->num_sms, s));
+      FT_CUDA(h, ftk::launch_grouped_gemm(1, gm, groups, h->d_offsets, T, k, h->I, h->H, h->d_y,
+                                          h->d_err, h->num_sms, s, gsc));
       if (se) {   // bf16 h, and the weights of each listed expert read once
         se->gu_bytes = list.n * 2.0 * h->H * h->I * 2 + pairs * (h->H * 2.0 + h->I * 2.0);
         se->d_bytes = list.n * 1.0 * h->H * h->I * 2 + pairs * (h->I * 2.0 + h->H * 4.0);
@@ -1111,6 +1159,8 @@ void ft_moe_destroy(ft_moe* h) {
   cudaFree(h->d_err);
   cudaFree(h->d_ticket);
   cudaFree(h->d_ctl);
+  cudaFree(h->stage);
+  cudaFree(h->d_stage_gs);
   if (h->h_err) cudaFreeHost(h->h_err);
   if (h->h_hold) cudaFreeHost(h->h_hold);
   if (h->copy) cudaStreamDestroy(h->copy);

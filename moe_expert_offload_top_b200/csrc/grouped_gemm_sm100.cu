@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmBr,
                     const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ GemmGroups groups,
                     const int* __restrict__ offsets, int T, int k, int I, int H,
-                    void* __restrict__ out, int* __restrict__ err) {
+                    void* __restrict__ out, int* __restrict__ err, const float* __restrict__ gscale) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   GemmSmem* S = reinterpret_cast<GemmSmem*>(base + STAGES * STAGE_BYTES);
@@ -242,6 +242,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const int valid = S->rows[g] - m * BM;
       const int row = S->row_start[g] + m * BM + r;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + b * BN;
+      // per-matrix fp32 scales of staged NVFP4 weights (gate, up, down of stage slot z)
+      const float* gs = gscale ? gscale + 3 * groups.z[g] : nullptr;
       if (MODE == 0) {
         uint16_t* hout = static_cast<uint16_t*>(out) + (size_t)row * ld_out + n * (BN / 2);
 #pragma unroll 1
@@ -249,6 +251,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           float u[32], v[32];
           tmem_ld32(tbase + j, u);
           tmem_ld32(tbase + BN / 2 + j, v);
+          if (gs) {
+            const float sg = gs[0], su = gs[1];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) { u[i] *= sg; v[i] *= su; }
+          }
           if (r < valid) {
             uint32_t pk[16];
 #pragma unroll
@@ -267,6 +274,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         for (int j = 0; j < BN; j += 32) {
           float v[32];
           tmem_ld32(tbase + j, v);
+          if (gs) {
+            const float sd = gs[2];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= sd;
+          }
           if (r < valid) {
             float4* dst = reinterpret_cast<float4*>(yout + j);
 #pragma unroll
@@ -334,7 +346,8 @@ cudaError_t launch_gather_rows(const void* x, const int* perm, int T, int k, int
 }
 
 cudaError_t launch_grouped_gemm(int mode, const GemmMaps& maps, const GemmGroups& groups, const int* offsets,
-                                int T, int k, int I, int H, void* out, int* err, int num_sms, cudaStream_t s) {
+                                int T, int k, int I, int H, void* out, int* err, int num_sms, cudaStream_t s,
+                                const float* gscale) {
   if (groups.n <= 0 || T <= 0) return cudaSuccess;
   const size_t smem = gemm_smem_bytes();
   // an upper bound of the tile count; CTAs beyond the real count exit at once
@@ -347,12 +360,12 @@ cudaError_t launch_grouped_gemm(int mode, const GemmMaps& maps, const GemmGroups
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     grouped_gemm_kernel<0><<<grid, GEMM_THREADS, smem, s>>>(maps.a_x, maps.b1_routed, maps.b1_shared, groups,
-                                                            offsets, T, k, I, H, out, err);
+                                                            offsets, T, k, I, H, out, err, gscale);
   } else {
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     grouped_gemm_kernel<1><<<grid, GEMM_THREADS, smem, s>>>(maps.a_h, maps.b2_routed, maps.b2_shared, groups,
-                                                            offsets, T, k, I, H, out, err);
+                                                            offsets, T, k, I, H, out, err, gscale);
   }
   return cudaGetLastError();
 }

@@ -121,8 +121,16 @@ cudaError_t launch_wait_selftest(unsigned long long limit_ns, int* err, cudaStre
 cudaError_t launch_gather_rows(const void* x, const int* perm, int T, int k, int H, bool with_shared,
                                void* A, cudaStream_t s);
 // mode 0: h = silu(A W_gate^T) * (A W_up^T) (bf16 [rows][I]); mode 1: y = h W_down^T (f32 [rows][H]).
+// gscale (optional, device): 3 fp32 scales (gate, up, down) per weight slot z, applied to the
+// accumulators (staged NVFP4 weights); null for bf16 weights.
 cudaError_t launch_grouped_gemm(int mode, const GemmMaps& maps, const GemmGroups& groups, const int* offsets,
-                                int T, int k, int I, int H, void* out, int* err, int num_sms, cudaStream_t s);
+                                int T, int k, int I, int H, void* out, int* err, int num_sms, cudaStream_t s,
+                                const float* gscale = nullptr);
+// Expands the NVFP4 blobs of list's entries to bf16 (e2m1 * e4m3, exact) in stage slot i
+// (3*H*I bf16 per slot, the bf16 blob layout) and writes their fp32 matrix scales to
+// gscale[3i .. 3i+2] (dequant_stage.cu).
+cudaError_t launch_dequant_nvfp4_stage(const ExpertList& list, int H, int I, void* stage, float* gscale, int num_sms,
+                                       cudaStream_t s);
 // 2-D / 3-D bf16 tensor maps with 128-byte swizzle (box inner extent 64 elements).
 bool encode_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
                    uint32_t box_rows);

@@ -100,6 +100,22 @@ def test_prefill_gemm_and_gemv_paths_match_oracle(gemm_threshold):
     assert st["misses"] == 0 and st["prefetch_misses"] == 2 * 16
 
 
+@pytest.mark.parametrize("gemm_threshold", [0, 1 << 30])
+def test_nvfp4_prefill_staged_gemm_and_gemv_paths_match_oracle(gemm_threshold):
+    # NVFP4 stacks in prefill: the selected experts are expanded to bf16 (exact) for the
+    # tcgen05 GEMMs, whose epilogue applies each matrix's fp32 scale; or the GEMV path
+    cfg = synth.MoeConfig("prefill-nvfp4", L=2, E=16, H=512, I=256, k=4, gating="sigmoid", wdtype="nvfp4",
+                          shared=True, C=32, tokens=700, batches=(700,), process="iid", mode="prefill")
+    st = run_and_check(cfg, 700, sample_steps=[0], gemm_threshold=gemm_threshold)
+    assert st["misses"] == 0 and st["prefetch_misses"] == 2 * 16
+
+
+def test_nvfp4_staged_gemm_uneven_groups():
+    cfg = synth.MoeConfig("skew-nvfp4", L=1, E=8, H=768, I=384, k=2, gating="softmax", wdtype="nvfp4",
+                          shared=False, C=8, tokens=400, batches=(400,), process="ar1", mode="decode")
+    run_and_check(cfg, 400, sample_steps=[0], gemm_threshold=0)
+
+
 def test_gemm_path_uneven_groups_and_many_tiles():
     # one hot expert with > 2 M-tiles, others tiny; H, I at the multiples the tiles need
     cfg = synth.MoeConfig("skew", L=1, E=8, H=768, I=384, k=2, gating="softmax", wdtype="bf16",
