@@ -348,6 +348,14 @@ FT_API int ft_cache_simulate_policy(int policy, int num_layers, int num_experts,
  * timed with CUDA events on a private stream.  Allocates and frees its own buffers. */
 FT_API int ft_probe_host_link(size_t bytes, int iters, double* h2d_gbs, double* d2h_gbs);
 
+/* Host memory copy bandwidth (no GPU): `iters` memcpy passes of `bytes` between two
+ * host buffers, split over `threads` threads (1..256), timed with a steady clock.
+ * *gbs = bytes * iters / seconds / 1e9 (copied bytes, not read + written).  With the
+ * link probe it forms the bandwidth profile a CPU/GPU placement policy would read
+ * ("FreeToken linux": the bandwidth check of the setup).  Allocates and frees its own
+ * buffers; FT_ERR_OOM if they cannot be allocated. */
+FT_API int ft_probe_host_memory(size_t bytes, int threads, int iters, double* gbs);
+
 /* ------------------------------------------------------------------------ *
  * Step-level kernels.  Each runs one step of the forward on caller-owned device
  * buffers, on `stream`, without the cache.  They are the same kernels the

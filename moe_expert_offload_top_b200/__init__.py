@@ -106,6 +106,7 @@ _SIGS = {
     "ft_cache_simulate_policy": ([_i, _i, _i, _i, _vp, _i, _vp, _i, ctypes.POINTER(_i),
                                   ctypes.POINTER(ft_cache_stats_t), ctypes.POINTER(_i)], _i),
     "ft_probe_host_link": ([_sz, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)], _i),
+    "ft_probe_host_memory": ([_sz, _i, _i, ctypes.POINTER(ctypes.c_double)], _i),
     "ft_cache_simulate": ([_i, _i, _i, _vp, _i, _vp, _i, ctypes.POINTER(_i),
                            ctypes.POINTER(ft_cache_stats_t), ctypes.POINTER(_i)], _i),
 }
@@ -382,6 +383,12 @@ def ft_probe_host_link(bytes_, iters=5):
     a, b = ctypes.c_double(0), ctypes.c_double(0)
     _check(None, _lib.ft_probe_host_link(bytes_, iters, ctypes.byref(a), ctypes.byref(b)))
     return a.value, b.value
+
+
+def ft_probe_host_memory(bytes_, threads=1, iters=3):
+    g = ctypes.c_double(0)
+    _check(None, _lib.ft_probe_host_memory(bytes_, threads, iters, ctypes.byref(g)))
+    return g.value
 
 
 def ft_version():

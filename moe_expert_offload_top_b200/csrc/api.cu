@@ -125,6 +125,7 @@ struct ft_moe {
   int inject_route_timeout = 0;   // countdown to a simulated routing-wait timeout
   int inject_fused_wait = 0;      // countdown to a fused decode FFN launch whose waits run out
   cudaEvent_t route_ev = nullptr;
+  cudaEvent_t xs_ev = nullptr;    // orders a forward after the previous stream's work
   int last_T = 0;
   int fused_ffn = 0;              // decode FFN + combine as one launch (ffn_decode_fused_kernel)
   int int4_tensor = 1;            // int4 decode GEMV on the tensor cores (mma.sync)
@@ -541,6 +542,7 @@ ft_moe* ft_moe_create(int num_experts, int top_k, int hidden, int inter, int wdt
     h->fill_ev_batch[i] = -1;
   }
   cudaEventCreateWithFlags(&h->route_ev, cudaEventDisableTiming);
+  cudaEventCreateWithFlags(&h->xs_ev, cudaEventDisableTiming);
   cudaMalloc(&h->d_err, sizeof(int));
   cudaMemset(h->d_err, 0, sizeof(int));
   cudaMalloc(&h->d_ticket, sizeof(int));
@@ -647,10 +649,11 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   const int T = n_tokens, E = h->E, k = h->k;
   int rc = ensure_scratch(h, T);
   if (rc) return rc;
-  // keep forwards of this handle ordered across streams
+  // keep forwards of this handle ordered across streams: all work queued so far on the
+  // previous stream completes before this call's first kernel
   if (h->has_last_stream && s != h->last_stream && h->call > 0) {
-    const int r = (int)((h->call - 1) % kRing);
-    FT_CUDA(h, cudaStreamWaitEvent(s, h->use_ev[r], 0));
+    FT_CUDA(h, cudaEventRecord(h->xs_ev, h->last_stream));
+    FT_CUDA(h, cudaStreamWaitEvent(s, h->xs_ev, 0));
   }
   const bool xbf16 = h->wdtype != FT_W_F32;
   if (h->stage_pending.size() > 256) harvest_stages(h, false);
@@ -790,6 +793,16 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
     se->d_bytes = list.n * wmat + pairs * (h->I * 4.0 + h->H * 4.0);
     se->flops = pairs * 6.0 * mat;
   }
+  // The slots of this call are read by the gate/up and down kernels only: use_ev marks
+  // their end (the copy stream waits on it before overwriting a slot).  Recorded before
+  // the combine, so that the next forward's routing kernel can follow the combine
+  // directly (programmatic dependent launch).
+  auto record_use = [&]() -> int {
+    const int r = (int)(call % kRing);
+    FT_CUDA(h, cudaEventRecord(h->use_ev[r], s));
+    h->use_ev_call[r] = call;
+    return FT_OK;
+  };
   hold.begin(h, se, s);
   const bool use_gemm = gemm_shapes_ok(h) && (long long)T * k >= (long long)h->gemm_min_avg_pairs * (long long)S.size();
   // Decode path: entries whose slots this stream has already waited for (and the shared
@@ -847,6 +860,8 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
       h->perf.kernel_launches += 1;
     }
     stage_mark(se, SE_C1, s);
+    rc = record_use();
+    if (rc) return rc;
   } else {
     if (use_gemm) {
       if (must_wait) {
@@ -910,18 +925,15 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
                                         h->int4_tensor != 0));
     }
     stage_mark(se, SE_D1, s);
+    rc = record_use();
+    if (rc) return rc;
     FT_CUDA(h, ftk::launch_combine(h->d_y, h->d_gates, h->d_inv, T, h->H, k, h->has_shared != 0,
                                    xbf16, out, s));
     stage_mark(se, SE_C1, s);
     h->perf.kernel_launches += 3;
   }
   hold.release();
-  {
-    const int r = (int)(call % kRing);
-    FT_CUDA(h, cudaEventRecord(h->use_ev[r], s));
-    h->use_ev_call[r] = call;
-    for (int key : keys) h->slot_last_use[h->lru.slot_of(key)] = call;
-  }
+  for (int key : keys) h->slot_last_use[h->lru.slot_of(key)] = call;
   h->last_stream = s;
   h->has_last_stream = true;
   h->call++;
@@ -1152,6 +1164,7 @@ void ft_moe_destroy(ft_moe* h) {
     if (h->fill_ev[i]) cudaEventDestroy(h->fill_ev[i]);
   }
   if (h->route_ev) cudaEventDestroy(h->route_ev);
+  if (h->xs_ev) cudaEventDestroy(h->xs_ev);
   harvest_stages(h, true);
   for (auto& se : h->stage_free)
     for (int i = 0; i < SE_N; ++i) cudaEventDestroy(se.ev[i]);
@@ -1262,6 +1275,33 @@ int ft_probe_host_link(size_t bytes, int iters, double* h2d_gbs, double* d2h_gbs
   if (dbuf) cudaFree(dbuf);
   if (hbuf) cudaFreeHost(hbuf);
   return rc;
+}
+
+int ft_probe_host_memory(size_t bytes, int threads, int iters, double* gbs) {
+  if (bytes < 4096 || threads < 1 || threads > 256 || iters < 1 || !gbs) return FT_ERR_INVALID;
+  std::vector<uint8_t> src, dst;
+  try {
+    src.assign(bytes, 1);
+    dst.assign(bytes, 0);
+  } catch (...) {
+    return FT_ERR_OOM;
+  }
+  auto pass = [&]() {
+    std::vector<std::thread> pool;
+    const size_t per = (bytes + threads - 1) / threads;
+    for (int t = 0; t < threads; ++t) {
+      const size_t b0 = std::min(bytes, (size_t)t * per), b1 = std::min(bytes, b0 + per);
+      if (b1 > b0) pool.emplace_back([&, b0, b1] { memcpy(dst.data() + b0, src.data() + b0, b1 - b0); });
+    }
+    for (auto& th : pool) th.join();
+  };
+  pass();   // warm-up: touches every page
+  const auto t0 = std::chrono::steady_clock::now();
+  for (int it = 0; it < iters; ++it) pass();
+  const double sec = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+  if (sec <= 0.0) return FT_ERR_INVALID;
+  *gbs = (double)bytes * iters / sec / 1e9;
+  return FT_OK;
 }
 
 int ft_cache_simulate(int num_layers, int num_experts, int capacity, const int* ops,

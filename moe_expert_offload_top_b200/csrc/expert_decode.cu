@@ -55,6 +55,8 @@ template <bool OUT_BF16>
 __global__ void combine_kernel(const float* __restrict__ y, const float* __restrict__ gates,
                                const int* __restrict__ inv, int T, int H, int k, int has_shared,
                                void* __restrict__ out) {
+  // the next forward's routing kernel may launch now (it waits for this grid itself)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int per_tok = H / 4;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;

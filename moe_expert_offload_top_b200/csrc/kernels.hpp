@@ -7,7 +7,10 @@
 
 namespace ftk {
 
-constexpr int kMaxList = 257;   // routed experts of one layer + the shared expert
+#ifndef FT_MAX_LIST
+#define FT_MAX_LIST 257
+#endif
+constexpr int kMaxList = FT_MAX_LIST;   // routed experts of one layer + the shared expert
 
 // Per-launch list of experts whose FFN runs: entry i reads its weights at blob[i];
 // its token pairs are offsets[expert[i]] .. offsets[expert[i]+1] of the permutation,

@@ -6,6 +6,7 @@
 // the lower expert index) and their gates are the softmax, or the sigmoid,
 // of the selected logits normalised to sum to 1.
 #include "common.cuh"
+#include "decode_gemv.cuh"
 #include "kernels.hpp"
 
 namespace ftk {
@@ -205,6 +206,15 @@ route_decode_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T
   __shared__ int s_ids[64 * 16];
   const int e0 = blockIdx.x * kRouterEPB, t0 = blockIdx.y * kRouterTPB;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Launched as a programmatic dependent of the previous kernel on the stream: the
+  // router rows do not depend on it, so they are brought toward L2 first (one prefetch
+  // per 128-byte line); everything the previous kernel may write or read (x, the
+  // routing buffers, the ticket) is touched only after griddepcontrol.wait.
+  for (int i = 0; i < kRouterEPB; ++i)
+    if (e0 + i < E)
+      for (int hh = threadIdx.x * 32; hh < H; hh += kRouterThreads * 32)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(__cvta_generic_to_global(w + (size_t)(e0 + i) * H + hh)));
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   {  // ---- logits of this CTA's experts and tokens (as router_logits_kernel)
     float acc[kRouterEPB][kRouterTPB];
 #pragma unroll
@@ -408,15 +418,15 @@ cudaError_t launch_route_decode(const void* x, bool x_bf16, const float* w_route
   if (T <= 0) return cudaSuccess;
   if (T > 64 || E > 256 || k > 16) return cudaErrorInvalidValue;
   dim3 grid((E + kRouterEPB - 1) / kRouterEPB, (T + kRouterTPB - 1) / kRouterTPB);
+  // programmatic dependent launch: may start while the previous kernel (the last forward's
+  // combine) finishes; the kernel orders itself with griddepcontrol.wait
   if (x_bf16)
-    route_decode_kernel<uint16_t><<<grid, kRouterThreads, 0, s>>>(static_cast<const uint16_t*>(x), w_router, T, H,
-                                                                  E, k, gating, logits, ids, gates, counts, offsets,
-                                                                  perm, inv, ticket, box, seq, err);
-  else
-    route_decode_kernel<float><<<grid, kRouterThreads, 0, s>>>(static_cast<const float*>(x), w_router, T, H, E, k,
-                                                               gating, logits, ids, gates, counts, offsets, perm,
-                                                               inv, ticket, box, seq, err);
-  return cudaGetLastError();
+    return gemv::launch_pdl(route_decode_kernel<uint16_t>, grid, dim3(kRouterThreads), s, true,
+                            static_cast<const uint16_t*>(x), w_router, T, H, E, k, gating, logits, ids, gates, counts,
+                            offsets, perm, inv, ticket, box, seq, err);
+  return gemv::launch_pdl(route_decode_kernel<float>, grid, dim3(kRouterThreads), s, true,
+                          static_cast<const float*>(x), w_router, T, H, E, k, gating, logits, ids, gates, counts,
+                          offsets, perm, inv, ticket, box, seq, err);
 }
 
 cudaError_t launch_router_logits(const void* x, bool x_bf16, const float* w_router, int T, int H,

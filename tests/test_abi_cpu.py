@@ -156,3 +156,16 @@ def test_lru_beats_static_split_on_locality_traces():
         rates[pol] = st["misses"] / st["routed"]
     assert rates[ft.FT_POLICY_LRU] < 0.5 * rates[ft.FT_POLICY_STATIC]
     assert 0.3 < rates[ft.FT_POLICY_STATIC] < 0.9
+
+
+def test_bandwidth_profile_host_part(tmp_path):
+    # the host half of the bandwidth profile runs without a GPU and writes its file
+    from moe_expert_offload_top_b200 import bwprofile
+    out = tmp_path / "bw.json"
+    assert bwprofile.main(["--host-only", "--out", str(out), "--bytes", str(1 << 22), "--iters", "2"]) == 0
+    import json
+    prof = json.loads(out.read_text())
+    assert prof["host_memcpy_gbs_1_thread"] > 0 and prof["host_memcpy_gbs_all_threads"] > 0
+    assert "h2d_gbs" not in prof
+    with pytest.raises(ft.FtError):
+        ft.ft_probe_host_memory(16, 1, 1)          # below the minimum size
