@@ -83,16 +83,11 @@ int4_mma_kernel(const uint16_t* __restrict__ x, int T, int H, int I, int k, cons
                 float* __restrict__ ybuf) {
   constexpr bool GU = MODE == 0;
   constexpr int NM = GU ? 2 : kDownTiles;   // 16x(K) weight tiles per CTA: gate and up, or down row tiles
-  if (GU) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  else asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float red[kQWarps][NM][16][8];
   const int e = list.expert[blockIdx.y];
   const uint8_t* blob = list.blob[blockIdx.y];
   const int K = GU ? H : I, rows = GU ? I : H;
   const int row0 = blockIdx.x * (GU ? 16 : 16 * kDownTiles);
-  const int q0 = e >= 0 ? offsets[e] : T * k;
-  const int q1 = e >= 0 ? offsets[e + 1] : T * k + T;
-  if (q1 <= q0 || row0 >= rows) return;   // the same for the whole CTA
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const size_t mat = (size_t)H * I;
   const uint16_t* sc = reinterpret_cast<const uint16_t*>(blob + 3 * mat / 2);
@@ -117,6 +112,11 @@ int4_mma_kernel(const uint16_t* __restrict__ x, int T, int H, int I, int k, cons
     }
   }
   const int b0 = warp * nb / kQWarps, b1 = (warp + 1) * nb / kQWarps;
+  if (GU) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  else asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int q0 = e >= 0 ? offsets[e] : T * k;
+  const int q1 = e >= 0 ? offsets[e + 1] : T * k + T;
+  if (q1 <= q0 || row0 >= rows) return;   // the same for the whole CTA
 
   for (int c0 = q0; c0 < q1; c0 += 8) {
     const int nt = min(8, q1 - c0);

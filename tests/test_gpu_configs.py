@@ -50,6 +50,11 @@ def run_and_check(cfg, batch, sample_steps, sample_tokens=None, gemm_threshold=N
                 outs[s] = out.float().cpu().numpy().copy()
         ft.ft_moe_sync(st.h)
         trace = st.trace()
+        if stack is not None and trace:
+            # a shared stack keeps counting forward calls across runs (the cache clear keeps
+            # the handle's counters): number this run's calls from 0, as the oracle does
+            base = trace[0][0]
+            trace = [(t[0] - base,) + tuple(t[1:]) for t in trace]
         stats = st.stats()
         # oracle: routing, cache trace, sampled outputs
         routers = [synth.router_weights(cfg, l) for l in range(cfg.L)]
