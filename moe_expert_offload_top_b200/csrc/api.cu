@@ -184,18 +184,26 @@ int wait_event(ft_moe* h, cudaEvent_t ev, const char* what) {
   }
 }
 
-// Host wait for the fused routing kernel's mailbox (mapped pinned memory): returns once
-// box[0] == seq.  Polls the routing event now and then to catch a failed kernel, and
-// gives up after the handle's deadline.
-int wait_box(ft_moe* h, int seq) {
-  const volatile int* flag = h->h_box;
+// Host wait for the fused routing kernel's mailbox (mapped pinned memory): every word
+// box[1] (error word) and box[2 .. 2+n) (ids) carries the call's tag above a 10-bit
+// value.  Returns once all of them show this call's tag, leaving the plain values in
+// place.  Polls the routing event now and then to catch a failed kernel, and gives up
+// after the handle's deadline.
+int wait_box(ft_moe* h, int seq, int n) {
+  volatile int* box = h->h_box;
+  auto tagged = [&]() {
+    if ((box[1] >> 10) != seq) return false;
+    for (int p = 0; p < n; ++p)
+      if ((box[2 + p] >> 10) != seq) return false;
+    return true;
+  };
   auto t0 = std::chrono::steady_clock::now();
   for (unsigned it = 1;; ++it) {
-    if (*flag == seq) break;
+    if (tagged()) break;
     if ((it & 255) == 0) {
       const cudaError_t q = cudaEventQuery(h->route_ev);
       if (q == cudaSuccess) {
-        if (*flag == seq) break;
+        if (tagged()) break;
         return fail(h, FT_ERR_CUDA, "routing kernel finished without publishing its ids");
       }
       if (q != cudaErrorNotReady) return cuda_fail(h, q, "routing ids");
@@ -205,7 +213,15 @@ int wait_box(ft_moe* h, int seq) {
     }
   }
   std::atomic_thread_fence(std::memory_order_acquire);
+  box[1] &= 0x3FF;
+  for (int p = 0; p < n; ++p) box[2 + p] &= 0x3FF;
   return FT_OK;
+}
+
+// Tag of the next fused routing call's mailbox words: 1 .. 2^21 - 1, never 0.
+int next_route_seq(ft_moe* h) {
+  h->route_seq = h->route_seq % ((1 << 21) - 1) + 1;
+  return h->route_seq;
 }
 
 void free_scratch(ft_moe* h) {
@@ -246,7 +262,7 @@ int ensure_scratch(ft_moe* h, int T) {
     free_scratch(h);
     return fail(h, FT_ERR_OOM, "scratch allocation failed");
   }
-  h->h_box[0] = h->h_box[1] = 0;
+  memset(h->h_box, 0, sizeof(int) * (2 + pairs));   // tag 0: never a call's tag
   h->h_ids = h->h_box + 2;
   h->cap_tokens = T;
   return FT_OK;
@@ -667,7 +683,7 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
     // the kernel also publishes the ids and the error word to the host mailbox
     FT_CUDA(h, ftk::launch_route_decode(x, xbf16, router_w, T, h->H, E, k, h->gating, h->d_logits, h->d_ids,
                                         h->d_gates, h->d_counts, h->d_offsets, h->d_perm, h->d_inv,
-                                        h->d_ticket, s, h->d_box, ++h->route_seq, h->d_err));
+                                        h->d_ticket, s, h->d_box, next_route_seq(h), h->d_err));
     stage_mark(se, SE_R1, s);
     FT_CUDA(h, cudaEventRecord(h->route_ev, s));
     stage_mark(se, SE_P0, s);
@@ -698,7 +714,7 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
       cudaEventSynchronize(h->route_ev);   // the work itself completes; only the report is injected
       return fail(h, FT_ERR_TIMEOUT, "timed out waiting for routing ids (injected)");
     }
-    rc = fused_route ? wait_box(h, h->route_seq) : wait_event(h, h->route_ev, "routing ids");
+    rc = fused_route ? wait_box(h, h->route_seq, T * k) : wait_event(h, h->route_ev, "routing ids");
     h->perf.host_wait_ms +=
         std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - w0).count();
   }

@@ -29,9 +29,9 @@ cudaError_t launch_topk_gates(const float* logits, int T, int E, int k, int gati
 // K1+K2 for decode (T <= 64, E <= 256, k <= 16) in one launch: logits, top-k + gates and
 // the stable permutation (the last router CTA does the second part).  *ticket must be 0
 // before the launch; the kernel leaves it 0.  box (optional, mapped pinned host memory of
-// 2 + T*k ints): the last CTA also writes the ids to box[2..], *err to box[1] and then,
-// after a system-scope fence, seq to box[0], so the host can take the routing as soon as
-// it exists.
+// 2 + T*k ints): the last CTA also writes seq << 10 | value to box[2 + p] (the ids, < 1024)
+// and box[1] (the low 10 bits of *err), so the host can take the routing as soon as every
+// word shows the tag; seq is in 1 .. 2^21 - 1.
 cudaError_t launch_route_decode(const void* x, bool x_bf16, const float* w_router, int T, int H, int E, int k,
                                 int gating, float* logits, int* ids, float* gates, int* counts, int* offsets,
                                 int* perm, int* inv, int* ticket, cudaStream_t s, int* box = nullptr,

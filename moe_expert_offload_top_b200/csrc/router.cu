@@ -262,9 +262,9 @@ route_decode_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T
         for (int wp = 0; wp < kRouterThreads / 32; ++wp) sum += part[wp][i][t];
         z[(size_t)(t0 + t) * E + e0 + i] = sum;
       }
+      __threadfence();   // the logit writers publish before the ticket
     }
   }
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
     const int nblocks = gridDim.x * gridDim.y;
@@ -272,7 +272,7 @@ route_decode_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T
   }
   __syncthreads();
   if (!last) return;
-  __threadfence();
+  if (warp < T) __threadfence();   // the warps that read the logits
   // ---- top-k + gates: one warp per token, logits read through L2
   for (int t = warp; t < T; t += kRouterThreads / 32) {
     float v[8];
@@ -385,13 +385,14 @@ route_decode_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T
     }
   }
   if (box) {
-    // publish to the host through mapped pinned memory: ids and the device error word,
-    // then (after a system-scope fence) the sequence number the host waits for
-    for (int p = threadIdx.x; p < n; p += kRouterThreads) box[2 + p] = s_ids[p];
-    if (threadIdx.x == 0) box[1] = *reinterpret_cast<const volatile int*>(err);
-    __threadfence_system();
-    __syncthreads();
-    if (threadIdx.x == 0) *reinterpret_cast<volatile int*>(box) = seq;
+    // publish to the host through mapped pinned memory: every word carries the call's
+    // tag (seq, 1 .. 2^21-1) above a 10-bit value (an id, or the device error word), so
+    // the host takes the words once all of them show the tag, whatever order they
+    // arrive in; no system-scope fence is needed.
+    const int tag = seq << 10;
+    volatile int* vb = reinterpret_cast<volatile int*>(box);
+    for (int p = threadIdx.x; p < n; p += kRouterThreads) vb[2 + p] = tag | s_ids[p];
+    if (threadIdx.x == 0) vb[1] = tag | (*reinterpret_cast<const volatile int*>(err) & 0x3FF);
   }
   if (threadIdx.x == 0) *ticket = 0;
 }
