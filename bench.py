@@ -369,7 +369,8 @@ def run_ours(args):
     barrier(dev)
     clk = clocks.stop()
     dt = e0.elapsed_time(e1) * 1e-3
-    launches = ft.ft_moe_perf(stack.h)["kernel_launches"]
+    perf_dev = ft.ft_moe_perf(stack.h)      # the uninstrumented leg's counters
+    launches = perf_dev["kernel_launches"]
     st = stack.stats()
     tokens, t_max = aggregate(K * cfg.batches[0], dt, dev)
 
@@ -452,6 +453,7 @@ def run_ours(args):
             "stages_us_per_forward": {k2: 1e3 * perf[k2 + "_ms"] / fwd for k2 in
                                       ("router", "permute", "ffn_gate_up", "ffn_down", "combine", "ffn_fused")},
             "host_wait_us_per_forward": 1e3 * perf["host_wait_ms"] / max(perf["forwards"], 1),
+            "host_issue_us_per_forward": 1e3 * perf_dev["host_issue_ms"] / max(perf_dev["forwards"], 1),
         }
         if world == 1 and args.prefill:
             line["prefill"] = run_prefill_leg(args, dev)

@@ -290,6 +290,8 @@ typedef struct {
   double ffn_fused_bytes;
   long long ffn_fused_launches;
   long long ffn_gate_up_launches;   /* per-pass gate/up launches (two where a forward is split) */
+  double host_issue_ms;  /* host time from the routing's arrival to the last launch queued: the
+                            LRU, the fills and the FFN launches (on the path of every forward) */
 } ft_perf_t;
 
 /* Stage timing holds the forward's stream with a one-thread kernel while the host queues

@@ -52,7 +52,8 @@ class ft_perf_t(ctypes.Structure):
                 ("ffn_gate_up_bytes", ctypes.c_double), ("ffn_down_bytes", ctypes.c_double),
                 ("ffn_flops", ctypes.c_double), ("host_wait_ms", ctypes.c_double),
                 ("ffn_fused_ms", ctypes.c_double), ("ffn_fused_bytes", ctypes.c_double),
-                ("ffn_fused_launches", ctypes.c_longlong), ("ffn_gate_up_launches", ctypes.c_longlong)]
+                ("ffn_fused_launches", ctypes.c_longlong), ("ffn_gate_up_launches", ctypes.c_longlong),
+                ("host_issue_ms", ctypes.c_double)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

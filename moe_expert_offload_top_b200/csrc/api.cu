@@ -719,6 +719,7 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
         std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - w0).count();
   }
   if (rc) return rc;
+  const auto t_routed = std::chrono::steady_clock::now();   // the routing is on the host
   h->last_T = T;
   // A failure from here on leaves no kernel of this call running: the caller's stream is
   // drained first, so a following forward on another stream cannot race on the scratch.
@@ -950,6 +951,8 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   }
   hold.release();
   for (int key : keys) h->slot_last_use[h->lru.slot_of(key)] = call;
+  h->perf.host_issue_ms +=
+      std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - t_routed).count();
   h->last_stream = s;
   h->has_last_stream = true;
   h->call++;
