@@ -150,11 +150,7 @@ cudaError_t launch_inst(const FusedParams& p, const ExpertList& list, int num_sm
   const long long nA = (p.I + kWarps * RG - 1) / (kWarps * RG);
   const long long nB = (p.H + kWarps * RD - 1) / (kWarps * RD);
   const long long tot = (long long)list.n * (nA + nB);
-#ifdef FT_FUSED_NO_GRID_CAP
-  const long long cap = tot;
-#else
   const long long cap = (long long)per_sm * (num_sms > 0 ? num_sms : 1);
-#endif
   const unsigned grid = (unsigned)(tot < cap ? tot : cap);
   ffn_decode_fused_kernel<WT, NT, RG, RD><<<grid, kThreads, 0, s>>>(p, list);
   return cudaGetLastError();
