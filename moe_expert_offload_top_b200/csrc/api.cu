@@ -728,6 +728,12 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
     cudaStreamSynchronize(s);
     return fail(h, code, msg);
   };
+  // CUDA failures from here on also drain the caller's stream (through bail)
+#define FT_CUDA_B(call)                                                                      \
+  do {                                                                                       \
+    cudaError_t _e = (call);                                                                 \
+    if (_e != cudaSuccess) return bail(FT_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(_e)); \
+  } while (0)
   int* dev_err = fused_route ? h->h_box + 1 : h->h_err;
   if (*dev_err) {
     const int code = *dev_err;
@@ -794,7 +800,7 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   const bool must_wait = need_fill > h->compute_waited_fill || (need_fill >= 0 && !same_stream);
   auto wait_fills = [&]() -> int {
     const int r = (int)(need_fill % kRing);
-    FT_CUDA(h, cudaStreamWaitEvent(s, h->fill_ev[r], 0));
+    FT_CUDA_B(cudaStreamWaitEvent(s, h->fill_ev[r], 0));
     h->compute_waited_fill = h->fill_ev_batch[r];
     return FT_OK;
   };
@@ -816,7 +822,7 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
   // directly (programmatic dependent launch).
   auto record_use = [&]() -> int {
     const int r = (int)(call % kRing);
-    FT_CUDA(h, cudaEventRecord(h->use_ev[r], s));
+    FT_CUDA_B(cudaEventRecord(h->use_ev[r], s));
     h->use_ev_call[r] = call;
     return FT_OK;
   };
@@ -854,13 +860,13 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
     if (split) {
       fp.combine = 0;
       stage_mark(se, SE_F0, s);
-      FT_CUDA(h, ftk::launch_ffn_fused(fp, h->wdtype, ready, max_pairs, h->num_sms, s));
+      FT_CUDA_B(ftk::launch_ffn_fused(fp, h->wdtype, ready, max_pairs, h->num_sms, s));
       stage_mark(se, SE_F1, s);
       rc = wait_fills();
       if (rc) return bail(rc, h->err);
       fp.combine = 1;
       stage_mark(se, SE_F2, s);
-      FT_CUDA(h, ftk::launch_ffn_fused(fp, h->wdtype, later, max_pairs, h->num_sms, s));
+      FT_CUDA_B(ftk::launch_ffn_fused(fp, h->wdtype, later, max_pairs, h->num_sms, s));
       stage_mark(se, SE_F3, s);
       if (se) se->fused_launches = 2;
       h->perf.kernel_launches += 2;
@@ -871,14 +877,14 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
       }
       fp.combine = 1;
       stage_mark(se, SE_F0, s);
-      FT_CUDA(h, ftk::launch_ffn_fused(fp, h->wdtype, list, max_pairs, h->num_sms, s));
+      FT_CUDA_B(ftk::launch_ffn_fused(fp, h->wdtype, list, max_pairs, h->num_sms, s));
       stage_mark(se, SE_F1, s);
       if (se) se->fused_launches = 1;
       h->perf.kernel_launches += 1;
     }
     stage_mark(se, SE_C1, s);
     rc = record_use();
-    if (rc) return rc;
+    if (rc) return bail(rc, h->err);
   } else {
     if (use_gemm) {
       if (must_wait) {
@@ -891,7 +897,7 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
         if (rc) return bail(rc, h->err);
       }
       rc = ensure_maps(h);
-      if (rc) return rc;
+      if (rc) return bail(rc, h->err);
       ftk::GemmGroups groups;
       groups.n = list.n;
       for (int i = 0; i < list.n; ++i) {
@@ -899,18 +905,18 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
         groups.z[i] = staged ? i : list.expert[i] >= 0 ? h->lru.slot_of(layer * E + list.expert[i]) : layer;
       }
       if (staged) {
-        FT_CUDA(h, ftk::launch_dequant_nvfp4_stage(list, h->H, h->I, h->stage, h->d_stage_gs, h->num_sms, s));
+        FT_CUDA_B(ftk::launch_dequant_nvfp4_stage(list, h->H, h->I, h->stage, h->d_stage_gs, h->num_sms, s));
         h->perf.kernel_launches += 1;
       }
       const ftk::GemmMaps& gm = staged ? h->smaps : h->maps;
       const float* gsc = staged ? h->d_stage_gs : nullptr;
-      FT_CUDA(h, ftk::launch_gather_rows(x, h->d_perm, T, k, h->H, h->has_shared != 0, h->d_ax, s));
+      FT_CUDA_B(ftk::launch_gather_rows(x, h->d_perm, T, k, h->H, h->has_shared != 0, h->d_ax, s));
       h->perf.kernel_launches += 1;
       stage_mark(se, SE_G0, s);
-      FT_CUDA(h, ftk::launch_grouped_gemm(0, gm, groups, h->d_offsets, T, k, h->I, h->H, h->d_h,
+      FT_CUDA_B(ftk::launch_grouped_gemm(0, gm, groups, h->d_offsets, T, k, h->I, h->H, h->d_h,
                                           h->d_err, h->num_sms, s, gsc));
       stage_mark(se, SE_G1, s);
-      FT_CUDA(h, ftk::launch_grouped_gemm(1, gm, groups, h->d_offsets, T, k, h->I, h->H, h->d_y,
+      FT_CUDA_B(ftk::launch_grouped_gemm(1, gm, groups, h->d_offsets, T, k, h->I, h->H, h->d_y,
                                           h->d_err, h->num_sms, s, gsc));
       if (se) {   // bf16 h, and the weights of each listed expert read once
         se->gu_bytes = list.n * 2.0 * h->H * h->I * 2 + pairs * (h->H * 2.0 + h->I * 2.0);
@@ -919,14 +925,14 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
     } else if (split) {
       // gate/up | G1 | down of the ready group, the wait, then gate/up | G3 | down of the rest
       stage_mark(se, SE_G0, s);
-      FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, ready, max_pairs, h->d_offsets,
+      FT_CUDA_B(ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, ready, max_pairs, h->d_offsets,
                                         h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr, h->d_err,
                                         h->int4_tensor != 0));
       stage_mark(se, SE_DA, s);
       rc = wait_fills();
       if (rc) return bail(rc, h->err);
       stage_mark(se, SE_G2, s);
-      FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, later, max_pairs, h->d_offsets,
+      FT_CUDA_B(ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, later, max_pairs, h->d_offsets,
                                         h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G3] : nullptr, h->d_err,
                                         h->int4_tensor != 0));
       if (se) se->split = 1;
@@ -937,19 +943,20 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
         if (rc) return bail(rc, h->err);
       }
       stage_mark(se, SE_G0, s);
-      FT_CUDA(h, ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, list, max_pairs, h->d_offsets,
+      FT_CUDA_B(ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, list, max_pairs, h->d_offsets,
                                         h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr, h->d_err,
                                         h->int4_tensor != 0));
     }
     stage_mark(se, SE_D1, s);
     rc = record_use();
-    if (rc) return rc;
-    FT_CUDA(h, ftk::launch_combine(h->d_y, h->d_gates, h->d_inv, T, h->H, k, h->has_shared != 0,
+    if (rc) return bail(rc, h->err);
+    FT_CUDA_B(ftk::launch_combine(h->d_y, h->d_gates, h->d_inv, T, h->H, k, h->has_shared != 0,
                                    xbf16, out, s));
     stage_mark(se, SE_C1, s);
     h->perf.kernel_launches += 3;
   }
   hold.release();
+#undef FT_CUDA_B
   for (int key : keys) h->slot_last_use[h->lru.slot_of(key)] = call;
   h->perf.host_issue_ms +=
       std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - t_routed).count();
