@@ -52,3 +52,25 @@ def test_single_process_aggregation_is_identity():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.aggregate(7, 2.5) == (7, 2.5)
+
+
+def test_reference_arm_json_line():
+    # the reference arm times the CPU oracle and prints the contract's JSON line (no GPU)
+    import json
+    import subprocess
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "3", "--reference-budget-s", "5"], cwd=ROOT, env=env,
+                         capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "dtype", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "tokens/s"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    # a rank other than 0 exits at once without a line
+    env1 = dict(os.environ, RANK="1", WORLD_SIZE="2")
+    out1 = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                           "--warmup", "3"], cwd=ROOT, env=env1, capture_output=True, text=True, timeout=120)
+    assert out1.returncode == 0 and out1.stdout.strip() == ""
