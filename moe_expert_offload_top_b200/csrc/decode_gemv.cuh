@@ -175,149 +175,174 @@ FT_DEVICE void gemv_rows(const void* __restrict__ xin, int T, int H, int I, int 
 #pragma unroll
         for (int t = 0; t < NT; ++t) acc[r][m][t] = 0.f;
 
-#pragma unroll kUnroll
-    for (int kk = lane * EL; kk < K; kk += 32 * EL) {
-      uint4 wc[RPW][NM];
-      float sc[RPW][NM];
-#pragma unroll
-      for (int r = 0; r < RPW; ++r)
-#pragma unroll
-        for (int m = 0; m < NM; ++m) {
-          const int rr = rok[r] ? rbase + r : rbase;
-          wc[r][m] = ldw(wmat[m] + (size_t)rr * row_bytes +
-                         ((WT == WT_INT4 || WT == WT_NVFP4) ? kk / 2 : kk * (WT == WT_F32 ? 4 : 2)));
-          if (WT == WT_INT4) sc[r][m] = bf16_to_f32(__ldg(smat[m] + (size_t)rr * (K / 128) + kk / 128));
-          if (WT == WT_NVFP4) {   // the chunk's two block scales, packed in sc as raw bits
-            const uint16_t two = __ldg(reinterpret_cast<const unsigned short*>(fmat[m] + (size_t)rr * (K / 16) + kk / 16));
-            sc[r][m] = __uint_as_float((uint32_t)two);
-          }
-        }
-      float part[RPW][NM][NT];
-#pragma unroll
-      for (int r = 0; r < RPW; ++r)
-#pragma unroll
-        for (int m = 0; m < NM; ++m)
-#pragma unroll
-          for (int t = 0; t < NT; ++t) part[r][m][t] = 0.f;
-      if constexpr (WT == WT_NVFP4) {
-        // e2m1 bytes -> f16x2 by the hardware conversion -> fp32; partial sums per
-        // 16-element block are scaled by that block's e4m3 scale.
-        float pb[RPW][NM][NT][2];
-#pragma unroll
+    // One K step of this warp's rows: the 16-byte chunks (and scales) at element kk ...
+    auto load_step = [&](int kk, uint4 (&wc)[RPW][NM], float (&sc)[RPW][NM]) {
+  #pragma unroll
         for (int r = 0; r < RPW; ++r)
-#pragma unroll
-          for (int m = 0; m < NM; ++m)
-#pragma unroll
-            for (int t = 0; t < NT; ++t) pb[r][m][t][0] = pb[r][m][t][1] = 0.f;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          float xv[NT][8];
-#pragma unroll
-          for (int t = 0; t < NT; ++t)
-            if (t < nt) ldin<8, BF16IN, COH>(in[t], kk + 8 * g, xv[t]);
-#pragma unroll
-          for (int r = 0; r < RPW; ++r)
-#pragma unroll
-            for (int m = 0; m < NM; ++m) {
-              const uint32_t w = g == 0 ? wc[r][m].x : g == 1 ? wc[r][m].y : g == 2 ? wc[r][m].z : wc[r][m].w;
-              float wv[8];
-#pragma unroll
-              for (int b = 0; b < 4; ++b) e2m1x2_to_f32((w >> (8 * b)) & 0xFFu, wv[2 * b], wv[2 * b + 1]);
-#pragma unroll
-              for (int t = 0; t < NT; ++t)
-                if (t < nt) {
-#pragma unroll
-                  for (int j = 0; j < 8; ++j) pb[r][m][t][g >> 1] = fmaf(wv[j], xv[t][j], pb[r][m][t][g >> 1]);
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < RPW; ++r)
-#pragma unroll
+  #pragma unroll
           for (int m = 0; m < NM; ++m) {
-            float s0, s1;
-            e4m3x2_to_f32(__float_as_uint(sc[r][m]), s0, s1);
-#pragma unroll
-            for (int t = 0; t < NT; ++t) part[r][m][t] = s0 * pb[r][m][t][0] + s1 * pb[r][m][t][1];
-          }
-      } else if constexpr (WT == WT_INT4) {
-        // Packed dequant.  Nibbles n and n+4 of a word sit in the two 16-bit halves of
-        // (w >> 4n) & 0x000F000F; xor with 0x4308 per half makes the bf16 128 + (q + 8)
-        // (0x4300 is 128.0 in bf16, its last mantissa bit 1.0; xor 8 maps a 4-bit
-        // two's-complement q to q + 8).  Widening to fp32 and one packed add of -136
-        // give the pair (q_n, q_{n+4}) exactly; packed fp32 FMAs meet the matching x
-        // pairs.  About 3 lane instructions per weight instead of 5.
-        float2 acc2[RPW][NM][NT];
-#pragma unroll
-        for (int r = 0; r < RPW; ++r)
-#pragma unroll
-          for (int m = 0; m < NM; ++m)
-#pragma unroll
-            for (int t = 0; t < NT; ++t) acc2[r][m][t] = make_float2(0.f, 0.f);
-        const float2 bias = make_float2(-136.f, -136.f);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          float2 xp[NT][4];
-#pragma unroll
-          for (int t = 0; t < NT; ++t)
-            if (t < nt) {
-              float xv[8];
-              ldin<8, BF16IN, COH>(in[t], kk + 8 * g, xv);
-#pragma unroll
-              for (int n = 0; n < 4; ++n) xp[t][n] = make_float2(xv[n], xv[n + 4]);
+            const int rr = rok[r] ? rbase + r : rbase;
+            wc[r][m] = ldw(wmat[m] + (size_t)rr * row_bytes +
+                           ((WT == WT_INT4 || WT == WT_NVFP4) ? kk / 2 : kk * (WT == WT_F32 ? 4 : 2)));
+            if (WT == WT_INT4) sc[r][m] = bf16_to_f32(__ldg(smat[m] + (size_t)rr * (K / 128) + kk / 128));
+            if (WT == WT_NVFP4) {   // the chunk's two block scales, packed in sc as raw bits
+              const uint16_t two = __ldg(reinterpret_cast<const unsigned short*>(fmat[m] + (size_t)rr * (K / 16) + kk / 16));
+              sc[r][m] = __uint_as_float((uint32_t)two);
             }
-#pragma unroll
+          }
+    };
+    // ... and their products with the token vectors, added to acc in K order.
+    auto compute_step = [&](int kk, const uint4 (&wc)[RPW][NM], const float (&sc)[RPW][NM]) {
+        float part[RPW][NM][NT];
+  #pragma unroll
+        for (int r = 0; r < RPW; ++r)
+  #pragma unroll
+          for (int m = 0; m < NM; ++m)
+  #pragma unroll
+            for (int t = 0; t < NT; ++t) part[r][m][t] = 0.f;
+        if constexpr (WT == WT_NVFP4) {
+          // e2m1 bytes -> f16x2 by the hardware conversion -> fp32; partial sums per
+          // 16-element block are scaled by that block's e4m3 scale.
+          float pb[RPW][NM][NT][2];
+  #pragma unroll
           for (int r = 0; r < RPW; ++r)
-#pragma unroll
-            for (int m = 0; m < NM; ++m) {
-              const uint32_t w = g == 0 ? wc[r][m].x : g == 1 ? wc[r][m].y : g == 2 ? wc[r][m].z : wc[r][m].w;
-#pragma unroll
-              for (int n = 0; n < 4; ++n) {
-                const uint32_t v = ((w >> (4 * n)) & 0x000F000Fu) ^ 0x43084308u;
-                const float2 q2 = __fadd2_rn(make_float2(bf16lo(v), bf16hi(v)), bias);
-#pragma unroll
-                for (int t = 0; t < NT; ++t)
-                  if (t < nt) acc2[r][m][t] = __ffma2_rn(q2, xp[t][n], acc2[r][m][t]);
-              }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < RPW; ++r)
-#pragma unroll
-          for (int m = 0; m < NM; ++m)
-#pragma unroll
-            for (int t = 0; t < NT; ++t) part[r][m][t] = acc2[r][m][t].x + acc2[r][m][t].y;
-      } else {
-#pragma unroll
-      for (int g = 0; g < NG; ++g) {
-        float wv[RPW][NM][GE];
-#pragma unroll
-        for (int r = 0; r < RPW; ++r)
-#pragma unroll
-          for (int m = 0; m < NM; ++m) wgroup<WT>(wc[r][m], g, wv[r][m]);
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          if (t < nt) {
-            float xv[GE];
-            ldin<GE, BF16IN, COH>(in[t], kk + g * GE, xv);
-#pragma unroll
+  #pragma unroll
+            for (int m = 0; m < NM; ++m)
+  #pragma unroll
+              for (int t = 0; t < NT; ++t) pb[r][m][t][0] = pb[r][m][t][1] = 0.f;
+  #pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            float xv[NT][8];
+  #pragma unroll
+            for (int t = 0; t < NT; ++t)
+              if (t < nt) ldin<8, BF16IN, COH>(in[t], kk + 8 * g, xv[t]);
+  #pragma unroll
             for (int r = 0; r < RPW; ++r)
-#pragma unroll
-              for (int m = 0; m < NM; ++m)
-#pragma unroll
-                for (int j = 0; j < GE; ++j) part[r][m][t] = fmaf(wv[r][m][j], xv[j], part[r][m][t]);
+  #pragma unroll
+              for (int m = 0; m < NM; ++m) {
+                const uint32_t w = g == 0 ? wc[r][m].x : g == 1 ? wc[r][m].y : g == 2 ? wc[r][m].z : wc[r][m].w;
+                float wv[8];
+  #pragma unroll
+                for (int b = 0; b < 4; ++b) e2m1x2_to_f32((w >> (8 * b)) & 0xFFu, wv[2 * b], wv[2 * b + 1]);
+  #pragma unroll
+                for (int t = 0; t < NT; ++t)
+                  if (t < nt) {
+  #pragma unroll
+                    for (int j = 0; j < 8; ++j) pb[r][m][t][g >> 1] = fmaf(wv[j], xv[t][j], pb[r][m][t][g >> 1]);
+                  }
+              }
+          }
+  #pragma unroll
+          for (int r = 0; r < RPW; ++r)
+  #pragma unroll
+            for (int m = 0; m < NM; ++m) {
+              float s0, s1;
+              e4m3x2_to_f32(__float_as_uint(sc[r][m]), s0, s1);
+  #pragma unroll
+              for (int t = 0; t < NT; ++t) part[r][m][t] = s0 * pb[r][m][t][0] + s1 * pb[r][m][t][1];
+            }
+        } else if constexpr (WT == WT_INT4) {
+          // Packed dequant.  Nibbles n and n+4 of a word sit in the two 16-bit halves of
+          // (w >> 4n) & 0x000F000F; xor with 0x4308 per half makes the bf16 128 + (q + 8)
+          // (0x4300 is 128.0 in bf16, its last mantissa bit 1.0; xor 8 maps a 4-bit
+          // two's-complement q to q + 8).  Widening to fp32 and one packed add of -136
+          // give the pair (q_n, q_{n+4}) exactly; packed fp32 FMAs meet the matching x
+          // pairs.  About 3 lane instructions per weight instead of 5.
+          float2 acc2[RPW][NM][NT];
+  #pragma unroll
+          for (int r = 0; r < RPW; ++r)
+  #pragma unroll
+            for (int m = 0; m < NM; ++m)
+  #pragma unroll
+              for (int t = 0; t < NT; ++t) acc2[r][m][t] = make_float2(0.f, 0.f);
+          const float2 bias = make_float2(-136.f, -136.f);
+  #pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            float2 xp[NT][4];
+  #pragma unroll
+            for (int t = 0; t < NT; ++t)
+              if (t < nt) {
+                float xv[8];
+                ldin<8, BF16IN, COH>(in[t], kk + 8 * g, xv);
+  #pragma unroll
+                for (int n = 0; n < 4; ++n) xp[t][n] = make_float2(xv[n], xv[n + 4]);
+              }
+  #pragma unroll
+            for (int r = 0; r < RPW; ++r)
+  #pragma unroll
+              for (int m = 0; m < NM; ++m) {
+                const uint32_t w = g == 0 ? wc[r][m].x : g == 1 ? wc[r][m].y : g == 2 ? wc[r][m].z : wc[r][m].w;
+  #pragma unroll
+                for (int n = 0; n < 4; ++n) {
+                  const uint32_t v = ((w >> (4 * n)) & 0x000F000Fu) ^ 0x43084308u;
+                  const float2 q2 = __fadd2_rn(make_float2(bf16lo(v), bf16hi(v)), bias);
+  #pragma unroll
+                  for (int t = 0; t < NT; ++t)
+                    if (t < nt) acc2[r][m][t] = __ffma2_rn(q2, xp[t][n], acc2[r][m][t]);
+                }
+              }
+          }
+  #pragma unroll
+          for (int r = 0; r < RPW; ++r)
+  #pragma unroll
+            for (int m = 0; m < NM; ++m)
+  #pragma unroll
+              for (int t = 0; t < NT; ++t) part[r][m][t] = acc2[r][m][t].x + acc2[r][m][t].y;
+        } else {
+  #pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          float wv[RPW][NM][GE];
+  #pragma unroll
+          for (int r = 0; r < RPW; ++r)
+  #pragma unroll
+            for (int m = 0; m < NM; ++m) wgroup<WT>(wc[r][m], g, wv[r][m]);
+  #pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            if (t < nt) {
+              float xv[GE];
+              ldin<GE, BF16IN, COH>(in[t], kk + g * GE, xv);
+  #pragma unroll
+              for (int r = 0; r < RPW; ++r)
+  #pragma unroll
+                for (int m = 0; m < NM; ++m)
+  #pragma unroll
+                  for (int j = 0; j < GE; ++j) part[r][m][t] = fmaf(wv[r][m][j], xv[j], part[r][m][t]);
+            }
           }
         }
+        }
+  #pragma unroll
+        for (int r = 0; r < RPW; ++r)
+  #pragma unroll
+          for (int m = 0; m < NM; ++m)
+  #pragma unroll
+            for (int t = 0; t < NT; ++t)
+              acc[r][m][t] = WT == WT_INT4 ? fmaf(sc[r][m], part[r][m][t], acc[r][m][t])
+                                           : acc[r][m][t] + part[r][m][t];
+    };
+    if constexpr (RPW == 1 && (WT == WT_BF16 || WT == WT_F32)) {
+      // One row (pair) per warp, the short-list and long-row case: bound by DRAM latency,
+      // so up to 8 K steps of loads are issued before the first is used (the summation
+      // order, and so every output, is the same as in the loop below).
+      constexpr int D = 8;
+      for (int kb = lane * EL; kb < K; kb += D * 32 * EL) {
+        uint4 wd[D][RPW][NM];
+        float sd[D][RPW][NM];
+#pragma unroll
+        for (int u = 0; u < D; ++u)
+          if (kb + u * 32 * EL < K) load_step(kb + u * 32 * EL, wd[u], sd[u]);
+#pragma unroll
+        for (int u = 0; u < D; ++u)
+          if (kb + u * 32 * EL < K) compute_step(kb + u * 32 * EL, wd[u], sd[u]);
       }
+    } else {
+#pragma unroll kUnroll
+      for (int kk = lane * EL; kk < K; kk += 32 * EL) {
+        uint4 wc[RPW][NM];
+        float sc[RPW][NM];
+        load_step(kk, wc, sc);
+        compute_step(kk, wc, sc);
       }
-#pragma unroll
-      for (int r = 0; r < RPW; ++r)
-#pragma unroll
-        for (int m = 0; m < NM; ++m)
-#pragma unroll
-          for (int t = 0; t < NT; ++t)
-            acc[r][m][t] = WT == WT_INT4 ? fmaf(sc[r][m], part[r][m][t], acc[r][m][t])
-                                         : acc[r][m][t] + part[r][m][t];
     }
 #pragma unroll
     for (int r = 0; r < RPW; ++r)
