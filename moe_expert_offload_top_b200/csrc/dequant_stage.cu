@@ -37,20 +37,26 @@ dequant_nvfp4_stage_kernel(const __grid_constant__ ExpertList list, int H, int I
     const size_t m = e0 / mat, off = e0 - m * mat;
     const uint4 q = __ldcs(reinterpret_cast<const uint4*>(blob + m * (mat / 2) + off / 2));
     const uint16_t sc2 = *reinterpret_cast<const uint16_t*>(blob + 3 * mat / 2 + m * (mat / 16) + off / 16);
-    float s0, s1;
-    e4m3x2_to_f32(sc2, s0, s1);                       // the two 16-element blocks of this chunk
+    // the two 16-element block scales as f16, each broadcast to both halves of a pair
+    uint32_t s2;
+    asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(s2) : "r"((uint32_t)sc2));
+    const uint32_t s_lo = __byte_perm(s2, 0, 0x1010), s_hi = __byte_perm(s2, 0, 0x3232);
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
     uint32_t out[16];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float s = i < 2 ? s0 : s1;
+      const uint32_t sp = i < 2 ? s_lo : s_hi;
 #pragma unroll
-      for (int b = 0; b < 4; b += 2) {
-        float v0, v1, v2, v3;
-        e2m1x2_to_f32((w[i] >> (8 * b)) & 0xFFu, v0, v1);
-        e2m1x2_to_f32((w[i] >> (8 * b + 8)) & 0xFFu, v2, v3);
-        out[4 * i + b] = (uint32_t)f32_to_bf16(v0 * s) | ((uint32_t)f32_to_bf16(v1 * s) << 16);
-        out[4 * i + b + 1] = (uint32_t)f32_to_bf16(v2 * s) | ((uint32_t)f32_to_bf16(v3 * s) << 16);
+      for (int b = 0; b < 4; ++b) {
+        // two e2m1 codes -> f16 pair (exact), times the f16 scale pair (exact: at most 6
+        // significant bits, within f16 range), -> two fp32 -> one bf16 pair (exact)
+        uint32_t h2, p2, o;
+        asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h2) : "r"((w[i] >> (8 * b)) & 0xFFu));
+        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p2) : "r"(h2), "r"(sp));
+        const float lo = __half2float(__ushort_as_half((unsigned short)(p2 & 0xFFFFu)));
+        const float hi = __half2float(__ushort_as_half((unsigned short)(p2 >> 16)));
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o) : "f"(hi), "f"(lo));
+        out[4 * i + b] = o;
       }
     }
     uint4* dst = reinterpret_cast<uint4*>(stage + (size_t)entry * blob_elems + e0);
