@@ -57,7 +57,8 @@ enum ft_status {
   FT_ERR_CAPACITY = 4,     /* one step needs more distinct experts than there are slots */
   FT_ERR_BUSY = 5,         /* resize or destroy requested while a forward is in flight */
   FT_ERR_TIMEOUT = 6,      /* a host wait on the GPU passed its deadline */
-  FT_ERR_DEVICE_CHECK = 7  /* a kernel's own bounds check failed (the kernel skipped the access) */
+  FT_ERR_DEVICE_CHECK = 7  /* a kernel's bounded wait gave up, or its own check failed (the message
+                              gives the code from the device error word) */
 };
 
 enum ft_wdtype { FT_W_F32 = 0, FT_W_BF16 = 1, FT_W_INT4_G128 = 2, FT_W_NVFP4 = 3 };
@@ -138,8 +139,9 @@ FT_API size_t ft_moe_blob_bytes(const ft_moe* h);
  *               e4m3 block scales S_gate [I][H/16], S_up [I][H/16], S_down [H][I/16] (one
  *               byte per 16 consecutive K elements), then the fp32 global scales g_gate,
  *               g_up, g_down and 4 zero bytes.  w = e2m1(q) * e4m3(s) * g.  H and I must
- *               be multiples of 32.  Decode only: nvfp4 stacks use the streaming GEMV for
- *               every batch size. */
+ *               be multiples of 32.  Decode runs the streaming GEMV on these codes;
+ *               prefill (the GEMM path) expands the selected experts exactly to bf16
+ *               (e2m1 * e4m3) and applies g to the GEMM accumulators. */
 FT_API void* ft_moe_pool_ptr(ft_moe* h, int layer, int expert);
 
 /* Copies the shared expert of `layer` (a host blob in the same layout) into resident
@@ -162,14 +164,16 @@ FT_API int ft_moe_reserve(ft_moe* h, int max_tokens);
  *   out      device [n_tokens][H], same type as x.
  *   stream   caller's stream; every kernel and the wait for slot fills run on it.
  * Steps: router logits (fp32) and top-k with normalised gates; one host read of
- * the selected expert ids (the host waits for it, with a deadline); the LRU
- * lookup and update over the distinct selected experts (hits in ascending expert
- * order first, then misses in ascending order, each taking the lowest free slot or
- * evicting the least recently used entry); copies of missed experts from the
+ * the selected expert ids (for up to 64 tokens the routing kernel writes them to mapped
+ * pinned memory, otherwise a device-to-host copy; the host waits, with a deadline);
+ * the LRU lookup and update over the distinct selected experts (hits in ascending
+ * expert order first, then misses in ascending order, each taking the lowest free slot
+ * or evicting the least recently used entry); copies of missed experts from the
  * pinned pool into their slots on the library's copy stream, each after the
  * kernels that last read the slot; token permutation by expert; the SwiGLU FFN of
- * every selected expert reading its weights from its slot; the gate-weighted sum of
- * the k outputs in ascending k order, plus the shared expert.
+ * every selected expert reading its weights from its slot (on the GEMV path the
+ * experts already resident run before the wait for this call's copies); the
+ * gate-weighted sum of the k outputs in ascending k order, plus the shared expert.
  * Returns FT_ERR_CAPACITY, before any state changes, if the distinct experts of
  * the call exceed the cache slots.  All forwards of a handle are ordered: a
  * forward on another stream first waits for the previous forward's kernels.  A forward
@@ -180,13 +184,14 @@ FT_API int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, con
                    void* out, void* stream);
 
 /* Waits for every forward and copy of the handle, then checks the device error word
- * that the prefill GEMM kernels set when one of their bounded waits gives up
- * (FT_ERR_DEVICE_CHECK; the word is cleared).  A forward also reports a word set by
- * an earlier forward. */
+ * that a kernel sets when one of its bounded waits gives up (FT_ERR_DEVICE_CHECK; the
+ * word is cleared): codes 101-104 the prefill GEMM's pipeline waits, 111 the fused
+ * decode FFN's wait for an expert's gate/up rows.  A forward also reports a word set
+ * by an earlier forward. */
 FT_API int ft_moe_sync(ft_moe* h);
 
-/* Expert FFN path: bf16 stacks with H % 256 == 0 and I % 128 == 0 use the tcgen05
- * grouped GEMMs when n_tokens * k >= min_avg_pairs * |S| (on average at least
+/* Expert FFN path: bf16 and nvfp4 stacks with H % 256 == 0 and I % 128 == 0 use the
+ * tcgen05 grouped GEMMs when n_tokens * k >= min_avg_pairs * |S| (on average at least
  * min_avg_pairs tokens per selected expert; default 32), else the streaming GEMV.
  * Both compute the same function.  0 always selects the GEMMs where shapes allow. */
 FT_API int ft_moe_set_gemm_threshold(ft_moe* h, int min_avg_pairs);
