@@ -169,3 +169,19 @@ def test_bandwidth_profile_host_part(tmp_path):
     assert "h2d_gbs" not in prof
     with pytest.raises(ft.FtError):
         ft.ft_probe_host_memory(16, 1, 1)          # below the minimum size
+
+
+def test_calls_fail_cleanly_without_a_device():
+    # with no GPU the library refuses with a message instead of crashing; invalid
+    # arguments are refused first in any case
+    import torch
+    with pytest.raises(ft.FtError) as ei:
+        ft.ft_moe_create(16, 20, 256, 128, "f32", 4)          # top_k > num_experts
+    assert "invalid argument" in str(ei.value)
+    with pytest.raises(ft.FtError):
+        ft.ft_moe_create(16, 2, 100, 128, "int4", 4)          # int4 needs multiples of 128
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    with pytest.raises(ft.FtError) as ei:
+        ft.ft_moe_create(16, 2, 256, 128, "f32", 4)
+    assert "allocation" in str(ei.value) or "CUDA" in str(ei.value)
