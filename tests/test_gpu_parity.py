@@ -369,3 +369,26 @@ def test_forwards_on_alternating_streams():
         for s in range(cfg.tokens):
             for l in range(cfg.L):
                 assert_close(got[s][l], ref["out"][(s, l)], "bf16", "step %d layer %d" % (s, l))
+
+
+def test_empty_forward_changes_nothing():
+    cfg = dataclasses.replace(synth.CONFIGS[2], L=1, tokens=4, C=16)
+    with GpuStack(cfg) as st:
+        vals, x = st.tokens(1)
+        out = torch.zeros((1, cfg.H), dtype=torch.bfloat16, device=DEV)
+        st.forward(0, x[0][:0], out[:0])                       # zero tokens: a no-op
+        torch.cuda.synchronize()
+        assert st.trace() == [] and st.stats()["routed"] == 0
+        assert float(out.abs().sum()) == 0.0
+
+
+def test_every_expert_selected():
+    # k = E: every expert of the layer is selected for every token (top-k is a sort)
+    cfg = synth.MoeConfig("k-eq-e", L=2, E=8, H=256, I=128, k=8, gating="softmax", wdtype="bf16",
+                          shared=False, C=16, tokens=6, batches=(1,), process="ar1", mode="decode")
+    with GpuStack(cfg) as st:
+        vals, x = st.tokens(1)
+        outs, ids = _run_gpu(st, x, cfg.tokens)
+        ref = oracle_run(cfg, st, vals)
+        _check_run(cfg, st, vals, outs, ids, ref, cfg.tokens)
+        assert st.stats()["misses"] == 16                      # only the first step's compulsory misses
