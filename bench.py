@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
-CONFIG_ID = 2
+WORKLOAD = "decode-locality-bf16"
 METRIC = "routed-MoE tokens/s (decode, prefill) and expert-weight HBM GB/s vs peak"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -229,7 +229,7 @@ def run_reference(args):
     rank, world, local = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
     if rank != 0:
         return 0
-    cfg = synth.CONFIGS[CONFIG_ID]
+    cfg = synth.CONFIGS[WORKLOAD]
     vals, _ = token_chain(cfg, 0, args.warmup + args.steps)
     # warm-up steps untimed, then the timed steps, bounded to a few minutes in all
     cpu_oracle_rate(cfg, vals[:args.warmup], budget_s=30.0, max_tokens=args.warmup)
@@ -262,7 +262,7 @@ def run_prefill_leg(args, dev):
     import moe_expert_offload_top_b200 as ft
     from moe_expert_offload_top_b200.workload import GpuStack
 
-    base = synth.CONFIGS[4]
+    base = synth.CONFIGS["dsv4flash-prefill-bf16"]
     T = args.prefill_tokens or base.tokens
     cfg = dataclasses.replace(base, tokens=T, batches=(T,))
     stack = GpuStack(cfg, device=dev, max_tokens=T)
@@ -333,7 +333,7 @@ def run_ours(args):
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    cfg = synth.CONFIGS[CONFIG_ID]
+    cfg = synth.CONFIGS[WORKLOAD]
     W, K = args.warmup, args.steps
     vals, bits = token_chain(cfg, rank, W + 3 * K)      # device leg, stage leg, e2e leg
     stack = GpuStack(cfg, device=dev)

@@ -60,19 +60,20 @@ def _slots(frac: float, L: int, E: int) -> int:
 AR_PHI = 0.9
 AR_SIG = 0.436
 
+# The stated workloads, by name.
 CONFIGS = {
-    1: MoeConfig("tiny-fp32", L=1, E=16, H=256, I=128, k=2, gating="softmax", wdtype="f32",
+    "tiny-fp32": MoeConfig("tiny-fp32", L=1, E=16, H=256, I=128, k=2, gating="softmax", wdtype="f32",
                  shared=False, C=4, tokens=8, batches=(1,), process="iid", mode="decode"),
-    2: MoeConfig("decode-locality-bf16", L=4, E=128, H=2048, I=768, k=8, gating="softmax",
+    "decode-locality-bf16": MoeConfig("decode-locality-bf16", L=4, E=128, H=2048, I=768, k=8, gating="softmax",
                  wdtype="bf16", shared=False, C=_slots(0.40, 4, 128), tokens=512, batches=(1,),
                  process="ar1", mode="decode"),
-    3: MoeConfig("dsv4flash-decode-bf16", L=8, E=256, H=4096, I=2048, k=6, gating="sigmoid",
+    "dsv4flash-decode-bf16": MoeConfig("dsv4flash-decode-bf16", L=8, E=256, H=4096, I=2048, k=6, gating="sigmoid",
                  wdtype="bf16", shared=True, C=_slots(0.25, 8, 256), tokens=1024, batches=(1,),
                  process="ar1", mode="decode"),
-    4: MoeConfig("dsv4flash-prefill-bf16", L=8, E=256, H=4096, I=2048, k=6, gating="sigmoid",
+    "dsv4flash-prefill-bf16": MoeConfig("dsv4flash-prefill-bf16", L=8, E=256, H=4096, I=2048, k=6, gating="sigmoid",
                  wdtype="bf16", shared=True, C=_slots(0.25, 8, 256), tokens=4096, batches=(4096,),
                  process="iid", mode="prefill"),
-    5: MoeConfig("int4-large-pool", L=16, E=256, H=7168, I=2048, k=8, gating="sigmoid",
+    "int4-large-pool": MoeConfig("int4-large-pool", L=16, E=256, H=7168, I=2048, k=8, gating="sigmoid",
                  wdtype="int4", shared=False, C=_slots(0.15, 16, 256), tokens=2048, batches=(1, 8, 32),
                  process="ar1", mode="decode", resize_to=_slots(0.30, 16, 256)),
 }

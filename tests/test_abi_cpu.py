@@ -142,7 +142,7 @@ def test_lru_beats_static_split_on_locality_traces():
     # static split of the same capacity.  A trend, not a pin.
     import synth
     from oracle import moe
-    cfg = synth.CONFIGS[2]
+    cfg = synth.CONFIGS["decode-locality-bf16"]
     vals, _ = synth.tokens(cfg, 1)
     routers = [synth.router_weights(cfg, l) for l in range(cfg.L)]
     ops = []

@@ -130,14 +130,14 @@ def test_gemm_path_uneven_groups_and_many_tiles():
 
 @pytest.mark.slow
 def test_config3_dsv4flash_decode_full_size():
-    cfg = synth.CONFIGS[3]
+    cfg = synth.CONFIGS["dsv4flash-decode-bf16"]
     st = run_and_check(cfg, 1, sample_steps=[5, 511, 1023])
     assert 0 < st["misses"] < st["routed"]
 
 
 @pytest.mark.slow
 def test_config4_prefill_double_buffer_full_size():
-    cfg = synth.CONFIGS[4]
+    cfg = synth.CONFIGS["dsv4flash-prefill-bf16"]
     rng = np.random.default_rng(4)
     toks = sorted(rng.choice(4096, 3, replace=False).tolist())
     st = run_and_check(cfg, 4096, sample_steps=[0], sample_tokens=toks)
@@ -147,7 +147,7 @@ def test_config4_prefill_double_buffer_full_size():
 @pytest.fixture(scope="module")
 def config5_stack():
     # the 93 GB int4 pool is generated and pinned once for the three batch sizes
-    st = GpuStack(synth.CONFIGS[5])
+    st = GpuStack(synth.CONFIGS["int4-large-pool"])
     yield st
     st.close()
 
@@ -155,7 +155,7 @@ def config5_stack():
 @pytest.mark.slow
 @pytest.mark.parametrize("batch", [1, 8, 32])
 def test_config5_int4_large_pool_with_resize(batch, config5_stack):
-    cfg = synth.CONFIGS[5]
+    cfg = synth.CONFIGS["int4-large-pool"]
     steps = cfg.tokens // batch
     toks = [0] if batch == 1 else [0, batch - 1]
     st = run_and_check(cfg, batch, sample_steps=[1, steps - 1], sample_tokens=toks,

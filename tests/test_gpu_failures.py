@@ -17,7 +17,7 @@ DEV = "cuda"
 
 
 def _cfg():
-    return dataclasses.replace(synth.CONFIGS[2], L=2, tokens=12, C=24)
+    return dataclasses.replace(synth.CONFIGS["decode-locality-bf16"], L=2, tokens=12, C=24)
 
 
 def test_failed_fill_rolls_back_and_next_forward_recovers():
@@ -71,7 +71,7 @@ def test_device_wait_gives_up_and_context_survives():
     assert rc == ft.FT_ERR_DEVICE_CHECK
     a = torch.ones(1024, device=DEV)
     assert float((a * 2).sum()) == 2048.0             # the context still runs work
-    cfg = synth.CONFIGS[1]
+    cfg = synth.CONFIGS["tiny-fp32"]
     with GpuStack(cfg) as st:
         vals, x = st.tokens(1)
         out = torch.empty((1, 1, cfg.H), dtype=torch.float32, device=DEV)
@@ -80,7 +80,7 @@ def test_device_wait_gives_up_and_context_survives():
 
 
 def test_step_larger_than_cache_is_rejected_first():
-    cfg = dataclasses.replace(synth.CONFIGS[2], L=1, tokens=4, C=5)   # k = 8 > 5 slots
+    cfg = dataclasses.replace(synth.CONFIGS["decode-locality-bf16"], L=1, tokens=4, C=5)   # k = 8 > 5 slots
     with GpuStack(cfg) as st:
         vals, x = st.tokens(1)
         out = torch.empty((1, cfg.H), dtype=torch.bfloat16, device=DEV)

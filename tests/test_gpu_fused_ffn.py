@@ -45,12 +45,12 @@ def _run(cfg, fused, batch=1, steps=None, gemm_threshold=None, stage_timing=Fals
 
 CASES = {
     # name: (config, batch)
-    "bf16-misses": (dataclasses.replace(synth.CONFIGS[2], L=2, tokens=24, C=40), 1),
-    "bf16-batch8": (dataclasses.replace(synth.CONFIGS[2], L=2, tokens=48, C=160), 8),
+    "bf16-misses": (dataclasses.replace(synth.CONFIGS["decode-locality-bf16"], L=2, tokens=24, C=40), 1),
+    "bf16-batch8": (dataclasses.replace(synth.CONFIGS["decode-locality-bf16"], L=2, tokens=48, C=160), 8),
     "bf16-shared": (synth.MoeConfig("shared-small", L=2, E=32, H=1024, I=512, k=6, gating="sigmoid",
                                     wdtype="bf16", shared=True, C=20, tokens=12, batches=(1,),
                                     process="ar1", mode="decode"), 1),
-    "f32-tiny": (synth.CONFIGS[1], 1),
+    "f32-tiny": (synth.CONFIGS["tiny-fp32"], 1),
     "int4": (synth.MoeConfig("int4-small", L=2, E=32, H=1024, I=512, k=8, gating="sigmoid", wdtype="int4",
                              shared=False, C=24, tokens=12, batches=(1,), process="ar1", mode="decode"), 1),
     "nvfp4": (synth.MoeConfig("nvfp4-small", L=2, E=32, H=1024, I=512, k=4, gating="softmax", wdtype="nvfp4",
@@ -98,7 +98,7 @@ def test_many_tokens_gemv_path_fused():
 def test_resident_experts_run_before_the_fill_wait():
     # fused launch shape: forwards with both resident and copied experts run two fused
     # launches (the resident experts, then the copied ones with the combine)
-    cfg = dataclasses.replace(synth.CONFIGS[2], L=2, tokens=24, C=40)
+    cfg = dataclasses.replace(synth.CONFIGS["decode-locality-bf16"], L=2, tokens=24, C=40)
     fwd = cfg.L * cfg.tokens
     a = _run(cfg, fused=True)
     p = a["perf"]
@@ -117,7 +117,7 @@ def test_resident_experts_run_before_the_fill_wait():
 def test_per_pass_kernels_split_around_the_fill_wait():
     # the default launch shape: forwards with both resident and copied experts run two
     # gate/up + down pairs (five FFN launches with the combine), the others one pair
-    cfg = dataclasses.replace(synth.CONFIGS[2], L=2, tokens=24, C=40)
+    cfg = dataclasses.replace(synth.CONFIGS["decode-locality-bf16"], L=2, tokens=24, C=40)
     fwd = cfg.L * cfg.tokens
     a = _run(cfg, fused=False)
     p = a["perf"]

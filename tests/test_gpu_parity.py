@@ -234,7 +234,7 @@ def _check_run(cfg, stack, vals, outs, ids, ref, steps):
 
 
 def test_config1_tiny_forward_parity():
-    cfg = synth.CONFIGS[1]
+    cfg = synth.CONFIGS["tiny-fp32"]
     with GpuStack(cfg) as st:
         vals, x = st.tokens(1)
         outs, ids = _run_gpu(st, x, cfg.tokens)
@@ -246,7 +246,7 @@ def test_config1_tiny_forward_parity():
 
 
 def test_config2_decode_locality_full_size_parity():
-    cfg = synth.CONFIGS[2]
+    cfg = synth.CONFIGS["decode-locality-bf16"]
     with GpuStack(cfg) as st:
         vals, x = st.tokens(1)
         steps = cfg.tokens
@@ -262,7 +262,7 @@ def test_config2_decode_locality_full_size_parity():
 def test_capacity_changes_speed_not_result():
     # FreeToken RTX 5090, dynamic reconfiguration: the output does not depend on the
     # cache size; with every expert resident (`fused`) it is the same again.
-    base = synth.CONFIGS[2]
+    base = synth.CONFIGS["decode-locality-bf16"]
     cfg = dataclasses.replace(base, tokens=24)
     results = []
     for C in (cfg.k, cfg.L * cfg.E // 3, cfg.L * cfg.E):
@@ -280,7 +280,7 @@ def test_capacity_changes_speed_not_result():
 
 def test_evict_every_step_war_hazard():
     # capacity = k: nearly every step overwrites slots read by the previous step's kernels
-    cfg = dataclasses.replace(synth.CONFIGS[2], L=2, tokens=40, C=8)
+    cfg = dataclasses.replace(synth.CONFIGS["decode-locality-bf16"], L=2, tokens=40, C=8)
     with GpuStack(cfg) as st:
         vals, x = st.tokens(1)
         outs, ids = _run_gpu(st, x, cfg.tokens)
@@ -290,7 +290,7 @@ def test_evict_every_step_war_hazard():
 
 
 def test_capacity_error_changes_nothing():
-    cfg = dataclasses.replace(synth.CONFIGS[1], C=1)
+    cfg = dataclasses.replace(synth.CONFIGS["tiny-fp32"], C=1)
     with GpuStack(cfg) as st:
         vals, x = st.tokens(1)
         out = torch.empty((1, cfg.H), dtype=torch.float32, device=DEV)
@@ -301,7 +301,7 @@ def test_capacity_error_changes_nothing():
 
 
 def test_resize_grow_and_shrink_mid_run():
-    cfg = dataclasses.replace(synth.CONFIGS[2], tokens=60)
+    cfg = dataclasses.replace(synth.CONFIGS["decode-locality-bf16"], tokens=60)
     with GpuStack(cfg, capacity=40) as st:
         vals, x = st.tokens(1)
         out = torch.empty((cfg.L, 1, cfg.H), dtype=torch.bfloat16, device=DEV)
@@ -354,7 +354,7 @@ def test_nvfp4_stack_decode_forward_parity():
 
 
 def test_forwards_on_alternating_streams():
-    cfg = dataclasses.replace(synth.CONFIGS[2], L=2, tokens=16, C=20)
+    cfg = dataclasses.replace(synth.CONFIGS["decode-locality-bf16"], L=2, tokens=16, C=20)
     s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
     with GpuStack(cfg) as st:
         vals, x = st.tokens(1)
@@ -372,7 +372,7 @@ def test_forwards_on_alternating_streams():
 
 
 def test_empty_forward_changes_nothing():
-    cfg = dataclasses.replace(synth.CONFIGS[2], L=1, tokens=4, C=16)
+    cfg = dataclasses.replace(synth.CONFIGS["decode-locality-bf16"], L=1, tokens=4, C=16)
     with GpuStack(cfg) as st:
         vals, x = st.tokens(1)
         out = torch.zeros((1, cfg.H), dtype=torch.bfloat16, device=DEV)

@@ -337,7 +337,7 @@ def test_capacity_independence_and_fused_equivalence():
 
 
 def test_config1_oracle_runs_and_gates_sum_to_one():
-    cfg = synth.CONFIGS[1]
+    cfg = synth.CONFIGS["tiny-fp32"]
     r = _tiny_run(cfg, cfg.C, True, steps=8)
     assert r["ids"].shape == (8, 1, 1, 2)
     assert np.allclose(r["gates"].sum(axis=-1), 1.0, atol=1e-12)
