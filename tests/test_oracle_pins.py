@@ -97,6 +97,14 @@ def test_topk_matches_stable_argsort_and_breaks_ties_low():
         assert np.array_equal(ids, ref)
     ids, _ = moe.topk(z, 3)
     assert ids[0].tolist() == [0, 1, 2] and ids[1].tolist() == [3, 9, 12]
+    # the near-tie gap: k-th largest minus (k+1)-th largest logit, from a library sort;
+    # zero on a tie at the cut, infinite when every expert is selected
+    srt = -np.sort(-z.astype(np.float64), axis=1)
+    for k in (1, 3, 14, 15, 16):
+        _, gap = moe.topk(z, k)
+        want = srt[:, k - 1] - srt[:, k] if k < 16 else np.full(z.shape[0], np.inf)
+        assert np.array_equal(gap, want)
+    assert moe.topk(z, 3)[1][0] == 0.0 and moe.topk(z, 13)[1][2] == 0.0
 
 
 def test_router_logits_rank1_closed_form_and_einsum():
