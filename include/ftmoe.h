@@ -218,7 +218,9 @@ FT_API int ft_moe_set_int4_tensor_cores(ft_moe* h, int enabled);
  *   FT_INJECT_COPY_FAIL: the countdown-th slot fill from now is reported failed instead
  *     of being issued.  The forward returns FT_ERR_CUDA before launching its FFN; the
  *     entries of that fill and of the later fills of the same set become not resident
- *     (their accesses stay in the trace).  The next forward works normally.
+ *     (their accesses stay in the trace); the fills of the set issued before it stay
+ *     resident, and a later forward that reads them waits for their copies.  The next
+ *     forward works normally.
  *   FT_INJECT_ROUTE_TIMEOUT: the countdown-th routing wait reports FT_ERR_TIMEOUT (after
  *     the GPU work completes); the cache is unchanged.
  *   FT_INJECT_FUSED_WAIT: in the countdown-th fused decode FFN launch every down item

@@ -346,6 +346,18 @@ int issue_fills(ft_moe* h, std::vector<ftc::Access>& recs, size_t first) {
       for (size_t j = i; j < recs.size(); ++j)
         if (!recs[j].hit) h->lru.drop(recs[j].slot);
       h->timing_free.push_back(tm);
+      // the copies issued before this one still land: their slots stay resident, so mark
+      // them with a fill event that a later forward reading them waits on
+      std::vector<int> issued;
+      for (size_t j = first; j < i; ++j)
+        if (!recs[j].hit) issued.push_back(recs[j].slot);
+      if (!issued.empty()) {
+        const long long b = h->fill_batches++;
+        const int r = (int)(b % kRing);
+        cudaEventRecord(h->fill_ev[r], h->copy);
+        h->fill_ev_batch[r] = b;
+        for (int s : issued) h->slot_fill_batch[s] = b;
+      }
       return cuda_fail(h, e, "cudaMemcpyAsync (slot fill)");
     }
     h->st.h2d_bytes += (long long)h->blob;
