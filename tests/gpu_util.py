@@ -45,8 +45,17 @@ def first_divergence(gpu_ids, ref_ids, gap, zsel=None):
             assert np.max(np.abs(zg - zs[i])) < TIE_GAP, "token %d: order %s vs oracle %s" % (
                 i, g[i].tolist(), r[i].tolist())
             continue
+        assert len(set(g[i].tolist())) == len(g[i]), "token %d: repeated ids %s" % (i, g[i].tolist())
         assert gp[i] < TIE_GAP, "token %d: ids %s vs oracle %s with logit gap %.3g" % (
             i, g[i].tolist(), r[i].tolist(), gp[i])
+        if zs is not None:
+            # the experts left out must sit at the oracle's cut (its k-th logit): a tie
+            # moves only those
+            zmap = dict(zip(r[i].tolist(), zs[i].tolist()))
+            cut = float(np.min(zs[i]))
+            dropped = [e for e in r[i].tolist() if e not in set(g[i].tolist())]
+            assert all(zmap[e] - cut < TIE_GAP for e in dropped), \
+                "token %d: ids %s vs oracle %s drop an expert above the cut" % (i, g[i].tolist(), r[i].tolist())
         return i
     return None
 
