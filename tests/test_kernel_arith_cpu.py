@@ -1,0 +1,76 @@
+"""Bit-level identities the decode and prefill kernels rely on, checked exhaustively
+on the CPU with numpy (the kernels themselves are checked against the oracle by the
+GPU parity tests):
+
+* int4 -> bf16 without a conversion: a nibble n of a 4-bit two's-complement q, put in
+  the low mantissa bits of 0x4300 (128.0) after xor 8, is the bf16 value 136 + q.
+* NVFP4 staging: every product of an e2m1 value and an e4m3 block scale is exact in
+  f16 and in bf16, so the staged bf16 weight carries no rounding.
+* The bf16 hi/lo split of the fp32 h that the tensor-core down projection reads:
+  hi + lo equals h within 2^-17 relative.
+"""
+import numpy as np
+
+import synth
+
+
+def _bf16_bits_to_f32(bits):
+    return (np.asarray(bits, dtype=np.uint32) << 16).view(np.float32)
+
+
+def _e2m1(code):
+    sign = -1.0 if code & 8 else 1.0
+    e, m = (code >> 1) & 3, code & 1
+    return sign * (m * 0.5 if e == 0 else (1 + m / 2) * 2.0 ** (e - 1))
+
+
+def _e4m3(code):
+    sign = -1.0 if code & 0x80 else 1.0
+    e, m = (code >> 3) & 15, code & 7
+    return sign * (m / 8 * 2.0 ** -6 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7))
+
+
+def test_int4_nibble_xor_gives_bf16_136_plus_q():
+    # a 32-bit word holds nibbles 0..7; (w >> 4n) & 0x000F000F puts nibbles n and n+4
+    # in the low bits of the two 16-bit halves, xor 0x4308 per half makes 136 + q
+    rng = np.random.default_rng(0)
+    words = np.concatenate([rng.integers(0, 2 ** 32, 4096, dtype=np.uint64).astype(np.uint32),
+                            np.array([0, 0xFFFFFFFF, 0x88888888, 0x77777777], dtype=np.uint32)])
+    for n in range(4):
+        pair = ((words >> np.uint32(4 * n)) & np.uint32(0x000F000F)) ^ np.uint32(0x43084308)
+        lo = _bf16_bits_to_f32(pair & np.uint32(0xFFFF)).astype(np.float64)
+        hi = _bf16_bits_to_f32(pair >> np.uint32(16)).astype(np.float64)
+        for half, nib in ((lo, n), (hi, n + 4)):
+            q = ((words >> np.uint32(4 * nib)) & np.uint32(0xF)).astype(np.int64)
+            q = np.where(q >= 8, q - 16, q)
+            assert np.array_equal(half, 136.0 + q)
+
+
+def test_e2m1_times_e4m3_is_exact_in_f16_and_bf16():
+    e2 = [_e2m1(c) for c in range(16)]
+    e4 = [_e4m3(c) for c in range(256) if (c & 0x7F) != 0x7F]      # 0x7F / 0xFF are NaN
+    prod = np.array([a * b for a in e2 for b in e4], dtype=np.float64)
+    # f16: the kernel multiplies the two as an f16 pair
+    assert np.array_equal(prod.astype(np.float16).astype(np.float64), prod)
+    # bf16: the staged weight
+    bits = synth.round_bf16(prod.astype(np.float32))
+    assert np.array_equal(_bf16_bits_to_f32(bits).astype(np.float64), prod)
+    # and both factors are exact in f16 (the hardware conversions lose nothing)
+    assert np.array_equal(np.array(e4).astype(np.float16).astype(np.float64), np.array(e4))
+
+
+def test_bf16_hi_lo_split_keeps_h_within_2_pow_minus_17():
+    rng = np.random.default_rng(1)
+    h = np.concatenate([rng.standard_normal(200000) * s for s in (1e-3, 1.0, 30.0)]).astype(np.float32)
+    h = np.concatenate([h, np.float32([0.0, -0.0, 1.0, -1.0, 65504.0, 1e-30, 3.0e38])])
+    hi_bits = synth.round_bf16(h)
+    hi = _bf16_bits_to_f32(hi_bits)
+    r = (h - hi).astype(np.float32)          # exact in fp32: h and hi share the exponent range
+    lo = _bf16_bits_to_f32(synth.round_bf16(r))
+    got = hi.astype(np.float64) + lo.astype(np.float64)
+    err = np.abs(got - h.astype(np.float64))
+    assert np.all(err <= 2.0 ** -17 * np.abs(h.astype(np.float64)))
+    # hi alone is the plain bf16 rounding (8 significant bits, 2^-8 relative): the split
+    # adds the next 9 bits, since |h - hi| is at most half an ulp of hi
+    assert np.all(np.abs(hi.astype(np.float64) - h) <= 2.0 ** -8 * np.abs(h.astype(np.float64)))
+    assert np.max(err / np.maximum(np.abs(h.astype(np.float64)), 1e-300)) > 2.0 ** -19   # the bound is nearly reached
