@@ -171,7 +171,9 @@ def gates(z_sel: np.ndarray, gating: str) -> np.ndarray:
 
 
 def selected_set(ids: np.ndarray) -> np.ndarray:
-    """S: the sorted distinct experts chosen by any token of the batch."""
+    """S: the sorted distinct experts chosen by any token of the batch - the experts
+    whose weights one forward reads (FreeToken linux, "FreeToken's MoE memory
+    handling": only the experts the router asks for are brought to the GPU)."""
     return np.unique(np.asarray(ids).reshape(-1)).astype(np.int32)
 
 
@@ -181,6 +183,8 @@ def permute(ids: np.ndarray, E: int):
     counts[e] = number of pairs routed to e; offsets = exclusive prefix sum
     (length E+1); perm lists the flat pair index t*k + j grouped by expert in
     ascending expert order and, inside an expert, by ascending token.
+    READING: the pages give no grouping; this stable order is the plainest one
+    that lets each expert's weights be read once per forward.
     """
     ids = np.asarray(ids)
     T, k = ids.shape
@@ -205,11 +209,17 @@ def permute(ids: np.ndarray, E: int):
 
 
 def silu(a: np.ndarray) -> np.ndarray:
+    """silu(a) = a * sigmoid(a).  READING: the pages name no expert FFN; the stated
+    workloads use SwiGLU experts, whose activation this is."""
     return a / (1.0 + np.exp(-a))
 
 
 def swiglu_ffn(a: np.ndarray, w_gate: np.ndarray, w_up: np.ndarray, w_down: np.ndarray) -> np.ndarray:
-    """y = W_down (silu(W_gate a) * (W_up a)) for each row a of `a` [n, H]."""
+    """y = W_down (silu(W_gate a) * (W_up a)) for each row a of `a` [n, H].
+
+    READING: one routed expert is a SwiGLU FFN with gate and up [I, H] and down
+    [H, I] (the stated workloads; the pages only say that each active expert runs
+    on the token - FreeToken linux, "FreeToken's MoE memory handling")."""
     a = np.asarray(a, dtype=np.float64)
     u = a @ w_gate.T
     v = a @ w_up.T
@@ -221,7 +231,9 @@ def swiglu_ffn(a: np.ndarray, w_gate: np.ndarray, w_up: np.ndarray, w_down: np.n
 
 
 def route(x, w_router, k, gating):
-    """Router + top-k + gates for a batch: returns dict(ids, gates, gap, z)."""
+    """Router + top-k + gates for a batch: returns dict(ids, gates, gap, z).
+    (FreeToken linux, "FreeToken's MoE memory handling": the router picks a few
+    experts per token; the readings are those of router_logits, topk and gates.)"""
     z = router_logits(x, w_router)
     ids, gap = topk(z, k)
     z_sel = np.take_along_axis(z, ids.astype(np.int64), axis=1)
@@ -231,7 +243,11 @@ def route(x, w_router, k, gating):
 def experts_and_combine(x, ids, g, E, wdtype, H, I, blob_of, shared_blob=None):
     """Permute the (token, slot) pairs by expert, run each selected expert's FFN on
     its tokens, and mix: out[t] = sum_{j<k} g[t,j] * y[t,j] (+ shared FFN(x_t)),
-    the sum taken in ascending j."""
+    the sum taken in ascending j.
+
+    (FreeToken linux, "FreeToken's MoE memory handling": each active expert runs on
+    the token and the outputs are mixed by the gate weights.  READINGS: the mixing
+    order is ascending j; a shared expert is added with weight 1.)"""
     x = np.asarray(x, dtype=np.float64)
     T, k = ids.shape
     counts, offsets, perm = permute(ids, E)
