@@ -11,6 +11,7 @@ import pytest
 import test_oracle_pins as pins
 from oracle import lru as olru
 from oracle import moe
+from oracle import run as orun
 
 _o = {n: getattr(moe, n) for n in (
     "widen_bf16", "decode_int4", "dequant_int4", "decode_e2m1", "decode_e4m3", "dequant_nvfp4",
@@ -149,6 +150,18 @@ class _HighestFreeSlot:
     heappop = staticmethod(lambda a: a.pop())
 
 
+class _NoLayer0Prefetch(olru.SharedLru):
+    def access_set(self, call, layer, experts, kind=olru.ROUTED):
+        if kind == olru.PREFETCH and layer == 0:
+            return []
+        return super().access_set(call, layer, experts, kind)
+
+
+class _PrefetchCountedAsRouted(olru.SharedLru):
+    def access_set(self, call, layer, experts, kind=olru.ROUTED):
+        return super().access_set(call, layer, experts, olru.ROUTED)
+
+
 MUTANTS = {
     # name: [(module, attribute, replacement)]
     "bf16 widened with a 15-bit shift": [
@@ -190,6 +203,8 @@ MUTANTS = {
          _o["experts_and_combine"](x, ids, g, E, wd, H, I, blob_of, None))],
     "only each token's first choice made resident": [
         (moe, "selected_set", lambda ids: _o["selected_set"](np.asarray(ids)[:, :1]))],
+    "prefill skips the prefetch of layer 0": [(orun, "SharedLru", _NoLayer0Prefetch)],
+    "prefill prefetches counted as routed accesses": [(orun, "SharedLru", _PrefetchCountedAsRouted)],
     "LRU evicts the most recently used": [(olru, "OrderedDict", _EvictMru)],
     "LRU hits not refreshed": [(olru, "OrderedDict", _NoRefresh)],
     "misses take the highest free slot": [(olru, "heapq", _HighestFreeSlot)],

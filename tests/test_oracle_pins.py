@@ -368,6 +368,38 @@ def test_prefill_double_buffer_evicts_exactly_the_previous_layer():
             assert a.ev_layer == a.layer - 2                   # victims: the layer before last
 
 
+def test_prefill_double_buffer_hand_worked_golden():
+    # routers built so that one-hot tokens make the file's selections (top-1, 2 tokens
+    # per step: token 0 picks the first listed expert, token 1 the last)
+    L, E, H, steps = 3, 3, 4, 2
+    sel, want, stats = {}, [], None
+    for f in _golden_lines("prefill_double_buffer_hand.txt"):
+        if f[0] == "select":
+            sel[(int(f[1]), int(f[2]))] = [int(v) for v in f[3:]]
+        elif f[0] == "stats":
+            stats = tuple(int(v) for v in f[1:])
+        else:
+            want.append((int(f[0]), int(f[1]), int(f[2]), olru.PREFETCH if f[3] == "P" else olru.ROUTED,
+                         f[4] == "hit", int(f[5]), int(f[6]), int(f[7])))
+    W = np.zeros((L, E, H), dtype=np.float32)
+    for (s_, l), es in sel.items():
+        W[l, es[0], 2 * s_] = 1.0
+        W[l, es[-1], 2 * s_ + 1] = 1.0
+    x = np.zeros((steps, 2, H))
+    for s_ in range(steps):
+        x[s_, 0, 2 * s_] = x[s_, 1, 2 * s_ + 1] = 1.0
+    r = run_workload(L=L, E=E, H=H, I=8, k=1, gating="softmax", wdtype="f32", capacity=2 * E,
+                     x_steps=x, router_of=lambda l: W[l], blob_of=lambda l, e: None,
+                     prefill=True, ffn_steps=[])
+    for (s_, l), es in sel.items():
+        assert sorted(set(r["ids"][s_, l].reshape(-1).tolist())) == es
+    got = [(a.call, a.layer, a.expert, a.kind, a.hit, a.slot, a.ev_layer, a.ev_expert) for a in r["trace"]]
+    assert got == want
+    st = r["stats"]
+    assert (st.routed, st.hits, st.misses, st.prefetch, st.prefetch_hits, st.prefetch_misses,
+            st.evictions) == stats
+
+
 def test_ar1_tokens_have_locality():
     x = synth.ar1_chain(0, 0, 4000, 64).astype(np.float64)
     assert abs(x.var() - 1.0) < 0.1
