@@ -162,6 +162,12 @@ class _PrefetchCountedAsRouted(olru.SharedLru):
         return super().access_set(call, layer, experts, olru.ROUTED)
 
 
+class _ShrinkMovesNotReported(olru.SharedLru):
+    def resize(self, new_capacity):
+        super().resize(new_capacity)
+        return []
+
+
 MUTANTS = {
     # name: [(module, attribute, replacement)]
     "bf16 widened with a 15-bit shift": [
@@ -203,6 +209,7 @@ MUTANTS = {
          _o["experts_and_combine"](x, ids, g, E, wd, H, I, blob_of, None))],
     "only each token's first choice made resident": [
         (moe, "selected_set", lambda ids: _o["selected_set"](np.asarray(ids)[:, :1]))],
+    "shrink moves not carried to the slot arena": [(orun, "SharedLru", _ShrinkMovesNotReported)],
     "prefill skips the prefetch of layer 0": [(orun, "SharedLru", _NoLayer0Prefetch)],
     "prefill prefetches counted as routed accesses": [(orun, "SharedLru", _PrefetchCountedAsRouted)],
     "LRU evicts the most recently used": [(olru, "OrderedDict", _EvictMru)],

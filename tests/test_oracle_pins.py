@@ -344,6 +344,28 @@ def test_capacity_independence_and_fused_equivalence():
     assert runs[0]["stats"].misses > runs[-1]["stats"].misses
 
 
+def test_results_unchanged_by_a_resize_through_the_slots():
+    # a grow and a shrink half-way (FreeToken RTX 5090, dynamic reconfiguration: the
+    # cache size changes speed, not the result); experts are read from the slot arena,
+    # so a shrink's slot moves must carry the bytes along
+    # one token per step and 2 of 8 experts per layer: the survivors a shrink moves are
+    # read again before they are evicted
+    cfg = synth.MoeConfig("t", L=2, E=8, H=32, I=16, k=2, gating="softmax", wdtype="bf16",
+                          shared=False, C=4, tokens=16, batches=(1,), process="ar1", mode="decode")
+    x, _ = synth.tokens(cfg, 1)
+    x = x[:12]
+    blobs = {(l, e): synth.expert_blob(cfg, l, e) for l in range(cfg.L) for e in range(cfg.E)}
+    kw = dict(L=cfg.L, E=cfg.E, H=cfg.H, I=cfg.I, k=cfg.k, gating=cfg.gating, wdtype=cfg.wdtype,
+              x_steps=x, router_of=lambda l: synth.router_weights(cfg, l), blob_of=lambda l, e: blobs[(l, e)])
+    direct = run_workload(capacity=cfg.L * cfg.E, through_slots=False, **kw)
+    for c0, c1 in ((20, 4), (4, 20)):
+        r = run_workload(capacity=c0, resize_to=c1, through_slots=True, **kw)
+        assert np.array_equal(r["ids"], direct["ids"])
+        for key in direct["out"]:
+            assert np.array_equal(r["out"][key], direct["out"][key]), (c0, c1, key)
+        assert r["lru"].capacity == c1
+
+
 def test_config1_oracle_runs_and_gates_sum_to_one():
     cfg = synth.CONFIGS["tiny-fp32"]
     r = _tiny_run(cfg, cfg.C, True, steps=8)
