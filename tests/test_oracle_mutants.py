@@ -3,11 +3,13 @@ oracle (a swapped operand, a wrong index, sign, bias or order, a dropped term), 
 every pin of `test_oracle_pins.py` against the planted oracle, and requires at least
 one pin to fail.  Mistakes are planted only in the oracle, on the CPU, through
 monkeypatch; nothing here touches the CUDA path."""
+import heapq
 from collections import OrderedDict
 
 import numpy as np
 import pytest
 
+import synth
 import test_oracle_pins as pins
 from oracle import lru as olru
 from oracle import moe
@@ -134,6 +136,48 @@ def _permute_inclusive_offsets(ids, E):
     return counts, np.concatenate([offsets[1:], offsets[-1:]]), perm
 
 
+def _int4_gate_up_scales_swapped(blob, wdtype, H, I):
+    if wdtype != "int4":
+        return _o["expert_weights"](blob, wdtype, H, I)
+    blob = np.asarray(blob, dtype=np.uint8).reshape(-1)
+    m, g = H * I, H * I // 128
+    q, s = blob[:3 * m // 2], blob[3 * m // 2:].view(np.uint16)
+    return (moe.dequant_int4(q[:m // 2].reshape(I, H // 2), s[g:2 * g].reshape(I, H // 128)),
+            moe.dequant_int4(q[m // 2:m].reshape(I, H // 2), s[:g].reshape(I, H // 128)),
+            moe.dequant_int4(q[m:3 * m // 2].reshape(H, I // 2), s[2 * g:3 * g].reshape(H, I // 128)))
+
+
+def _nvfp4_swap_regions(first, size):
+    def expert_weights(blob, wdtype, H, I):
+        if wdtype != "nvfp4":
+            return _o["expert_weights"](blob, wdtype, H, I)
+        b = np.array(blob, dtype=np.uint8).reshape(-1)
+        o, n = first(H * I), size(H * I)
+        a, c = b[o:o + n].copy(), b[o + n:o + 2 * n].copy()
+        b[o:o + n], b[o + n:o + 2 * n] = c, a
+        return _o["expert_weights"](b, wdtype, H, I)
+    return expert_weights
+
+
+def _router_rounded_to_bf16(x, w):
+    z = _o["router_logits"](x, w)
+    return (synth.round_bf16(z).astype(np.uint32) << 16).view(np.float32)
+
+
+def _shared_expert_halved(x, ids, g, E, wd, H, I, blob_of, shared_blob=None):
+    out = _o["experts_and_combine"](x, ids, g, E, wd, H, I, blob_of, None)
+    if shared_blob is not None:
+        wg, wu, wdn = moe.expert_weights(shared_blob, wd, H, I)
+        out = out + 0.5 * moe.swiglu_ffn(np.asarray(x, np.float64), wg, wu, wdn)
+    return out
+
+
+class _GrowAddsNoFreeSlot:
+    heapify = staticmethod(heapq.heapify)
+    heappop = staticmethod(heapq.heappop)
+    heappush = staticmethod(lambda a, v: None)
+
+
 class _EvictMru(OrderedDict):
     def popitem(self, last=True):
         return super().popitem(last=True)
@@ -183,6 +227,14 @@ MUTANTS = {
     "nvfp4 nibbles in swapped order": [
         (moe, "dequant_nvfp4", lambda p, s, g: _o["dequant_nvfp4"](_swap_nibbles(p), s, g))],
     "nvfp4 tensor scale dropped": [(moe, "dequant_nvfp4", lambda p, s, g: _o["dequant_nvfp4"](p, s, 1.0))],
+    "int4 gate and up scale arrays swapped": [(moe, "expert_weights", _int4_gate_up_scales_swapped)],
+    "nvfp4 gate and up tensor scales swapped": [
+        (moe, "expert_weights", _nvfp4_swap_regions(lambda m: 3 * m // 2 + 3 * m // 16, lambda m: 4))],
+    "nvfp4 gate and up block-scale arrays swapped": [
+        (moe, "expert_weights", _nvfp4_swap_regions(lambda m: 3 * m // 2, lambda m: m // 16))],
+    "router logits rounded to bf16": [(moe, "router_logits", _router_rounded_to_bf16)],
+    "shared expert at weight 1/2": [(moe, "experts_and_combine", _shared_expert_halved)],
+    "grow adds no free slot": [(olru, "heapq", _GrowAddsNoFreeSlot)],
     "gate and up swapped in the blob": [
         (moe, "expert_weights", lambda b, w, H, I: (lambda r: (r[1], r[0], r[2]))(_o["expert_weights"](b, w, H, I)))],
     "down matrix read transposed": [(moe, "expert_weights", _down_read_transposed)],
