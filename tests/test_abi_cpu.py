@@ -185,3 +185,18 @@ def test_calls_fail_cleanly_without_a_device():
     with pytest.raises(ft.FtError) as ei:
         ft.ft_moe_create(16, 2, 256, 128, "f32", 4)
     assert "allocation" in str(ei.value) or "CUDA" in str(ei.value)
+
+
+def test_import_fails_loudly_without_the_library(tmp_path):
+    # the package's Python files without libftmoe.so: no fallback, the import raises
+    import shutil
+    import sys
+    src = os.path.dirname(ft.__file__)
+    dst = tmp_path / "moe_expert_offload_top_b200"
+    dst.mkdir()
+    for name in os.listdir(src):
+        if name.endswith(".py"):
+            shutil.copy(os.path.join(src, name), dst / name)
+    r = subprocess.run([sys.executable, "-c", "import moe_expert_offload_top_b200"], cwd=tmp_path,
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "ImportError" in r.stderr and "not built" in r.stderr
