@@ -49,6 +49,8 @@ def lib():
             L.synth_expert_blob.argtypes = [u64, i32, i32, i32, i32, i32, i32, f32, vp]
             L.synth_fill_pool.argtypes = [u64, i32, i32, i32, i32, i32, f32, vp, u64, i32]
             L.synth_ar1.argtypes = [u64, i32, i32, i32, f32, f32, vp]
+            L.synth_philox4x32_10.argtypes = [vp, vp, vp]
+            L.synth_normal_f32_scalar.argtypes = [u64, i32, i32, i32, u64, u64, f32, vp]
             _lib = L
     return _lib
 
@@ -61,6 +63,23 @@ def _ptr(a: np.ndarray) -> int:
 def normal_f32(seed, tensor, layer, expert, n, sigma=1.0, offset=0) -> np.ndarray:
     out = np.empty(n, dtype=np.float32)
     lib().synth_normal_f32(seed, tensor, layer, expert, offset, n, sigma, _ptr(out))
+    return out
+
+
+def philox4x32_10(ctr, key) -> np.ndarray:
+    """The bare Philox-4x32-10 bijection of the generator (4 counter words, 2 key words)."""
+    c = np.ascontiguousarray(ctr, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    assert c.shape == (4,) and k.shape == (2,)
+    out = np.empty(4, dtype=np.uint32)
+    lib().synth_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def normal_f32_scalar(seed, tensor, layer, expert, n, sigma=1.0, offset=0) -> np.ndarray:
+    """normal_f32 through the scalar one-block path (for checking the vectorised path)."""
+    out = np.empty(n, dtype=np.float32)
+    lib().synth_normal_f32_scalar(seed, tensor, layer, expert, offset, n, sigma, _ptr(out))
     return out
 
 

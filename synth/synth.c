@@ -175,6 +175,27 @@ SYNTH_API void synth_normal_f32(uint64_t seed, int tensor, int layer, int expert
   }
 }
 
+/* The bare Philox-4x32-10 bijection: out = Philox(ctr, key).  Exported so that the
+ * published known-answer vectors can be checked against the generator's own rounds. */
+SYNTH_API void synth_philox4x32_10(const uint32_t* ctr, const uint32_t* key, uint32_t* out) {
+  uint32_t c[4] = {ctr[0], ctr[1], ctr[2], ctr[3]};
+  philox4x32_10(c, key[0], key[1]);
+  memcpy(out, c, sizeof c);
+}
+
+/* synth_normal_f32 computed one counter block at a time through the scalar rounds:
+ * a check of the 16-block (vectorised) path, which must give the same bits. */
+SYNTH_API void synth_normal_f32_scalar(uint64_t seed, int tensor, int layer, int expert,
+                                       uint64_t offset, uint64_t n, float sigma, float* dst) {
+  pthread_once(&g_q_once, init_quantiles);
+  uint64_t key = tensor_key(seed, tensor, layer, expert);
+  for (uint64_t i = offset; i < offset + n; ++i) {
+    float blk[4];
+    normal_block(key, i >> 2, blk);
+    dst[i - offset] = sigma * blk[i & 3];
+  }
+}
+
 static inline uint16_t bf16_rne(float f) {
   uint32_t u;
   memcpy(&u, &f, 4);

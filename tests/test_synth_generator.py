@@ -1,0 +1,48 @@
+"""The seeded input generator (`synth`), checked against facts other than itself: the
+published Philox-4x32-10 known-answer vectors, its vectorised path against its scalar
+one, and the moments of the normals it draws."""
+import os
+
+import numpy as np
+
+import synth
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def test_philox_known_answer_vectors():
+    n = 0
+    with open(os.path.join(GOLD, "philox4x32_10_kat.txt")) as f:
+        for ln in f:
+            if not ln.strip() or ln.startswith("#"):
+                continue
+            w = [int(v, 16) for v in ln.split()]
+            got = synth.philox4x32_10(w[0:4], w[4:6])
+            assert got.tolist() == w[6:10], ln
+            n += 1
+    assert n == 3
+
+
+def test_vectorised_normals_equal_the_scalar_path():
+    # offsets and lengths that start and end inside a 16-block group
+    for seed, tensor, layer, expert in ((0, 1, 0, 0), (7, 4, 3, 255), (123456789, 8, 15, 17)):
+        for off, n in ((0, 64), (0, 1000), (13, 51), (63, 2), (1000003, 777)):
+            a = synth.normal_f32(seed, tensor, layer, expert, n, 0.02, off)
+            b = synth.normal_f32_scalar(seed, tensor, layer, expert, n, 0.02, off)
+            assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    # a slice of a longer draw is the draw of that slice
+    full = synth.normal_f32(3, 2, 1, 5, 4096)
+    assert np.array_equal(full[1000:1500], synth.normal_f32(3, 2, 1, 5, 500, offset=1000))
+
+
+def test_normals_have_standard_moments_and_bounded_tails():
+    z = synth.normal_f32(11, 1, 0, 0, 1 << 21).astype(np.float64)
+    n = z.size
+    assert abs(z.mean()) < 5 / np.sqrt(n)
+    assert abs(z.var() - 1) < 5 * np.sqrt(2 / n) + 1e-4      # the table's tails end at 4.42
+    assert abs(np.mean(z ** 3)) < 5 * np.sqrt(15 / n)
+    assert abs(np.mean(z ** 4) - 3) < 0.02
+    assert np.abs(z).max() <= 4.43
+    # distinct tensors, layers and experts draw unrelated streams
+    w = synth.normal_f32(11, 1, 0, 1, 1 << 21).astype(np.float64)
+    assert abs(np.corrcoef(z, w)[0, 1]) < 5 / np.sqrt(n)
