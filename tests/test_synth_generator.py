@@ -46,3 +46,14 @@ def test_normals_have_standard_moments_and_bounded_tails():
     # distinct tensors, layers and experts draw unrelated streams
     w = synth.normal_f32(11, 1, 0, 1, 1 << 21).astype(np.float64)
     assert abs(np.corrcoef(z, w)[0, 1]) < 5 / np.sqrt(n)
+
+
+def test_bf16_rounding_matches_torch_round_to_nearest_even():
+    import torch
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.standard_normal(100000).astype(np.float32) * s for s in (1e-30, 1e-3, 1.0, 1e30)])
+    # exact halfway points between two bf16 values, both parities of the kept bit
+    halves = (np.arange(0, 1 << 16, 97, dtype=np.uint32) << 16 | 0x8000).view(np.float32)
+    x = np.concatenate([x, halves[np.isfinite(halves)], np.float32([0.0, -0.0, 1.0, -1.0, 3.0e38, -3.0e38])])
+    want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(synth.round_bf16(x), want)
