@@ -57,3 +57,32 @@ def test_bf16_rounding_matches_torch_round_to_nearest_even():
     x = np.concatenate([x, halves[np.isfinite(halves)], np.float32([0.0, -0.0, 1.0, -1.0, 3.0e38, -3.0e38])])
     want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(synth.round_bf16(x), want)
+
+
+def test_int4_quantiser_follows_the_stated_rule():
+    # s = bf16(max|w| / 7) per 128 reduction-axis elements, q = clamp(rint(w / s), -8, 7)
+    # with ties to even, element 2b in the low nibble of byte b
+    rng = np.random.default_rng(9)
+    w = (rng.standard_normal((6, 512)) * 0.02).astype(np.float32)
+    w[1, 128:256] = 0.0                                       # an all-zero group: s = 0, q = 0
+    q, sbits = synth.quantise_int4(w)
+    s = (sbits.astype(np.uint32) << 16).view(np.float32)
+    amax = np.abs(w.reshape(6, 4, 128)).max(axis=2)
+    assert np.array_equal(sbits, synth.round_bf16((amax / np.float32(7)).astype(np.float32)))
+    # exact ties: w = (n + 1/2) s for a group's own s must round to the even neighbour
+    w2 = w.copy()
+    for g in range(4):
+        sg = s[0, g]
+        w2[0, 128 * g + 1:128 * g + 9] = (np.arange(-4, 4, dtype=np.float32) + np.float32(0.5)) * sg
+    q2, s2 = synth.quantise_int4(w2)
+    for ww, qq, ss in ((w, q, sbits), (w2, q2, s2)):
+        sv = np.repeat((ss.astype(np.uint32) << 16).view(np.float32), 128, axis=1)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            want = np.where(sv == 0, 0, np.clip(np.rint(ww / sv), -8, 7)).astype(np.int64)
+        lo = (qq & 0x0F).astype(np.int64)
+        hi = (qq >> 4).astype(np.int64)
+        got = np.empty_like(want)
+        got[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
+        got[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
+        assert np.array_equal(got, want)
+    assert np.all(q[1, 64:128] == 0)
