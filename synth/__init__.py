@@ -178,5 +178,6 @@ def tokens(cfg: MoeConfig, batch: int):
     return x, None
 
 
-__all__ = ["MoeConfig", "CONFIGS", "build", "lib", "normal_f32", "round_bf16", "quantise_int4", "quantise_nvfp4",
-           "expert_weights_f32", "expert_blob", "fill_pool", "router_weights", "ar1_chain", "tokens"]
+__all__ = ["MoeConfig", "CONFIGS", "build", "lib", "normal_f32", "normal_f32_scalar", "philox4x32_10", "round_bf16",
+           "quantise_int4", "quantise_nvfp4", "expert_weights_f32", "expert_blob", "fill_pool", "router_weights",
+           "ar1_chain", "tokens"]
