@@ -9,13 +9,16 @@ AR(1) process x_t = 0.9 x_{t-1} + 0.436 eps_t (routing locality), batch 1.
 Synthetic data stands in for the agent workloads and replayed traces of the
 FreeToken pages.
 
-    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--prefill]
 
 Reports (one JSON line, rank 0): decode tokens/s timed on the device with
 CUDA events (max over ranks), an end-to-end figure through host buffers, the
-roofline of the dominant kernel (the fused decode expert FFN, HBM-bound) from
-live CUDA events, cache miss rate and H2D fill bandwidth, SM clocks sampled
-during the timed region, and the CPU oracle timed on a bounded sample.
+roofline of the dominant kernel (the decode gate/up expert GEMV, HBM-bound) from
+live CUDA events, cache miss rate and H2D fill bandwidth, the cold-start figure
+of the warm-up steps, SM clocks sampled during the timed region, and the CPU
+oracle timed on a bounded sample.  --prefill adds the 4096-token prefill of the
+DeepSeek-V4-Flash-shaped stack (8 layers, 256 experts), offloaded and resident.
+--impl reference times the CPU oracle alone on the same workload.
 N > 1 runs independent replicas (one stack per GPU, its own token chain):
 the path has no exchange step.
 """
