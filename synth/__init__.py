@@ -1,8 +1,9 @@
 """Seeded synthetic inputs shared by the oracle and the CUDA path.
 
-Holds no arithmetic of the method: it draws numbers (Philox-4x32-10 +
-Box-Muller, see synth.c), rounds them to the stored formats, and writes expert
-blobs in the runtime layout.  The C source is compiled on first use.
+Holds no arithmetic of the method: it draws numbers (Philox-4x32-10, and
+normals by inversion through a 65 536-cell quantile table; see synth.c), rounds
+them to the stored formats, and writes expert blobs in the runtime layout.  The
+C source is compiled on first use.
 """
 import ctypes
 import os
