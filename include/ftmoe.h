@@ -414,6 +414,29 @@ FT_API int ft_expert_ffn_decode(const void* x, int T, int H, int I, int top_k, i
                          int max_pairs_per_expert, const int* offsets, const int* perm, float* h,
                          float* y, void* stream);
 
+/* SwiGLU FFN of a list of experts for prefill-sized batches, on the tcgen05 grouped GEMMs
+ * that ft_moe_forward runs in prefill ("FreeToken linux", "FreeToken's MoE memory
+ * handling": in prefill every selected expert runs from the slot that holds it, while
+ * the next layer's experts are copied in).  bf16 weights; H % 256 == 0, I % 128 == 0.
+ *   weights: DEVICE array of n_slots bf16 expert blobs (runtime layout, see
+ *     ft_moe_pool_ptr), 3*H*I*2 bytes apart, 16-byte aligned.  experts, slots: HOST
+ *     arrays of n_list entries (n_list <= FT_MAX_EXPERTS + 1): entry i is routed expert
+ *     experts[i] (its pairs q in [offsets[e], offsets[e+1])) or, for experts[i] = -1 (at
+ *     most one entry), a shared expert (pairs q = T*k + t for every token t); its weights
+ *     are blob slots[i] (0 <= slots[i] < n_slots) of `weights`.
+ *   x: [T][H] bf16.  offsets [E+1], perm [T*k]: as written by ft_permute.
+ *   a_rows: [T*k + T][H] bf16 scratch (written: the gathered token row of every pair).
+ *   h: [T*k + T][I] bf16 (written): h[q] = bf16(silu(W_gate x_t) * (W_up x_t)), fp32 accumulation.
+ *   y: [T*k + T][H] f32 (written): y[q] = W_down h[q], fp32 accumulation.
+ *   err: a DEVICE int, 0 before the call; a kernel whose bounded pipeline wait gives up
+ *     writes 101-104 there (the outputs are then incomplete).
+ * Rows that no entry owns are not written.  Allocates nothing (the tensor maps are built
+ * on the host per call).  FT_ERR_INVALID (message in ft_last_error(NULL)) for bad sizes,
+ * entries or alignment; FT_ERR_CUDA if a launch fails. */
+FT_API int ft_expert_ffn_prefill(const void* x, int T, int H, int I, int top_k, const void* weights, int n_slots,
+                                 const int* experts, const int* slots, int n_list, const int* offsets,
+                                 const int* perm, void* a_rows, void* h, float* y, int* err, void* stream);
+
 /* Gate-weighted combine: out[t] = sum_{j<k} gates[t][j] * y[inv[t*k+j]], summed in
  * ascending j in fp32, plus y[T*k + t] (weight 1) when has_shared.
  *   y: device f32 rows (see ft_expert_ffn_decode), gates: [T][k] f32, inv: [T*k] int32,
@@ -442,10 +465,13 @@ FT_API int ft_combine(const float* y, const float* gates, const int* inv, int T,
  *  - Calls no cudaMalloc, cudaFree or other allocating routine.  The first call on a
  *    device looks up the array's device address (cudaGetSymbolAddress, with that device
  *    current) and caches it; make that first call before any stream capture.
- *  - Every call on a device uses the same array, which keeps the last call's contents
- *    (nothing in it needs to start at zero: each call writes every row it reads).  Calls
- *    whose kernels overlap on the GPU (other streams, other threads) race on it: order
- *    them on one stream. */
+ *  - Every call on a device uses the same array, which keeps the last call's contents.
+ *    Nothing in it needs to start at zero, because each call writes every row it reads,
+ *    provided the list is complete: it must hold every expert that occurs in the routed
+ *    ids (the rows of an expert missing from it would be read as left by an earlier call,
+ *    possibly of another model), and exactly one entry -1 when has_shared is set (none
+ *    otherwise; checked, FT_ERR_INVALID).  Calls whose kernels overlap on the GPU (other
+ *    streams, other threads) race on the array: order them on one stream. */
 FT_API int ft_expert_ffn_decode_noalloc(const void* x, int T, int H, int I, int top_k, int wdtype,
                                         const void* const* blobs, const int* experts, int n_list,
                                         int max_pairs_per_expert, const int* offsets, const int* perm,

@@ -91,6 +91,8 @@ _SIGS = {
     "ft_route_decode": ([_vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
     "ft_expert_ffn_decode": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp], _i),
     "ft_combine": ([_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp], _i),
+    "ft_expert_ffn_prefill": ([_vp, _i, _i, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+                              _i),
     "ft_expert_ffn_decode_noalloc": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _i,
                                       _vp, _vp], _i),
     "ft_version": ([], ctypes.c_char_p),
@@ -323,6 +325,17 @@ def ft_expert_ffn_decode(x, T, H, I, top_k, wdtype, blobs, experts, max_pairs_pe
     return _check(None, _lib.ft_expert_ffn_decode(
         _p(x), T, H, I, top_k, WDTYPE.get(wdtype, wdtype), ctypes.cast(bl, ctypes.c_void_p),
         ctypes.cast(ex, ctypes.c_void_p), n, max_pairs_per_expert, _p(offsets), _p(perm), _p(h), _p(y),
+        _s(stream)))
+
+
+def ft_expert_ffn_prefill(x, T, H, I, top_k, weights, n_slots, experts, slots, offsets, perm, a_rows, h, y, err,
+                          stream=None):
+    n = len(experts)
+    ex = _int_array(list(experts) or [0])
+    sl = _int_array(list(slots) or [0])
+    return _check(None, _lib.ft_expert_ffn_prefill(
+        _p(x), T, H, I, top_k, _p(weights), n_slots, ctypes.cast(ex, ctypes.c_void_p),
+        ctypes.cast(sl, ctypes.c_void_p), n, _p(offsets), _p(perm), _p(a_rows), _p(h), _p(y), _p(err),
         _s(stream)))
 
 

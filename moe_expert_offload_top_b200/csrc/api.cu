@@ -1466,6 +1466,61 @@ int ft_expert_ffn_decode(const void* x, int T, int H, int I, int top_k, int wdty
              : FT_ERR_CUDA;
 }
 
+int ft_expert_ffn_prefill(const void* x, int T, int H, int I, int top_k, const void* weights, int n_slots,
+                          const int* experts, const int* slots, int n_list, const int* offsets, const int* perm,
+                          void* a_rows, void* h, float* y, int* err, void* stream) {
+  auto bad = [](const char* why) {
+    ftk::set_step_error(std::string("ft_expert_ffn_prefill: ") + why);
+    return FT_ERR_INVALID;
+  };
+  if (T < 0 || top_k < 1 || n_list < 0 || n_list > ftk::kMaxList || n_slots < 1)
+    return bad("invalid size");
+  if (H < 256 || I < 128 || H % 256 || I % 128) return bad("H must be a multiple of 256 and I of 128");
+  if (T == 0 || n_list == 0) return FT_OK;
+  if (!x || !weights || !experts || !slots || !offsets || !perm || !a_rows || !h || !y || !err)
+    return bad("null pointer");
+  if (((uintptr_t)weights | (uintptr_t)a_rows | (uintptr_t)h) & 15) return bad("buffers must be 16-byte aligned");
+  ftk::GemmGroups groups;
+  groups.n = n_list;
+  int n_shared = 0;
+  for (int i = 0; i < n_list; ++i) {
+    if (experts[i] < -1 || experts[i] >= FT_MAX_EXPERTS || slots[i] < 0 || slots[i] >= n_slots)
+      return bad("bad expert list entry");
+    n_shared += experts[i] < 0;
+    groups.expert[i] = experts[i];
+    groups.z[i] = slots[i];
+  }
+  if (n_shared > 1) return bad("more than one shared-expert entry");
+  const uint64_t rows = (uint64_t)T * top_k + T;
+  const uint64_t blob = 3ull * H * I * 2;
+  const unsigned char* w = static_cast<const unsigned char*>(weights);
+  ftk::GemmMaps m;
+  bool ok = ftk::encode_map_2d(&m.a_x, a_rows, H, rows, (uint64_t)H * 2, 128) &&
+            ftk::encode_map_2d(&m.a_h, h, I, rows, (uint64_t)I * 2, 128) &&
+            ftk::encode_map_3d(&m.b1_routed, w, H, 2ull * I, n_slots, (uint64_t)H * 2, blob, 128) &&
+            ftk::encode_map_3d(&m.b2_routed, w + 2ull * I * H * 2, I, H, n_slots, (uint64_t)I * 2, blob, 256);
+  if (!ok) {
+    ftk::set_step_error("ft_expert_ffn_prefill: cuTensorMapEncodeTiled failed");
+    return FT_ERR_CUDA;
+  }
+  m.b1_shared = m.b1_routed;   // the shared expert is a slot of the same array
+  m.b2_shared = m.b2_routed;
+  int dev = 0, num_sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = ftk::launch_gather_rows(x, perm, T, top_k, H, n_shared > 0, a_rows, s);
+  if (e == cudaSuccess)
+    e = ftk::launch_grouped_gemm(0, m, groups, offsets, T, top_k, I, H, h, err, num_sms, s);
+  if (e == cudaSuccess)
+    e = ftk::launch_grouped_gemm(1, m, groups, offsets, T, top_k, I, H, y, err, num_sms, s);
+  if (e != cudaSuccess) {
+    ftk::set_step_error(std::string("ft_expert_ffn_prefill: launch: ") + cudaGetErrorString(e));
+    return FT_ERR_CUDA;
+  }
+  return FT_OK;
+}
+
 int ft_combine(const float* y, const float* gates, const int* inv, int T, int H, int top_k,
                int has_shared, int out_is_bf16, void* out, void* stream) {
   if (T < 0 || H < 4 || H % 4 || top_k < 1 || (T > 0 && (!y || !gates || !inv || !out)))

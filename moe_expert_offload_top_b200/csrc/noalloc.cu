@@ -69,13 +69,22 @@ extern "C" int ft_expert_ffn_decode_noalloc(const void* x, int T, int H, int I, 
   if (T == 0) return FT_OK;
   ftk::ExpertList list;
   list.n = n_list;
+  int n_shared = 0;
   for (int i = 0; i < n_list; ++i) {
     if (experts[i] < -1 || experts[i] >= FT_MAX_EXPERTS || !blobs[i]) {
       ftk::set_step_error("ft_expert_ffn_decode_noalloc: bad expert list entry");
       return FT_ERR_INVALID;
     }
+    n_shared += experts[i] < 0;
     list.expert[i] = experts[i];
     list.blob[i] = static_cast<const uint8_t*>(blobs[i]);
+  }
+  // the combine reads the shared expert's rows exactly when has_shared is set: they must be
+  // written by this call, not left in the shared array by an earlier one
+  if ((has_shared != 0) != (n_shared == 1) || n_shared > 1) {
+    ftk::set_step_error("ft_expert_ffn_decode_noalloc: has_shared needs exactly one list entry -1, "
+                        "and no such entry without it");
+    return FT_ERR_INVALID;
   }
   float* scratch = nullptr;
   cudaError_t e = scratch_for_current_device(&scratch);

@@ -24,16 +24,15 @@ def decode_int4(packed: np.ndarray) -> np.ndarray:
 
     READING (the pages name a 4-bit release but no layout): byte b of a row holds
     element 2b in its low nibble and element 2b+1 in its high nibble, each a
-    4-bit two's-complement integer.
+    4-bit two's-complement integer: codes 0..7 stand for themselves, codes 8..15
+    for code - 16.
     """
     p = np.asarray(packed, dtype=np.uint8)
-    lo = (p & 0x0F).astype(np.int64)
-    hi = (p >> 4).astype(np.int64)
-    lo = np.where(lo >= 8, lo - 16, lo)
-    hi = np.where(hi >= 8, hi - 16, hi)
+    code = np.arange(16, dtype=np.int64)
+    value_of_code = np.where(code >= 8, code - 16, code)
     out = np.empty((p.shape[0], p.shape[1] * 2), dtype=np.int64)
-    out[:, 0::2] = lo
-    out[:, 1::2] = hi
+    out[:, 0::2] = value_of_code[p & 0x0F]
+    out[:, 1::2] = value_of_code[p >> 4]
     return out
 
 
@@ -42,7 +41,8 @@ def dequant_int4(packed: np.ndarray, scale_bits: np.ndarray) -> np.ndarray:
     elements of a row (READING: symmetric int4, group 128 along K)."""
     q = decode_int4(packed).astype(np.float64)
     s = widen_bf16(scale_bits)
-    return q * np.repeat(s, 128, axis=1)
+    R = q.shape[0]
+    return (q.reshape(R, -1, 128) * s[:, :, None]).reshape(R, -1)
 
 
 def decode_e2m1(codes: np.ndarray) -> np.ndarray:

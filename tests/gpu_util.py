@@ -78,3 +78,110 @@ def oracle_run(cfg, stack, vals, capacity=None, ffn_steps=None, resize_to=None, 
                         shared_of=(lambda l: stack.shared_blobs[l]) if cfg.shared else None,
                         prefill=cfg.mode == "prefill" if prefill is None else prefill,
                         resize_to=resize_to, ffn_steps=ffn_steps)
+
+
+def run_and_check(cfg, batch, sample_steps, sample_tokens=None, gemm_threshold=None, capacity=None,
+                  resize_at=None, resize_to=None, n_steps=None, stack=None, sample_layers=None,
+                  full_layers=(), workers=None):
+    """Runs a workload through the C ABI (GpuStack) and checks it against the oracle.
+
+    Routing and the cache trace are compared on every step (bit-exact up to near-ties,
+    see first_divergence).  Outputs are compared at the steps in sample_steps: on the
+    tokens sample_tokens (all when None) of the layers sample_layers (all when None),
+    and on every token of the layers in full_layers.  The oracle's per-(step, layer)
+    evaluations run in a thread pool (numpy releases the GIL in its array loops).
+    A shared `stack` starts from an empty cache of `capacity` slots."""
+    import concurrent.futures
+    import contextlib
+    import os
+
+    import torch
+
+    import moe_expert_offload_top_b200 as ft
+    from moe_expert_offload_top_b200.workload import GpuStack
+    from oracle import lru as olru
+
+    ctx = contextlib.nullcontext(stack) if stack is not None else GpuStack(cfg, capacity=capacity)
+    with ctx as st:
+        if stack is not None:
+            ft.ft_moe_set_mode(st.h, cfg.mode == "prefill")
+            ft.ft_cache_resize(st.h, capacity or cfg.C)
+            st.C = capacity or cfg.C
+            ft.ft_cache_clear(st.h)
+            ft.ft_cache_set_trace(st.h, 0)
+            ft.ft_cache_set_trace(st.h, 1)
+            st.reset_stats()
+        if gemm_threshold is not None:
+            ft.ft_moe_set_gemm_threshold(st.h, gemm_threshold)
+        from moe_expert_offload_top_b200.workload import _to_device_tokens
+        vals, bits = synth.tokens(cfg, batch)       # cfg's token process (a shared stack may have another)
+        x = _to_device_tokens(cfg, vals, bits, st.device)
+        steps = n_steps or vals.shape[0]
+        out = torch.empty((cfg.L, batch, cfg.H), dtype=st.xdt, device=st.device)
+        gpu_ids = np.zeros((steps, cfg.L, batch, cfg.k), dtype=np.int32)
+        outs = {}
+        for s in range(steps):
+            if resize_at is not None and s == resize_at:
+                st.resize(resize_to)
+            for l in range(cfg.L):
+                st.forward(l, x[s], out[l])
+                gpu_ids[s, l] = st.last_routing(batch)[0]
+            if s in sample_steps:
+                outs[s] = out.float().cpu().numpy().copy()
+        ft.ft_moe_sync(st.h)
+        trace = st.trace()
+        if stack is not None and trace:
+            # a shared stack keeps counting forward calls across runs (the cache clear keeps
+            # the handle's counters): number this run's calls from 0, as the oracle does
+            base = trace[0][0]
+            trace = [(t[0] - base,) + tuple(t[1:]) for t in trace]
+        stats = st.stats()
+        # oracle: routing and cache trace of every step
+        routers = [synth.router_weights(cfg, l) for l in range(cfg.L)]
+        ref_lru = olru.SharedLru(capacity or cfg.C)
+        ref_ids = np.zeros_like(gpu_ids)
+        gaps = np.zeros((steps, cfg.L, batch))
+        zsel = np.zeros(gpu_ids.shape)
+        for s in range(steps):
+            if resize_at is not None and s == resize_at:
+                ref_lru.resize(resize_to)
+            for l in range(cfg.L):
+                r = moe.route(vals[s], routers[l], cfg.k, cfg.gating)
+                ref_ids[s, l], gaps[s, l] = r["ids"], r["gap"]
+                zsel[s, l] = np.take_along_axis(r["z"], r["ids"].astype(np.int64), axis=1)
+                call = s * cfg.L + l
+                if cfg.mode == "prefill" and l == 0:
+                    ref_lru.access_set(call, 0, range(cfg.E), olru.PREFETCH)
+                ref_lru.access_set(call, l, moe.selected_set(r["ids"]))
+                if cfg.mode == "prefill" and l + 1 < cfg.L:
+                    ref_lru.access_set(call, l + 1, range(cfg.E), olru.PREFETCH)
+        div = first_divergence(gpu_ids, ref_ids, gaps, zsel)
+        want = trace_tuples(ref_lru.trace)
+        if div is None:
+            assert [tuple(t) for t in trace] == want
+        else:
+            last = div // (cfg.L * batch)
+            n = sum(1 for a in ref_lru.trace if a.call < last * cfg.L)
+            assert [tuple(t) for t in trace[:n]] == want[:n]
+        # oracle: outputs of the sampled (step, layer, tokens)
+        jobs = []
+        for s in sample_steps:
+            layers = set(range(cfg.L) if sample_layers is None else sample_layers) | set(full_layers)
+            for l in sorted(layers):
+                if not np.all(same_selection(gpu_ids[s, l], ref_ids[s, l])):
+                    continue      # a near-tie flip (checked above): another valid selection
+                toks = list(range(batch)) if (sample_tokens is None or l in full_layers) else list(sample_tokens)
+                jobs.append((s, l, toks))
+
+        def oracle_out(job):
+            s, l, toks = job
+            r = moe.route(vals[s][toks], routers[l], cfg.k, cfg.gating)
+            return moe.experts_and_combine(vals[s][toks], r["ids"], r["gates"], cfg.E, cfg.wdtype, cfg.H, cfg.I,
+                                           lambda e, l=l: st.pool_blob(l, e),
+                                           st.shared_blobs[l] if cfg.shared else None)
+
+        nw = workers or min(8, os.cpu_count() or 1, max(len(jobs), 1))
+        with concurrent.futures.ThreadPoolExecutor(max_workers=nw) as ex:
+            for (s, l, toks), ref in zip(jobs, ex.map(oracle_out, jobs)):
+                assert_close(outs[s][l][toks], ref, cfg.wdtype, "step %d layer %d (%d tokens)" % (s, l, len(toks)))
+        return {**stats, "compared": [(s, l, len(t)) for s, l, t in jobs]}

@@ -69,6 +69,10 @@ def test_reference_arm_json_line():
         assert key in line, key
     assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "tokens/s"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    # the same config dict as the GPU arm's line, so the two lines describe one workload
+    sys.path.insert(0, ROOT)
+    import bench
+    assert line["config"] == bench.headline_config(1)
     # a rank other than 0 exits at once without a line
     env1 = dict(os.environ, RANK="1", WORLD_SIZE="2")
     out1 = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",

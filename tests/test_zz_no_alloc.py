@@ -2,7 +2,9 @@
 may not allocate device memory (their intermediate rows live in the library's
 static device array).  Checked through the C ABI against the allocating entry
 points (ft_expert_ffn_decode with caller scratch, then ft_combine) on two calls
-in a row, and for its size limit."""
+in a row, for bf16 and int4 weights: both run the same kernels on the same
+inputs, so the outputs must agree bit for bit.  Also checked: its size limit
+and its check of the shared-expert entry."""
 import numpy as np
 import pytest
 import torch
@@ -16,8 +18,8 @@ DEV = "cuda"
 E, K, H, I, T = 16, 8, 2048, 768, 3
 
 
-def _inputs(seed):
-    cfg = synth.MoeConfig("t", 1, E, H, I, K, "sigmoid", "bf16", True, E, T, (T,), "iid", "decode")
+def _inputs(seed, wdtype="bf16"):
+    cfg = synth.MoeConfig("t", 1, E, H, I, K, "sigmoid", wdtype, True, E, T, (T,), "iid", "decode")
     rng = np.random.default_rng(seed)
     ids = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
     gates = rng.random((T, K)).astype(np.float32)
@@ -34,14 +36,14 @@ def _inputs(seed):
     inv = torch.empty(T * K, dtype=torch.int32, device=DEV)
     ft.ft_permute(idd, T, K, E, counts, offs, perm, inv)
     maxp = int(np.bincount(ids.reshape(-1), minlength=E).max())
-    return dict(x=torch.from_numpy(x).view(torch.bfloat16).to(DEV), blobs=blobs, experts=experts,
+    return dict(wdtype=wdtype, x=torch.from_numpy(x).view(torch.bfloat16).to(DEV), blobs=blobs, experts=experts,
                 maxp=maxp, offs=offs, perm=perm, inv=inv, gates=torch.from_numpy(gates).to(DEV))
 
 
 def _with_caller_scratch(a):
     h = torch.empty((T * K + T, I), device=DEV)
     y = torch.empty((T * K + T, H), device=DEV)
-    ft.ft_expert_ffn_decode(a["x"], T, H, I, K, "bf16", a["blobs"], a["experts"], a["maxp"], a["offs"],
+    ft.ft_expert_ffn_decode(a["x"], T, H, I, K, a["wdtype"], a["blobs"], a["experts"], a["maxp"], a["offs"],
                             a["perm"], h, y)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=DEV)
     ft.ft_combine(y, a["gates"], a["inv"], T, H, K, True, True, out)
@@ -50,21 +52,23 @@ def _with_caller_scratch(a):
 
 def _no_alloc(a):
     out = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device=DEV)
-    ft.ft_expert_ffn_decode_noalloc(a["x"], T, H, I, K, "bf16", a["blobs"], a["experts"], a["maxp"], a["offs"],
+    ft.ft_expert_ffn_decode_noalloc(a["x"], T, H, I, K, a["wdtype"], a["blobs"], a["experts"], a["maxp"], a["offs"],
                                     a["perm"], a["gates"], a["inv"], True, out)
     return out
 
 
-def test_no_alloc_entry_matches_the_allocating_path_twice():
-    first, second = _inputs(21), _inputs(22)
+@pytest.mark.parametrize("wdtype", ["bf16", "int4"])
+def test_no_alloc_entry_matches_the_allocating_path_twice(wdtype):
+    first, second = _inputs(21, wdtype), _inputs(22, wdtype)
     for a in (first, second):          # two calls in a row share the static scratch
         got = _no_alloc(a)
         torch.cuda.synchronize()
         ref = _with_caller_scratch(a)
         torch.cuda.synchronize()
-        g, r = got.float().cpu().numpy(), ref.float().cpu().numpy()
-        assert np.all(np.isfinite(g))
-        assert_close(g, r, "bf16", "no-alloc vs caller scratch")
+        assert np.all(np.isfinite(got.float().cpu().numpy()))
+        # the same kernels on the same inputs: identical bits
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16)), "no-alloc output differs from caller scratch"
+        assert_close(got.float().cpu().numpy(), ref.float().cpu().numpy(), wdtype, "no-alloc vs caller scratch")
 
 
 def test_no_alloc_entry_rejects_sizes_beyond_its_scratch():
@@ -76,3 +80,12 @@ def test_no_alloc_entry_rejects_sizes_beyond_its_scratch():
                                         a["offs"], a["perm"], a["gates"], a["inv"], True, out)
     assert ei.value.code == ft.FT_ERR_INVALID
     assert "exceeds the static scratch" in str(ei.value)
+
+
+def test_no_alloc_entry_checks_the_shared_entry():
+    a = _inputs(24)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ft.FtError) as ei:      # has_shared without a -1 entry
+        ft.ft_expert_ffn_decode_noalloc(a["x"], T, H, I, K, "bf16", a["blobs"][:-1], a["experts"][:-1], a["maxp"],
+                                        a["offs"], a["perm"], a["gates"], a["inv"], True, out)
+    assert ei.value.code == ft.FT_ERR_INVALID
