@@ -102,6 +102,10 @@ typedef struct {
  * ------------------------------------------------------------------------ */
 
 /* Creates a stack description with `cache_slots` expert slots of one blob each.
+ * Source: "FreeToken linux", "FreeToken's MoE memory handling" (the routed experts
+ * live in host memory; a fixed share of GPU memory holds expert slots; e.g. 6 of 256
+ * experts per token) and "FreeToken gguf", MoE backends (`offload`: the experts stay
+ * in host memory and a GPU cache holds the hot ones).
  *   num_experts E (1..FT_MAX_EXPERTS), top_k k (1..min(E, FT_MAX_TOPK)),
  *   hidden H and inter I (SwiGLU intermediate): multiples of 8.  For
  *   FT_W_INT4_G128 they must be multiples of 128, for FT_W_NVFP4 of 32.  wdtype is an
@@ -113,7 +117,9 @@ typedef struct {
 FT_API ft_moe* ft_moe_create(int num_experts, int top_k, int hidden, int inter, int wdtype,
                       int cache_slots);
 
-/* Sets the number of layers L, the gating (ft_gating) and whether each layer has one
+/* Source: "FreeToken linux", "FreeToken's MoE memory handling" (one cache shared by
+ * every MoE layer of the model).
+ * Sets the number of layers L, the gating (ft_gating) and whether each layer has one
  * always-on shared expert (gate weight 1).  (Re)allocates the pinned host pool of
  * L*E expert blobs (contents undefined until written) and the resident shared-expert
  * memory (zeroed).  The cache is emptied.  Not allowed while a forward is in flight. */
@@ -122,7 +128,10 @@ FT_API int ft_moe_set_layers(ft_moe* h, int num_layers, int gating, int has_shar
 /* Bytes of one expert blob (the runtime layout below). */
 FT_API size_t ft_moe_blob_bytes(const ft_moe* h);
 
-/* Host address of routed expert (layer, expert) in the library-owned pinned pool,
+/* Source: "FreeToken linux", "FreeToken's MoE memory handling" (the full routed-expert
+ * pool stays in host memory as the reference copy; misses are copied from it) and
+ * "FreeToken linux", setup (the weights are prepared once in the runtime layout).
+ * Host address of routed expert (layer, expert) in the library-owned pinned pool,
  * or NULL for bad indices.  Blobs are contiguous in (layer, expert) order:
  * ft_moe_pool_ptr(h, l, e) = ft_moe_pool_ptr(h, 0, 0) + (l*E + e) * ft_moe_blob_bytes(h).  The caller writes the expert's blob there before the
  * first forward that can read it.  A blob already copied into a slot is not copied
@@ -144,11 +153,16 @@ FT_API size_t ft_moe_blob_bytes(const ft_moe* h);
  *               (e2m1 * e4m3) and applies g to the GEMM accumulators. */
 FT_API void* ft_moe_pool_ptr(ft_moe* h, int layer, int expert);
 
-/* Copies the shared expert of `layer` (a host blob in the same layout) into resident
+/* Source: the stated DeepSeek-V4-Flash-shaped workloads (one always-on shared expert;
+ * the pages name none, so it is kept resident and added with weight 1).
+ * Copies the shared expert of `layer` (a host blob in the same layout) into resident
  * device memory.  Synchronous. */
 FT_API int ft_moe_set_shared(ft_moe* h, int layer, const void* host_blob);
 
-/* Decode (0) or prefill (1) cache policy.  Prefill: a forward of layer 0 first
+/* Source: "FreeToken linux", "FreeToken's MoE memory handling", and "FreeToken RTX
+ * 5090", prefill and decode (whole-layer double buffering during prefill: the next
+ * layer's experts stream in while the current layer computes).
+ * Decode (0) or prefill (1) cache policy.  Prefill: a forward of layer 0 first
  * prefetches every expert of layer 0, and each forward of layer l issues the
  * prefetch of every expert of layer l+1 on the copy stream after its own routed
  * accesses, so the copy overlaps layer l's kernels. */
@@ -159,6 +173,11 @@ FT_API int ft_moe_set_mode(ft_moe* h, int prefill);
 FT_API int ft_moe_reserve(ft_moe* h, int max_tokens);
 
 /* One MoE layer on n_tokens tokens.
+ * Source: "FreeToken linux", "FreeToken's MoE memory handling" (the router picks a few
+ * experts per token; each picked expert runs from the GPU slot that holds it, a missed
+ * one being copied there over PCIe first; the outputs are mixed by the gate weights)
+ * and "FreeToken RTX 5090", dynamic reconfiguration (capacity changes speed, never the
+ * result: every forward computes the dense MoE layer exactly).
  *   x        device [n_tokens][H], float32 for FT_W_F32 stacks, bf16 otherwise.
  *   router_w device [E][H] float32.
  *   out      device [n_tokens][H], same type as x.
@@ -242,7 +261,11 @@ FT_API int ft_debug_device_wait_selftest(int limit_us, void* stream);
  * Either pointer may be NULL. */
 FT_API int ft_moe_last_routing(const ft_moe* h, int* ids, float* gates, int* n_tokens);
 
-/* Changes the number of slots at a safe point: waits for all work of the handle,
+/* Source: "FreeToken RTX 5090", dynamic reconfiguration, and "FreeToken linux", elastic
+ * cache resize (the cache grows or shrinks at a safe point without a restart; a shrink
+ * under memory pressure costs some speed, e.g. -7% from 58% to 40% of the model in the
+ * cache demo of "this tool runs datacenter AI on your PC").
+ * Changes the number of slots at a safe point: waits for all work of the handle,
  * then grows (entries keep slot and recency; new slots are free) or shrinks
  * (least recently used entries are evicted down to the new size; survivors in
  * slots >= slots are moved, most recent first, into the lowest free slots below
@@ -254,11 +277,16 @@ FT_API int ft_cache_resize(ft_moe* h, int slots);
  * free, capacity, counters and trace are kept. */
 FT_API int ft_cache_clear(ft_moe* h);
 
-/* Reads the counters (waits for the copy stream so h2d_seconds is complete). */
+/* Source: "FreeToken linux", performance (the miss rate of expert reads, e.g. 16% for
+ * the shared LRU against 62% for a static split) and "FreeToken's MoE memory handling"
+ * (the runtime measures the pinned-memory transfer bandwidth over PCIe).
+ * Reads the counters (waits for the copy stream so h2d_seconds is complete). */
 FT_API int ft_cache_stats(const ft_moe* h, ft_cache_stats_t* out);
 FT_API int ft_cache_reset_stats(ft_moe* h);
 
-/* Copies up to `cap` trace records, oldest first, into buf and sets *n to the
+/* Source: "FreeToken RTX 5090" (miss rates of the cache policies measured on the same
+ * replayed routing traces).
+ * Copies up to `cap` trace records, oldest first, into buf and sets *n to the
  * number recorded since the trace was last cleared (may exceed cap).  Tracing is
  * on by default; ft_cache_set_trace(h, 0) turns it off and clears it. */
 FT_API int ft_cache_trace(const ft_moe* h, ft_access_t* buf, int cap, int* n);
@@ -314,11 +342,13 @@ FT_API int ft_moe_reset_perf(ft_moe* h);
 /* Deadline of every host wait on the GPU, in milliseconds (default 20000). */
 FT_API int ft_moe_set_timeout_ms(ft_moe* h, int ms);
 
-/* Message of the last failed call on h, or of the last failed ft_moe_create when
+/* The pages give no error reporting; this is the plainest completion of their API.
+ * Message of the last failed call on h, or of the last failed ft_moe_create when
  * h is NULL (per host thread). */
 FT_API const char* ft_last_error(const ft_moe* h);
 
-/* Waits for the handle's work and frees everything it owns. */
+/* The pages give no teardown; this is the plainest completion of their API.
+ * Waits for the handle's work and frees everything it owns. */
 FT_API void ft_moe_destroy(ft_moe* h);
 
 /* Host-only replay of the cache policy (no GPU, no allocation on the device): runs the

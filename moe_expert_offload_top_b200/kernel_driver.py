@@ -1,0 +1,54 @@
+"""Runs a named workload at reduced size through the C ABI, for kernel profiling.
+
+    python -m moe_expert_offload_top_b200.kernel_driver --workload NAME
+        [--layers L] [--experts E] [--slots C] [--steps S] [--batch B] [--tokens T]
+
+The workload keeps its shapes (hidden, intermediate, top-k, gating, weight format,
+shared expert) and token process; --layers / --experts shrink the pool so that a
+profiler's capture stays small (a few GB on the device), and --slots defaults to every
+expert resident, so the launches are the kernels alone.  Decode workloads run S steps of
+B tokens; prefill workloads run S forwards of T tokens through every layer.  Prints one
+line with the steps run and the cache counters.
+"""
+import argparse
+import dataclasses
+import json
+import sys
+
+import torch
+
+import synth
+from moe_expert_offload_top_b200.workload import GpuStack
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--workload", required=True, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--layers", type=int, default=1)
+    ap.add_argument("--experts", type=int, default=None)
+    ap.add_argument("--slots", type=int, default=None, help="cache slots (default: every expert resident)")
+    ap.add_argument("--steps", type=int, default=12)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--tokens", type=int, default=None, help="prefill: tokens per forward")
+    a = ap.parse_args(argv)
+    base = synth.CONFIGS[a.workload]
+    E = a.experts or base.E
+    k = min(base.k, E)
+    prefill = base.mode == "prefill"
+    T = (a.tokens or base.tokens) if prefill else a.batch
+    n_tok = T * a.steps if prefill else max(base.tokens, T * a.steps)
+    cfg = dataclasses.replace(base, L=a.layers, E=E, k=k, C=a.slots or a.layers * E, tokens=n_tok,
+                              batches=(T,), resize_to=None)
+    with GpuStack(cfg, max_tokens=T) as st:
+        vals, x = st.tokens(T)
+        out = torch.empty((cfg.L, T, cfg.H), dtype=st.xdt, device=st.device)
+        for s in range(a.steps):
+            st.step(x[s % x.shape[0]], out)
+        torch.cuda.synchronize()
+        print(json.dumps({"workload": cfg.name, "layers": cfg.L, "experts": cfg.E, "slots": cfg.C, "steps": a.steps,
+                          "tokens_per_step": T, "cache": st.stats()}))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
