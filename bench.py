@@ -27,9 +27,10 @@ The one JSON line (rank 0) carries:
   - legs (N = 1 only): "int4-large-pool" decode at batch 1 (16 layers, H=7168, int4
     g128, 15% cached); "prefill" of the headline shapes (4096 tokens through the 8
     layers with whole-layer double buffering over PCIe, the same with every expert
-    resident, and a tensor-pipe sweep of one resident layer at 16k/32k/64k tokens);
-    "shrink": decode tokens/s before and after shrinking the cache from 58% to 40% of
-    the experts ("this tool runs datacenter AI on your PC", the cache shrink demo).
+    resident, a tensor-pipe sweep of one resident layer at 16k/32k/64k tokens, and one
+    layer with NVFP4 weights, every expert resident); "shrink": decode
+    tokens/s before and after shrinking the cache from 58% to 40% of the experts ("this
+    tool runs datacenter AI on your PC", the cache shrink demo).
 --impl reference times the CPU oracle alone on the headline workload.
 N > 1 runs independent replicas (one stack per GPU, its own token chain, the
 headline legs only): the path has no exchange step.
@@ -569,6 +570,9 @@ def prefill_leg(args, stack, dev, peaks, peak_src):
                            "peak_source": peak_src + " bf16_tflops_sustained (cuBLAS bf16, seconds-long loop)",
                            "kernel": top["kernel"], "at_tokens": max(sweep, key=lambda s: s["grouped_gemm"]["tflops"]
                                                                       or 0)["tokens"]}
+    if args.nvfp4:
+        res["nvfp4_resident"] = nvfp4_prefill(args, dev, peaks, x_dev[:T], res["resident"]["ms_per_layer"],
+                                              gemm_figures)
     if not args.no_cpu_baseline:
         # the oracle on the first layer of the prompt (every expert of the layer is read)
         from oracle import moe
@@ -583,6 +587,53 @@ def prefill_leg(args, stack, dev, peaks, peak_src):
                                                            "numpy oracle, %.1f s), scaled to the whole stack"
                                                            % (T, cfg.L, cdt)}
     return res
+
+
+def nvfp4_prefill(args, dev, peaks, x, bf16_ms_per_layer, gemm_figures):
+    """The prefill shapes with NVFP4 expert weights (e2m1 codes, an e4m3 scale per 16
+    elements, an fp32 scale per matrix; "FreeToken linux", performance: the NVFP4 4-bit
+    release), every expert resident: the GEMMs expand each weight tile to bf16 in shared
+    memory.  One layer (its 256 experts: generating NVFP4 blobs is slow on the host)."""
+    import dataclasses
+
+    import torch
+
+    import moe_expert_offload_top_b200 as ft
+    from moe_expert_offload_top_b200.workload import GpuStack
+    base = synth.CONFIGS[PREFILL]
+    cfg = dataclasses.replace(base, name="dsv4flash-prefill-nvfp4", wdtype="nvfp4", L=1, C=base.E)
+    T = x.shape[0]
+    t0 = time.perf_counter()
+    stack = GpuStack(cfg, device=dev, max_tokens=T)
+    setup_s = time.perf_counter() - t0
+    stream = torch.cuda.current_stream(dev)
+    out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
+    try:
+        stack.forward(0, x, out, stream)              # warm-up (and the one-time prefetch of layer 0)
+        ft.ft_moe_sync(stack.h)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.prefill_passes):
+            stack.forward(0, x, out, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        dt = e0.elapsed_time(e1) * 1e-3 / args.prefill_passes
+        ft.ft_moe_reset_perf(stack.h)
+        ft.ft_moe_set_stage_timing(stack.h, 1)
+        stack.forward(0, x, out, stream)
+        torch.cuda.synchronize(dev)
+        perf = ft.ft_moe_perf(stack.h)
+        ft.ft_moe_set_stage_timing(stack.h, 0)
+    finally:
+        stack.close()
+    return {"workload": "%s: 1 layer, E=%d, H=%d, I=%d, top-%d %s + shared expert, NVFP4 weights, %d N(0,1) "
+                        "tokens, prefill, every expert resident" % (cfg.name, cfg.E, cfg.H, cfg.I, cfg.k, cfg.gating, T),
+            "ms_per_layer": 1e3 * dt, "tokens_per_s_per_layer": T / dt,
+            "vs_bf16_resident_ms_per_layer": 1e3 * dt / bf16_ms_per_layer,
+            "grouped_gemm": dict(gemm_figures(perf), kernel="grouped_gemm_kernel<0,1>+<1,1> (NVFP4 tiles expanded "
+                                                           "to bf16 in shared memory, tcgen05 kind::f16)"),
+            "stages_ms_per_layer": {k2: v / 1e3 for k2, v in stage_us(perf).items()}, "pool_setup_s": setup_s}
 
 
 # -------------------------------------------------------------- shrink leg --
@@ -714,6 +765,7 @@ def main(argv=None):
     ap.add_argument("--shrink-steps", type=int, default=256)
     ap.add_argument("--prefill-passes", type=int, default=2)
     ap.add_argument("--no-sweep", dest="sweep", action="store_false", help="skip the prefill token sweep")
+    ap.add_argument("--no-nvfp4", dest="nvfp4", action="store_false", help="skip the NVFP4 prefill layer")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
     ap.add_argument("--reference-budget-s", type=float, default=90.0)
     ap.add_argument("--reference-max-tokens", type=int, default=12)

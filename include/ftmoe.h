@@ -149,8 +149,9 @@ FT_API size_t ft_moe_blob_bytes(const ft_moe* h);
  *               byte per 16 consecutive K elements), then the fp32 global scales g_gate,
  *               g_up, g_down and 4 zero bytes.  w = e2m1(q) * e4m3(s) * g.  H and I must
  *               be multiples of 32.  Decode runs the streaming GEMV on these codes;
- *               prefill (the GEMM path) expands the selected experts exactly to bf16
- *               (e2m1 * e4m3) and applies g to the GEMM accumulators. */
+ *               prefill (the GEMM path) expands each weight tile exactly to bf16
+ *               (e2m1 * e4m3) in shared memory inside the GEMM and applies g to its
+ *               accumulators. */
 FT_API void* ft_moe_pool_ptr(ft_moe* h, int layer, int expert);
 
 /* Source: the stated DeepSeek-V4-Flash-shaped workloads (one always-on shared expert;
@@ -204,13 +205,13 @@ FT_API int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, con
 
 /* Waits for every forward and copy of the handle, then checks the device error word
  * that a kernel sets when one of its bounded waits gives up (FT_ERR_DEVICE_CHECK; the
- * word is cleared): codes 101-104 the prefill GEMM's pipeline waits, 111 the fused
+ * word is cleared): codes 101-106 the prefill GEMM's pipeline waits, 111 the fused
  * decode FFN's wait for an expert's gate/up rows.  A forward also reports a word set
  * by an earlier forward. */
 FT_API int ft_moe_sync(ft_moe* h);
 
-/* Expert FFN path: bf16 and nvfp4 stacks with H % 256 == 0 and I % 128 == 0 use the
- * tcgen05 grouped GEMMs when n_tokens * k >= min_avg_pairs * |S| (on average at least
+/* Expert FFN path: bf16 stacks with H % 256 == 0 and I % 128 == 0, and nvfp4 stacks with
+ * H % 256 == 0 and I % 256 == 0, use the tcgen05 grouped GEMMs when n_tokens * k >= min_avg_pairs * |S| (on average at least
  * min_avg_pairs tokens per selected expert; default 32), else the streaming GEMV.
  * Both compute the same function.  0 always selects the GEMMs where shapes allow. */
 FT_API int ft_moe_set_gemm_threshold(ft_moe* h, int min_avg_pairs);

@@ -114,10 +114,7 @@ struct ft_moe {
   ftk::GemmMaps maps;
   bool maps_dirty = true;
   // NVFP4 prefill: the selected experts expanded to bf16 for the tcgen05 GEMMs
-  uint8_t* stage = nullptr;       // stage_cap bf16 expert blobs (3*H*I*2 bytes each)
-  int stage_cap = 0;
-  float* d_stage_gs = nullptr;    // 3 fp32 matrix scales per stage slot
-  ftk::GemmMaps smaps;            // a_x, a_h as maps; B maps over the stage
+  ftk::GemmFp4 fp4 = {};          // NVFP4 stacks: maps over the slots' codes and block scales
   int num_sms = 148;
   int gemm_min_avg_pairs = 32;    // tcgen05 path when bf16 and T*k/|S| >= this
   int fused_routing = 1;          // one-launch routing for decode-sized calls
@@ -374,28 +371,10 @@ int issue_fills(ft_moe* h, std::vector<ftc::Access>& recs, size_t first) {
 }
 
 bool gemm_shapes_ok(const ft_moe* h) {
-  return (h->wdtype == FT_W_BF16 || h->wdtype == FT_W_NVFP4) && h->H % 256 == 0 && h->I % 128 == 0;
-}
-
-// Room for n bf16 expert blobs in the NVFP4 staging arena (grows only).
-int ensure_stage(ft_moe* h, int n) {
-  if (n <= h->stage_cap) return FT_OK;
-  if (h->has_last_stream) FT_CUDA(h, cudaStreamSynchronize(h->last_stream));
-  cudaFree(h->stage);
-  cudaFree(h->d_stage_gs);
-  h->stage = nullptr;
-  h->d_stage_gs = nullptr;
-  h->stage_cap = 0;
-  const size_t bytes = (size_t)n * 3 * h->H * h->I * 2;
-  if (cudaMalloc(&h->stage, bytes) != cudaSuccess || cudaMalloc(&h->d_stage_gs, sizeof(float) * 3 * n) != cudaSuccess) {
-    cudaGetLastError();
-    cudaFree(h->stage);
-    h->stage = nullptr;
-    return fail(h, FT_ERR_OOM, "NVFP4 staging arena allocation failed");
-  }
-  h->stage_cap = n;
-  h->maps_dirty = true;
-  return FT_OK;
+  // bf16: 256-column tiles of the outputs, 64-element K blocks; NVFP4 also reads its block
+  // scales in 16-byte boxes (256 elements of K per row), so I must be a multiple of 256 too
+  return (h->wdtype == FT_W_BF16 && h->H % 256 == 0 && h->I % 128 == 0) ||
+         (h->wdtype == FT_W_NVFP4 && h->H % 256 == 0 && h->I % 256 == 0);
 }
 
 int ensure_maps(ft_moe* h) {
@@ -404,25 +383,37 @@ int ensure_maps(ft_moe* h) {
   const uint64_t H = h->H, I = h->I;
   bool ok = ftk::encode_map_2d(&h->maps.a_x, h->d_ax, H, rows, H * 2, 128) &&
             ftk::encode_map_2d(&h->maps.a_h, h->d_h, I, rows, I * 2, 128);
-  // slot maps only where the slots hold bf16 blobs (NVFP4 stacks use the staged copies)
-  if (ok && h->wdtype == FT_W_BF16)
+  if (ok && h->wdtype == FT_W_BF16) {
     ok = ftk::encode_map_3d(&h->maps.b1_routed, h->arena, H, 2 * I, h->C, H * 2, h->blob, 128) &&
          ftk::encode_map_3d(&h->maps.b2_routed, h->arena + 2 * I * H * 2, I, H, h->C, I * 2, h->blob, 256);
-  if (ok && h->shared && h->wdtype == FT_W_BF16) {
-    ok = ftk::encode_map_3d(&h->maps.b1_shared, h->shared, H, 2 * I, h->L, H * 2, h->blob, 128) &&
-         ftk::encode_map_3d(&h->maps.b2_shared, h->shared + 2 * I * H * 2, I, H, h->L, I * 2, h->blob, 256);
-  } else {
-    h->maps.b1_shared = h->maps.b1_routed;
-    h->maps.b2_shared = h->maps.b2_routed;
+    if (ok && h->shared) {
+      ok = ftk::encode_map_3d(&h->maps.b1_shared, h->shared, H, 2 * I, h->L, H * 2, h->blob, 128) &&
+           ftk::encode_map_3d(&h->maps.b2_shared, h->shared + 2 * I * H * 2, I, H, h->L, I * 2, h->blob, 256);
+    } else {
+      h->maps.b1_shared = h->maps.b1_routed;
+      h->maps.b2_shared = h->maps.b2_routed;
+    }
   }
-  if (ok && h->stage) {   // staged NVFP4 experts: routed and shared alike, slot z = list index
-    const uint64_t sblob = 3 * H * I * 2;
-    h->smaps.a_x = h->maps.a_x;
-    h->smaps.a_h = h->maps.a_h;
-    ok = ftk::encode_map_3d(&h->smaps.b1_routed, h->stage, H, 2 * I, h->stage_cap, H * 2, sblob, 128) &&
-         ftk::encode_map_3d(&h->smaps.b2_routed, h->stage + 2 * I * H * 2, I, H, h->stage_cap, I * 2, sblob, 256);
-    h->smaps.b1_shared = h->smaps.b1_routed;
-    h->smaps.b2_shared = h->smaps.b2_routed;
+  if (ok && h->wdtype == FT_W_NVFP4) {
+    // blob: codes Q_gate|Q_up [2I][H/2], Q_down [H][I/2]; block scales S_gate|S_up [2I][H/16],
+    // S_down [H][I/16]; then the three fp32 matrix scales
+    const uint64_t mat = H * I, q2 = mat, s1 = 3 * mat / 2, s2 = s1 + mat / 8;
+    auto maps_over = [&](const uint8_t* b, uint64_t depth, CUtensorMap* q, CUtensorMap* sc) {
+      return ftk::encode_map_u8_3d(&q[0], b, H / 2, 2 * I, depth, H / 2, h->blob, 32, 128) &&
+             ftk::encode_map_u8_3d(&q[1], b + q2, I / 2, H, depth, I / 2, h->blob, 32, 128) &&
+             ftk::encode_map_u8_3d(&sc[0], b + s1, H / 16, 2 * I, depth, H / 16, h->blob, 16, 128) &&
+             ftk::encode_map_u8_3d(&sc[1], b + s2, I / 16, H, depth, I / 16, h->blob, 16, 128);
+    };
+    ok = maps_over(h->arena, h->C, h->fp4.q_routed, h->fp4.s_routed);
+    if (ok && h->shared) {
+      ok = maps_over(h->shared, h->L, h->fp4.q_shared, h->fp4.s_shared);
+    } else {
+      for (int i = 0; i < 2; ++i) { h->fp4.q_shared[i] = h->fp4.q_routed[i]; h->fp4.s_shared[i] = h->fp4.s_routed[i]; }
+    }
+    h->fp4.g_routed = h->arena;
+    h->fp4.g_shared = h->shared ? h->shared : h->arena;
+    h->fp4.blob = h->blob;
+    h->fp4.g_off = 3 * mat / 2 + 3 * mat / 16;
   }
   if (!ok) return fail(h, FT_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   h->maps_dirty = false;
@@ -903,36 +894,27 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
         rc = wait_fills();
         if (rc) return bail(rc, h->err);
       }
-      const bool staged = h->wdtype == FT_W_NVFP4;   // expanded to bf16 for the tensor cores
-      if (staged) {
-        rc = ensure_stage(h, list.n);
-        if (rc) return bail(rc, h->err);
-      }
+      // NVFP4 slots are expanded to bf16 inside the GEMMs (exact), bf16 slots read as they are
+      const ftk::GemmFp4* fp4 = h->wdtype == FT_W_NVFP4 ? &h->fp4 : nullptr;
       rc = ensure_maps(h);
       if (rc) return bail(rc, h->err);
       ftk::GemmGroups groups;
       groups.n = list.n;
       for (int i = 0; i < list.n; ++i) {
         groups.expert[i] = list.expert[i];
-        groups.z[i] = staged ? i : list.expert[i] >= 0 ? h->lru.slot_of(layer * E + list.expert[i]) : layer;
+        groups.z[i] = list.expert[i] >= 0 ? h->lru.slot_of(layer * E + list.expert[i]) : layer;
       }
-      if (staged) {
-        FT_CUDA_B(ftk::launch_dequant_nvfp4_stage(list, h->H, h->I, h->stage, h->d_stage_gs, h->num_sms, s));
-        h->perf.kernel_launches += 1;
-      }
-      const ftk::GemmMaps& gm = staged ? h->smaps : h->maps;
-      const float* gsc = staged ? h->d_stage_gs : nullptr;
       FT_CUDA_B(ftk::launch_gather_rows(x, h->d_perm, T, k, h->H, h->has_shared != 0, h->d_ax, s));
       h->perf.kernel_launches += 1;
       stage_mark(se, SE_G0, s);
-      FT_CUDA_B(ftk::launch_grouped_gemm(0, gm, groups, h->d_offsets, T, k, h->I, h->H, h->d_h,
-                                          h->d_err, h->num_sms, s, gsc));
+      FT_CUDA_B(ftk::launch_grouped_gemm(0, h->maps, groups, h->d_offsets, T, k, h->I, h->H, h->d_h,
+                                          h->d_err, h->num_sms, s, fp4));
       stage_mark(se, SE_G1, s);
-      FT_CUDA_B(ftk::launch_grouped_gemm(1, gm, groups, h->d_offsets, T, k, h->I, h->H, h->d_y,
-                                          h->d_err, h->num_sms, s, gsc));
-      if (se) {   // bf16 h, and the weights of each listed expert read once
-        se->gu_bytes = list.n * 2.0 * h->H * h->I * 2 + pairs * (h->H * 2.0 + h->I * 2.0);
-        se->d_bytes = list.n * 1.0 * h->H * h->I * 2 + pairs * (h->I * 2.0 + h->H * 4.0);
+      FT_CUDA_B(ftk::launch_grouped_gemm(1, h->maps, groups, h->d_offsets, T, k, h->I, h->H, h->d_y,
+                                          h->d_err, h->num_sms, s, fp4));
+      if (se) {   // bf16 h, and the weights of each listed expert read once (in their stored format)
+        se->gu_bytes = list.n * 2.0 * wmat + pairs * (h->H * 2.0 + h->I * 2.0);
+        se->d_bytes = list.n * wmat + pairs * (h->I * 2.0 + h->H * 4.0);
       }
     } else if (split) {
       // gate/up | G1 | down of the ready group, the wait, then gate/up | G3 | down of the rest
@@ -1210,8 +1192,6 @@ void ft_moe_destroy(ft_moe* h) {
   cudaFree(h->d_err);
   cudaFree(h->d_ticket);
   cudaFree(h->d_ctl);
-  cudaFree(h->stage);
-  cudaFree(h->d_stage_gs);
   if (h->h_err) cudaFreeHost(h->h_err);
   if (h->h_hold) cudaFreeHost(h->h_hold);
   if (h->copy) cudaStreamDestroy(h->copy);

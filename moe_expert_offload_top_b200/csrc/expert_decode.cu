@@ -120,7 +120,7 @@ cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdt
   (void)err;
   if (list.n <= 0 || T <= 0) return cudaSuccess;
   if (wdtype == WT_INT4 && int4_tensor)
-    return launch_ffn_int4_mma(x, T, H, I, k, list, offsets, perm, h, y, s, between);
+    return launch_ffn_int4_mma(x, T, H, I, k, list, offsets, perm, h, y, s, between, max_pairs_per_expert);
   int nt = max_pairs_per_expert < T ? max_pairs_per_expert : T;
   if (nt < 1) nt = 1;
   auto bytes_of = [&](int K) -> size_t {

@@ -7,15 +7,24 @@
 // (stated workloads): h = silu(A W_gate^T) * (A W_up^T) in bf16, y = h W_down^T
 // in fp32, with A the expert's gathered token rows.
 //
-// One persistent kernel per GEMM, one CTA per SM, 192 threads:
-//   warp 0  TMA producer: A tile [128 x 64] and B tile [256 x 64] bf16 per
-//           stage, 128-byte swizzle, 4 stages (no multicast: every CTA loads
-//           its own tiles from this GPU's memory).
+// One persistent kernel per GEMM, one CTA per SM:
+//   warp 0  TMA producer: A tile [128 x 64] bf16 and the B tile per stage, no
+//           multicast (every CTA loads its own tiles from this GPU's memory).
+//           bf16 weights: B [256 x 64] bf16 with 128-byte swizzle, 4 stages.
+//           NVFP4 weights: the B tile's packed e2m1 codes [256 x 32 bytes] and,
+//           every fourth stage, its e4m3 block scales for the next 256 columns
+//           [256 x 16 bytes], 3 stages.
 //   warp 1  MMA issuer: tcgen05.mma.cta_group::1.kind::f16, M=128, N=256,
 //           K=16, fp32 accumulators in TMEM, two accumulator buffers of 256
 //           columns so the epilogue of one tile overlaps the next tile's MMAs.
 //   warps 2-5  epilogue: tcgen05.ld 32x32b rows of the accumulator, SwiGLU
 //           (gate/up) or plain (down), masked row stores to global memory.
+//   warps 6-9  (NVFP4 only) expansion: each stage's codes times their block scales
+//           become the bf16 B tile, written in the 128-byte-swizzled layout the MMA
+//           reads, then handed to the MMA warp through the async proxy.  An e2m1
+//           value (2 significant bits) times an e4m3 scale (4) has at most 6
+//           significant bits and lies in bf16's range, so the operand is exact; the
+//           fp32 scale of each matrix multiplies the accumulator in the epilogue.
 // Tiles: per group (a selected expert or the shared expert) ceil(rows/128)
 // M-tiles times the N-tiles of the output, N-major inside a group so that the
 // M-tiles sharing one weight tile run back to back.  An M-tile may read rows
@@ -25,6 +34,7 @@
 // code in *err, sets the CTA's abort flag, and all roles drain and leave; the
 // TMEM columns are always released.
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "kernels.hpp"
@@ -35,15 +45,24 @@ namespace ftk {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;      // 16 KB
 constexpr int B_BYTES = BN * BK * 2;      // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int GEMM_THREADS = 192;
 constexpr int TMEM_COLS = 512;            // two 128 x 256 fp32 accumulators
+constexpr int MAX_STAGES = 4;
+
+// Per weight format: pipeline stages, threads, and the raw bytes of a B tile's codes.
+template <int WT> struct GemmCfg;
+template <> struct GemmCfg<GW_BF16> {
+  static constexpr int STAGES = 4, THREADS = 192, RAW = 0, SCALE_RING = 0;
+};
+template <> struct GemmCfg<GW_NVFP4> {
+  static constexpr int STAGES = 3, THREADS = 320, RAW = BN * BK / 2;   // 8 KB of e2m1 codes
+  static constexpr int SCALE_RING = 2 * BN * 16;                       // two blocks of 4 stages' scales
+};
+template <int WT> constexpr int stage_bytes() { return A_BYTES + B_BYTES + GemmCfg<WT>::RAW; }
 
 struct GemmSmem {
-  uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2];
+  uint64_t full[MAX_STAGES], empty[MAX_STAGES], conv[MAX_STAGES], tfull[2], tempty[2];
   uint32_t tmem_base;
   int abort;
   int mt_start[kMaxList + 1];   // prefix of M-tiles over groups
@@ -111,17 +130,36 @@ FT_DEVICE void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Two e2m1 codes of `byte`, times the f16 pair `sp` (a block scale in both halves), as one
+// bf16 pair: the e2m1 pair converts exactly to f16, the product is exact in f16 (at most
+// 6 significant bits, magnitudes 2^-10 .. 2688), and each f16 converts exactly to bf16.
+FT_DEVICE uint32_t e2m1x2_times(uint32_t byte, uint32_t sp) {
+  uint32_t h2, p2, o;
+  asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h2) : "r"(byte));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p2) : "r"(h2), "r"(sp));
+  const float lo = __half2float(__ushort_as_half((unsigned short)(p2 & 0xFFFFu)));
+  const float hi = __half2float(__ushort_as_half((unsigned short)(p2 >> 16)));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o) : "f"(hi), "f"(lo));
+  return o;
+}
+
 // MODE 0: gate/up + SwiGLU (B = [W_gate rows n0..n0+127 ; W_up rows n0..n0+127], out = h bf16 [rows][I])
 // MODE 1: down (B = W_down rows n0..n0+255, out = y f32 [rows][H])
-template <int MODE>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+// WT: GW_BF16 (B read as bf16 through tmBr / tmBs) or GW_NVFP4 (codes and scales through
+// fp4's maps, expanded in shared memory; tmBr / tmBs unused).
+template <int MODE, int WT>
+__global__ void __launch_bounds__(GemmCfg<WT>::THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmBr,
                     const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ GemmGroups groups,
-                    const int* __restrict__ offsets, int T, int k, int I, int H,
-                    void* __restrict__ out, int* __restrict__ err, const float* __restrict__ gscale) {
+                    const __grid_constant__ GemmFp4 fp4, const int* __restrict__ offsets, int T, int k, int I,
+                    int H, void* __restrict__ out, int* __restrict__ err) {
+  constexpr int STAGES = GemmCfg<WT>::STAGES;
+  constexpr int STAGE_BYTES = stage_bytes<WT>();
+  constexpr bool FP4 = WT == GW_NVFP4;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  GemmSmem* S = reinterpret_cast<GemmSmem*>(base + STAGES * STAGE_BYTES);
+  unsigned char* scale_ring = base + STAGES * STAGE_BYTES;   // NVFP4: [2][BN rows][16 bytes]
+  GemmSmem* S = reinterpret_cast<GemmSmem*>(scale_ring + GemmCfg<WT>::SCALE_RING);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = MODE == 0 ? H : I;
   const int KB = K / BK;
@@ -129,7 +167,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   const int ld_out = MODE == 0 ? I : H;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(&S->full[s], 1); mbar_init(&S->empty[s], 1); }
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&S->full[s], 1);
+      mbar_init(&S->empty[s], 1);
+      mbar_init(&S->conv[s], 128);
+    }
     for (int b = 0; b < 2; ++b) { mbar_init(&S->tfull[b], 1); mbar_init(&S->tempty[b], 128); }
     S->abort = 0;
     int acc = 0;
@@ -174,29 +216,51 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
   if (warp == 0) {
     if (lane == 0) {   // ---------------------------------------------- TMA producer
-      int it = 0;
+      int it = 0, sblk = 0;
       for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
         int g, m, n;
         decode(t, g, m, n);
         const int row0 = S->row_start[g] + m * BM;
         const bool sh = groups.expert[g] < 0;
-        const CUtensorMap* mb = sh ? &tmBs : &tmBr;
         const int z = groups.z[g];
+        // B rows of the tile: gate rows n*128.. and up rows I + n*128.., or down rows n*256..
+        const int br0 = MODE == 0 ? n * (BN / 2) : n * BN;
+        const int br1 = MODE == 0 ? I + n * (BN / 2) : n * BN + BN / 2;
+        bool stop = false;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t par = ((it / STAGES) & 1) ^ 1;
-          if (!mbar_wait(&S->empty[s], par, abort_flag, err, 101)) break;
+          if (!mbar_wait(&S->empty[s], par, abort_flag, err, 101)) { stop = true; break; }
           unsigned char* sa = base + s * STAGE_BYTES;
           unsigned char* sb = sa + A_BYTES;
-          mbar_expect_tx(&S->full[s], STAGE_BYTES);
-          tma_load_2d(sa, &tmA, &S->full[s], kb * BK, row0);
-          if (MODE == 0) {
-            tma_load_3d(sb, mb, &S->full[s], kb * BK, n * (BN / 2), z);
-            tma_load_3d(sb + B_BYTES / 2, mb, &S->full[s], kb * BK, I + n * (BN / 2), z);
+          if constexpr (!FP4) {
+            const CUtensorMap* mb = sh ? &tmBs : &tmBr;
+            mbar_expect_tx(&S->full[s], A_BYTES + B_BYTES);
+            tma_load_2d(sa, &tmA, &S->full[s], kb * BK, row0);
+            if (MODE == 0) {   // boxes of 128 rows: gate rows, then up rows
+              tma_load_3d(sb, mb, &S->full[s], kb * BK, br0, z);
+              tma_load_3d(sb + B_BYTES / 2, mb, &S->full[s], kb * BK, br1, z);
+            } else {           // one box of 256 down rows
+              tma_load_3d(sb, mb, &S->full[s], kb * BK, br0, z);
+            }
           } else {
-            tma_load_3d(sb, mb, &S->full[s], kb * BK, n * BN, z);
+            const CUtensorMap* mq = sh ? &fp4.q_shared[MODE] : &fp4.q_routed[MODE];
+            const CUtensorMap* ms = sh ? &fp4.s_shared[MODE] : &fp4.s_routed[MODE];
+            unsigned char* raw = sb + B_BYTES;
+            const bool scales = (kb & 3) == 0;   // a new block of 4 stages' block scales
+            mbar_expect_tx(&S->full[s], A_BYTES + GemmCfg<WT>::RAW + (scales ? BN * 16 : 0));
+            tma_load_2d(sa, &tmA, &S->full[s], kb * BK, row0);
+            tma_load_3d(raw, mq, &S->full[s], kb * (BK / 2), br0, z);
+            tma_load_3d(raw + GemmCfg<WT>::RAW / 2, mq, &S->full[s], kb * (BK / 2), br1, z);
+            if (scales) {
+              unsigned char* sdst = scale_ring + (sblk & 1) * (BN * 16);
+              tma_load_3d(sdst, ms, &S->full[s], (kb / 4) * 16, br0, z);
+              tma_load_3d(sdst + BN / 2 * 16, ms, &S->full[s], (kb / 4) * 16, br1, z);
+              ++sblk;
+            }
           }
         }
+        if (stop) break;
       }
       // drain: wait (bounded) until every issued stage has landed
       const int issued = it;
@@ -217,6 +281,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(&S->full[s], (it / STAGES) & 1, abort_flag, err, 103)) { ok = false; break; }
+          if (FP4 && !mbar_wait(&S->conv[s], (it / STAGES) & 1, abort_flag, err, 106)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(base + s * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
@@ -229,7 +294,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         mma_commit(&S->tfull[b]);
       }
     }
-  } else {             // ---------------------------------------------- epilogue (warps 2..5)
+  } else if (warp < 6) {   // ------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;                   // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;              // tile row of this thread
     int tl = 0;
@@ -242,8 +307,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const int valid = S->rows[g] - m * BM;
       const int row = S->row_start[g] + m * BM + r;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + b * BN;
-      // per-matrix fp32 scales of staged NVFP4 weights (gate, up, down of stage slot z)
-      const float* gs = gscale ? gscale + 3 * groups.z[g] : nullptr;
+      // NVFP4: the fp32 scales of gate, up and down, stored in the expert's blob
+      float sg = 1.f, su = 1.f, sd = 1.f;
+      if constexpr (FP4) {
+        const uint8_t* gb = (groups.expert[g] < 0 ? fp4.g_shared : fp4.g_routed) +
+                            (size_t)groups.z[g] * fp4.blob + fp4.g_off;
+        const float* gl = reinterpret_cast<const float*>(gb);
+        sg = gl[0]; su = gl[1]; sd = gl[2];
+      }
       if (MODE == 0) {
         uint16_t* hout = static_cast<uint16_t*>(out) + (size_t)row * ld_out + n * (BN / 2);
 #pragma unroll 1
@@ -251,8 +322,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           float u[32], v[32];
           tmem_ld32(tbase + j, u);
           tmem_ld32(tbase + BN / 2 + j, v);
-          if (gs) {
-            const float sg = gs[0], su = gs[1];
+          if constexpr (FP4) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) { u[i] *= sg; v[i] *= su; }
           }
@@ -274,8 +344,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         for (int j = 0; j < BN; j += 32) {
           float v[32];
           tmem_ld32(tbase + j, v);
-          if (gs) {
-            const float sd = gs[2];
+          if constexpr (FP4) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] *= sd;
           }
@@ -288,6 +357,49 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       }
       tc_fence_before();
       mbar_arrive(&S->tempty[b]);
+    }
+  } else if constexpr (FP4) {   // ---------------------------------- expansion (warps 6..9)
+    // 512 items per stage: B row rr (0..255) and half hf (K elements 32 hf .. 32 hf + 31 of
+    // the stage): 16 bytes of codes -> 64 bytes (four 16-byte chunks) of bf16, chunk c of
+    // row rr stored at rr * 128 + ((c ^ (rr & 7)) * 16) (the 128-byte swizzle); a thread
+    // takes items ct, ct + 128, ct + 256, ct + 384.
+    const int ct = threadIdx.x - 192;
+    int it = 0, sblk = 0;
+    for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
+      bool stop = false;
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = it % STAGES;
+        if (!mbar_wait(&S->full[s], (it / STAGES) & 1, abort_flag, err, 105)) { stop = true; break; }
+        if ((kb & 3) == 0) ++sblk;
+        const unsigned char* sblock = scale_ring + ((sblk - 1) & 1) * (BN * 16) + (kb & 3) * 4;
+        unsigned char* sb = base + s * STAGE_BYTES + A_BYTES;
+        const unsigned char* raw = sb + B_BYTES;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int item = ct + 128 * i;
+          const int rr = item >> 1, hf = item & 1;
+          const uint4 qv = *reinterpret_cast<const uint4*>(raw + rr * 32 + hf * 16);
+          const uint32_t sc2 = *reinterpret_cast<const uint16_t*>(sblock + rr * 16 + hf * 2);
+          uint32_t s2;   // the two 16-element block scales as f16, each in both halves of a pair
+          asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(s2) : "r"(sc2));
+          const uint32_t s_lo = __byte_perm(s2, 0, 0x1010), s_hi = __byte_perm(s2, 0, 0x3232);
+          const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {   // word j: elements 8j .. 8j+7 of the half -> chunk 4 hf + j
+            const uint32_t sp = j < 2 ? s_lo : s_hi;
+            uint4 o;
+            o.x = e2m1x2_times(w[j] & 0xFFu, sp);
+            o.y = e2m1x2_times((w[j] >> 8) & 0xFFu, sp);
+            o.z = e2m1x2_times((w[j] >> 16) & 0xFFu, sp);
+            o.w = e2m1x2_times(w[j] >> 24, sp);
+            const int c = 4 * hf + j;
+            *reinterpret_cast<uint4*>(sb + rr * 128 + ((c ^ (rr & 7)) * 16)) = o;
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
+        mbar_arrive(&S->conv[s]);
+      }
+      if (stop) break;
     }
   }
   tc_fence_before();
@@ -330,7 +442,11 @@ cudaError_t launch_wait_selftest(unsigned long long limit_ns, int* err, cudaStre
   return cudaGetLastError();
 }
 
-size_t gemm_smem_bytes() { return 1024 + STAGES * STAGE_BYTES + sizeof(GemmSmem); }
+size_t gemm_smem_bytes(int wt) {
+  return wt == GW_NVFP4
+             ? 1024 + GemmCfg<GW_NVFP4>::STAGES * stage_bytes<GW_NVFP4>() + GemmCfg<GW_NVFP4>::SCALE_RING + sizeof(GemmSmem)
+             : 1024 + GemmCfg<GW_BF16>::STAGES * stage_bytes<GW_BF16>() + sizeof(GemmSmem);
+}
 
 cudaError_t launch_gather_rows(const void* x, const int* perm, int T, int k, int H, bool with_shared,
                                void* A, cudaStream_t s) {
@@ -345,29 +461,41 @@ cudaError_t launch_gather_rows(const void* x, const int* perm, int T, int k, int
   return cudaGetLastError();
 }
 
+namespace {
+template <int MODE, int WT>
+cudaError_t launch_gemm_t(const GemmMaps& maps, const GemmGroups& groups, const GemmFp4& fp4, const int* offsets,
+                          int T, int k, int I, int H, void* out, int* err, int grid, cudaStream_t s) {
+  const size_t smem = gemm_smem_bytes(WT);
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const CUtensorMap& a = MODE == 0 ? maps.a_x : maps.a_h;
+  const CUtensorMap& br = MODE == 0 ? maps.b1_routed : maps.b2_routed;
+  const CUtensorMap& bs = MODE == 0 ? maps.b1_shared : maps.b2_shared;
+  grouped_gemm_kernel<MODE, WT><<<grid, GemmCfg<WT>::THREADS, smem, s>>>(a, br, bs, groups, fp4, offsets, T, k, I, H,
+                                                                         out, err);
+  return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t launch_grouped_gemm(int mode, const GemmMaps& maps, const GemmGroups& groups, const int* offsets,
                                 int T, int k, int I, int H, void* out, int* err, int num_sms, cudaStream_t s,
-                                const float* gscale) {
+                                const GemmFp4* fp4) {
   if (groups.n <= 0 || T <= 0) return cudaSuccess;
-  const size_t smem = gemm_smem_bytes();
   // an upper bound of the tile count; CTAs beyond the real count exit at once
   const long long rows_max = (long long)T * k + T;
   const int n_tiles = mode == 0 ? I / (BN / 2) : H / BN;
   long long tiles_max = ((rows_max + BM - 1) / BM + groups.n) * n_tiles;
   int grid = num_sms;
   if (tiles_max < grid) grid = (int)tiles_max;
-  if (mode == 0) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<0><<<grid, GEMM_THREADS, smem, s>>>(maps.a_x, maps.b1_routed, maps.b1_shared, groups,
-                                                            offsets, T, k, I, H, out, err, gscale);
-  } else {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<1><<<grid, GEMM_THREADS, smem, s>>>(maps.a_h, maps.b2_routed, maps.b2_shared, groups,
-                                                            offsets, T, k, I, H, out, err, gscale);
+  static const GemmFp4 no_fp4 = {};
+  if (fp4) {
+    if (H % 256 || I % 256) return cudaErrorInvalidValue;
+    return mode == 0 ? launch_gemm_t<0, GW_NVFP4>(maps, groups, *fp4, offsets, T, k, I, H, out, err, grid, s)
+                     : launch_gemm_t<1, GW_NVFP4>(maps, groups, *fp4, offsets, T, k, I, H, out, err, grid, s);
   }
-  return cudaGetLastError();
+  return mode == 0 ? launch_gemm_t<0, GW_BF16>(maps, groups, no_fp4, offsets, T, k, I, H, out, err, grid, s)
+                   : launch_gemm_t<1, GW_BF16>(maps, groups, no_fp4, offsets, T, k, I, H, out, err, grid, s);
 }
 
 }  // namespace ftk
@@ -415,6 +543,19 @@ bool encode_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t ro
   cuuint32_t es[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_map_u8_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                      uint64_t row_bytes, uint64_t depth_bytes, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, depth};
+  cuuint64_t strides[2] = {row_bytes, depth_bytes};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

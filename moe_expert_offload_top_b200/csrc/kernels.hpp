@@ -51,8 +51,10 @@ cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdt
                               const int* perm, float* h, float* y, cudaStream_t s,
                               cudaEvent_t between = nullptr, int* err = nullptr, bool int4_tensor = true);
 // K3 (decode) for int4 group-128 weights with mma.sync (gemv_int4_mma.cu); x bf16.
+// max_pairs_per_expert: the most pairs one entry owns (sizes per-CTA input staging).
 cudaError_t launch_ffn_int4_mma(const void* x, int T, int H, int I, int k, const ExpertList& list, const int* offsets,
-                                const int* perm, float* h, float* y, cudaStream_t s, cudaEvent_t between);
+                                const int* perm, float* h, float* y, cudaStream_t s, cudaEvent_t between,
+                                int max_pairs_per_expert);
 // K3 + K5 (decode) in one launch (ffn_fused.cuh): gate/up + SwiGLU into h, down into y
 // and, with `combine`, out[t] = sum_j gates[t][j] * y[inv[t*k+j]] (+ shared) for the
 // entries of `list`.  The combine of a launch covers every pair of the forward, so
@@ -117,23 +119,38 @@ struct GemmMaps {
   CUtensorMap b2_shared;  // down rows of shared experts [L][H][I]
 };
 
-size_t gemm_smem_bytes();
+// Weight format of the prefill GEMMs.
+enum { GW_BF16 = 0, GW_NVFP4 = 1 };
+// NVFP4 slots for the prefill GEMMs, expanded to bf16 inside the GEMM: tensor maps over
+// the packed e2m1 codes and the e4m3 block scales of the slot arena and of the shared
+// experts (index 0: the gate|up rows [2I][H/2 or H/16], 1: the down rows [H][I/2 or I/16];
+// uint8, boxes of 32 or 16 bytes x 128 rows), and where each blob's three fp32 matrix
+// scales lie: g_routed + z * blob + g_off (slot z), or g_shared + layer * blob + g_off.
+struct GemmFp4 {
+  CUtensorMap q_routed[2], q_shared[2];
+  CUtensorMap s_routed[2], s_shared[2];
+  const uint8_t* g_routed;
+  const uint8_t* g_shared;
+  unsigned long long blob;
+  unsigned long long g_off;
+};
+
+size_t gemm_smem_bytes(int wt);
 // One CTA waits (bounded by limit_ns) on an mbarrier nobody arrives on; sets *err = 199.
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, int* err, cudaStream_t s);
 // A[q] = x[perm[q] / k] for q < T*k; A[T*k + t] = x[t] when with_shared (bf16 rows of H).
 cudaError_t launch_gather_rows(const void* x, const int* perm, int T, int k, int H, bool with_shared,
                                void* A, cudaStream_t s);
 // mode 0: h = silu(A W_gate^T) * (A W_up^T) (bf16 [rows][I]); mode 1: y = h W_down^T (f32 [rows][H]).
-// gscale (optional, device): 3 fp32 scales (gate, up, down) per weight slot z, applied to the
-// accumulators (staged NVFP4 weights); null for bf16 weights.
+// bf16 weights through maps.b*; with fp4 (H, I multiples of 256), NVFP4 weights expanded in
+// the GEMM, whose epilogue applies each matrix's fp32 scale.  Bounded pipeline waits that give
+// up write 101-106 to *err.
 cudaError_t launch_grouped_gemm(int mode, const GemmMaps& maps, const GemmGroups& groups, const int* offsets,
                                 int T, int k, int I, int H, void* out, int* err, int num_sms, cudaStream_t s,
-                                const float* gscale = nullptr);
-// Expands the NVFP4 blobs of list's entries to bf16 (e2m1 * e4m3, exact) in stage slot i
-// (3*H*I bf16 per slot, the bf16 blob layout) and writes their fp32 matrix scales to
-// gscale[3i .. 3i+2] (dequant_stage.cu).
-cudaError_t launch_dequant_nvfp4_stage(const ExpertList& list, int H, int I, void* stage, float* gscale, int num_sms,
-                                       cudaStream_t s);
+                                const GemmFp4* fp4 = nullptr);
+// uint8 3-D tensor map without swizzle (box box_inner bytes x box_rows rows x 1).
+bool encode_map_u8_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                      uint64_t row_bytes, uint64_t depth_bytes, uint32_t box_inner, uint32_t box_rows);
 // 2-D / 3-D bf16 tensor maps with 128-byte swizzle (box inner extent 64 elements).
 bool encode_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
                    uint32_t box_rows);

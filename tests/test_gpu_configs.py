@@ -24,17 +24,18 @@ def test_prefill_gemm_and_gemv_paths_match_oracle(gemm_threshold):
 
 
 @pytest.mark.parametrize("gemm_threshold", [0, 1 << 30])
-def test_nvfp4_prefill_staged_gemm_and_gemv_paths_match_oracle(gemm_threshold):
-    # NVFP4 stacks in prefill: the selected experts are expanded to bf16 (exact) for the
-    # tcgen05 GEMMs, whose epilogue applies each matrix's fp32 scale; or the GEMV path
+def test_nvfp4_prefill_fused_gemm_and_gemv_paths_match_oracle(gemm_threshold):
+    # NVFP4 stacks in prefill: the GEMMs expand each weight tile to bf16 (exact) in shared
+    # memory, and their epilogue applies each matrix's fp32 scale; or the GEMV path
     cfg = synth.MoeConfig("prefill-nvfp4", L=2, E=16, H=512, I=256, k=4, gating="sigmoid", wdtype="nvfp4",
                           shared=True, C=32, tokens=700, batches=(700,), process="iid", mode="prefill")
     st = run_and_check(cfg, 700, sample_steps=[0], gemm_threshold=gemm_threshold)
     assert st["misses"] == 0 and st["prefetch_misses"] == 2 * 16
 
 
-def test_nvfp4_staged_gemm_uneven_groups():
-    cfg = synth.MoeConfig("skew-nvfp4", L=1, E=8, H=768, I=384, k=2, gating="softmax", wdtype="nvfp4",
+def test_nvfp4_fused_gemm_uneven_groups():
+    # NVFP4 on the GEMM path needs H and I multiples of 256 (block scales in 16-byte boxes)
+    cfg = synth.MoeConfig("skew-nvfp4", L=1, E=8, H=768, I=512, k=2, gating="softmax", wdtype="nvfp4",
                           shared=False, C=8, tokens=400, batches=(400,), process="ar1", mode="decode")
     run_and_check(cfg, 400, sample_steps=[0], gemm_threshold=0)
 

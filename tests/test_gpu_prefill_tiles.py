@@ -5,7 +5,8 @@ flips and the pipeline's stage reuse across tiles are all exercised.
 64 experts, H=1024, I=512, top-6 sigmoid plus a shared expert, 2048 tokens: the
 gate/up and down GEMMs each have about 700 tiles for the 148 CTAs.  Checked
 through the C ABI on every y row of the step-level entry (ft_expert_ffn_prefill)
-and on every token of the forward (ft_moe_forward in prefill mode)."""
+and on every token of the forward (ft_moe_forward in prefill mode), for bf16 and
+NVFP4 weights."""
 import numpy as np
 import pytest
 import torch
@@ -21,8 +22,8 @@ E, K, H, I, T = 64, 6, 1024, 512, 2048
 BM, BN = 128, 256   # the GEMM tile: 128 pair rows x 256 accumulator columns
 
 
-def _cfg(L=1):
-    return synth.MoeConfig("prefill-tiles", L=L, E=E, H=H, I=I, k=K, gating="sigmoid", wdtype="bf16",
+def _cfg(L=1, wdtype="bf16"):
+    return synth.MoeConfig("prefill-tiles", L=L, E=E, H=H, I=I, k=K, gating="sigmoid", wdtype=wdtype,
                            shared=True, C=L * E, tokens=T, batches=(T,), process="iid", mode="prefill")
 
 
@@ -93,8 +94,11 @@ def test_step_level_prefill_gemms_every_y_row():
     assert_close(out.float().cpu().numpy(), ref, "bf16", "combined output")
 
 
-def test_prefill_forward_many_tiles_per_cta_every_token():
-    cfg = _cfg(L=2)
+@pytest.mark.parametrize("wdtype", ["bf16", "nvfp4"])
+def test_prefill_forward_many_tiles_per_cta_every_token(wdtype):
+    # nvfp4: each CTA expands its weight tiles in shared memory, and its block-scale ring
+    # (two slots of 4 stages) turns over across the tiles it runs
+    cfg = _cfg(L=2, wdtype=wdtype)
     st = run_and_check(cfg, T, sample_steps=[0], gemm_threshold=0)
     assert st["misses"] == 0 and st["prefetch_misses"] == 2 * E
     assert (0, 0, T) in st["compared"] and (0, 1, T) in st["compared"]
