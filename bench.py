@@ -25,7 +25,8 @@ The one JSON line (rank 0) carries:
     cold-start figure of the warm-up steps, SM clocks sampled during the timed region,
     the CPU oracle timed on a bounded sample;
   - legs (N = 1 only): "int4-large-pool" decode at batch 1 (16 layers, H=7168, int4
-    g128, 15% cached); "prefill" of the headline shapes (4096 tokens through the 8
+    g128, 15% cached), and at batch 8 and 32 before and after the stated growth of the
+    cache from 15% to 30%; "prefill" of the headline shapes (4096 tokens through the 8
     layers with whole-layer double buffering over PCIe, the same with every expert
     resident, a tensor-pipe sweep of one resident layer at 16k/32k/64k tokens, and one
     layer with NVFP4 weights, every expert resident); "shrink": decode
@@ -460,6 +461,8 @@ def int4_leg(args, dev, peaks, peak_src, link_h2d):
                               "miss_rate": r["cold_st"]["misses"] / max(r["cold_st"]["routed"], 1)},
                "stages_us_per_forward": stage_us(r["perf"]), "pool_setup_s": setup_s,
                "note": "fixed capacity (no resize inside the timed steps)"}
+        if args.int4_batch_steps > 0:
+            res["batches"] = int4_batches(args, stack, cfg, dev)
         if not args.no_cpu_baseline:
             vals, _ = token_chain(cfg, 0, args.warmup + 1)
             rate, layers, cdt = cpu_oracle_rate(cfg, vals[args.warmup:], stack.pool_blob,
@@ -470,6 +473,39 @@ def int4_leg(args, dev, peaks, peak_src, link_h2d):
                                              % (args.warmup, layers, cfg.L, cdt)}
     finally:
         stack.close()
+    return res
+
+
+def int4_batches(args, stack, cfg, dev):
+    """The int4-large-pool workload at decode batch 8 and 32 (independent AR(1) chains), with
+    the stated mid-run cache resize: steps at 15% of the experts, then at 30% after growing
+    the cache at a safe point.  Device-timed with CUDA events, a few steps per point (a step
+    at batch 32 reads several hundred experts over PCIe)."""
+    import torch
+
+    import moe_expert_offload_top_b200 as ft
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    K, W = args.int4_batch_steps, 2
+    for B in (8, 32):
+        vals, bits = synth.tokens(cfg, B)
+        x = torch.from_numpy(bits[:W + 2 * K]).view(torch.bfloat16).to(dev)
+        out = torch.empty((cfg.L, B, cfg.H), dtype=torch.bfloat16, device=dev)
+        stack.resize(cfg.C)
+        ft.ft_cache_clear(stack.h)
+        timed_steps(stack, list(x[:W]), out, stream, dev)
+        pts = {}
+        for label, lo in (("slots_15pct", W), ("slots_30pct", W + K)):
+            if label == "slots_30pct":
+                stack.resize(cfg.resize_to)
+            stack.reset_stats()
+            dt = timed_steps(stack, list(x[lo:lo + K]), out, stream, dev)
+            st = stack.stats()
+            pts[label] = {"cache_slots": stack.C, "tokens_per_s": B * K / dt, "ms_per_step": 1e3 * dt / K,
+                          "miss_rate": st["misses"] / max(st["routed"], 1),
+                          "h2d_gbs": st["h2d_bytes"] / st["h2d_seconds"] / 1e9 if st["h2d_seconds"] > 0 else None}
+        res["batch_%d" % B] = dict(steps=K, warmup=W, **pts)
+    stack.resize(cfg.C)
     return res
 
 
@@ -762,6 +798,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--legs", default="all", help="comma list of %s, or all (N = 1 only)" % ",".join(ALL_LEGS))
     ap.add_argument("--int4-steps", type=int, default=96)
+    ap.add_argument("--int4-batch-steps", type=int, default=4, help="steps per point at batch 8 and 32 (0: skip)")
     ap.add_argument("--shrink-steps", type=int, default=256)
     ap.add_argument("--prefill-passes", type=int, default=2)
     ap.add_argument("--no-sweep", dest="sweep", action="store_false", help="skip the prefill token sweep")

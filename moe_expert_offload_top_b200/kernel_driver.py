@@ -8,7 +8,9 @@ shared expert) and token process; --layers / --experts shrink the pool so that a
 profiler's capture stays small (a few GB on the device), and --slots defaults to every
 expert resident, so the launches are the kernels alone.  Decode workloads run S steps of
 B tokens; prefill workloads run S forwards of T tokens through every layer.  Prints one
-line with the steps run and the cache counters.
+line with the steps run and the cache counters (with --perf, stage timing is on and the
+line adds each FFN launch's algorithmic bytes and flops, averaged over the launches, for
+setting a profiler's DRAM counters against).
 """
 import argparse
 import dataclasses
@@ -17,6 +19,7 @@ import sys
 
 import torch
 
+import moe_expert_offload_top_b200 as ft
 import synth
 from moe_expert_offload_top_b200.workload import GpuStack
 
@@ -30,6 +33,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=12)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--tokens", type=int, default=None, help="prefill: tokens per forward")
+    ap.add_argument("--perf", action="store_true",
+                    help="stage timing on: also print the algorithmic bytes and flops per FFN launch")
     a = ap.parse_args(argv)
     base = synth.CONFIGS[a.workload]
     E = a.experts or base.E
@@ -42,11 +47,20 @@ def main(argv=None):
     with GpuStack(cfg, max_tokens=T) as st:
         vals, x = st.tokens(T)
         out = torch.empty((cfg.L, T, cfg.H), dtype=st.xdt, device=st.device)
+        if a.perf:
+            ft.ft_moe_set_stage_timing(st.h, 1)
         for s in range(a.steps):
             st.step(x[s % x.shape[0]], out)
         torch.cuda.synchronize()
-        print(json.dumps({"workload": cfg.name, "layers": cfg.L, "experts": cfg.E, "slots": cfg.C, "steps": a.steps,
-                          "tokens_per_step": T, "cache": st.stats()}))
+        line = {"workload": cfg.name, "layers": cfg.L, "experts": cfg.E, "slots": cfg.C, "steps": a.steps,
+                "tokens_per_step": T, "cache": st.stats()}
+        if a.perf:
+            p = ft.ft_moe_perf(st.h)
+            n = max(p["ffn_gate_up_launches"], 1)
+            line["per_launch"] = {"gate_up_bytes": p["ffn_gate_up_bytes"] / n, "down_bytes": p["ffn_down_bytes"] / n,
+                                  "flops": p["ffn_flops"] / n, "gate_up_us": 1e3 * p["ffn_gate_up_ms"] / n,
+                                  "down_us": 1e3 * p["ffn_down_ms"] / n, "launches": n}
+        print(json.dumps(line))
     return 0
 
 

@@ -12,15 +12,35 @@ BOUNDS = {"bf16": (5e-3, 2e-2), "int4": (5e-3, 2e-2), "nvfp4": (5e-3, 2e-2), "f3
 TIE_GAP = 1e-5   # logit gap below which either top-k choice is correct
 
 
-def assert_close(got, ref, wdtype, what=""):
+def bf16_half_ulp(v):
+    """Half the spacing of bf16 values at |v| (the largest rounding error of storing v as
+    bf16, round to nearest): |v| in [2^e, 2^(e+1)) has 8 significant bits, ulp 2^(e-7)."""
+    m, e = np.frexp(np.abs(np.asarray(v, dtype=np.float64)))   # |v| = m 2^e, m in [0.5, 1)
+    return np.where(m == 0, 0.0, np.ldexp(1.0, (e - 9).astype(np.int64)))
+
+
+def assert_close(got, ref, wdtype, what="", stored_bf16=False):
+    """The stated parity bound: relative L2 <= rl2 and max-abs <= rmax * rms(ref).
+
+    stored_bf16: got holds bf16 outputs of the library.  Storing a value as bf16 rounds it by
+    up to half an ulp of itself, on top of any error of the computation; the max-abs bound is
+    applied to the computation, so each element is allowed its own half ulp in addition.
+    (Without it, even the exact result rounded to bf16 fails the bound on outputs beyond about
+    five times rms(out), which full-layer comparisons of millions of outputs contain.)"""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     rl2, rmax = BOUNDS[wdtype]
     rms = np.sqrt(np.mean(ref * ref))
     rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
-    mx = np.max(np.abs(got - ref)) if got.size else 0.0
     assert rel <= rl2, "%s: relative L2 %.3g > %.3g" % (what, rel, rl2)
-    assert mx <= rmax * rms, "%s: max-abs %.3g > %.3g * rms %.3g" % (what, mx, rmax, rms)
+    if got.size:
+        err = np.abs(got - ref)
+        allow = rmax * rms + (bf16_half_ulp(np.maximum(np.abs(got), np.abs(ref))) if stored_bf16 else 0.0)
+        i = int(np.argmax(err - allow))
+        assert err.flat[i] <= np.broadcast_to(allow, err.shape).flat[i], \
+            "%s: max-abs %.3g > %.3g (%.3g * rms %.3g%s) at %.4g vs %.4g" % (
+                what, err.flat[i], np.broadcast_to(allow, err.shape).flat[i], rmax, rms,
+                " + half an ulp of the stored bf16" if stored_bf16 else "", got.flat[i], ref.flat[i])
     return rel
 
 
@@ -183,5 +203,6 @@ def run_and_check(cfg, batch, sample_steps, sample_tokens=None, gemm_threshold=N
         nw = workers or min(8, os.cpu_count() or 1, max(len(jobs), 1))
         with concurrent.futures.ThreadPoolExecutor(max_workers=nw) as ex:
             for (s, l, toks), ref in zip(jobs, ex.map(oracle_out, jobs)):
-                assert_close(outs[s][l][toks], ref, cfg.wdtype, "step %d layer %d (%d tokens)" % (s, l, len(toks)))
+                assert_close(outs[s][l][toks], ref, cfg.wdtype, "step %d layer %d (%d tokens)" % (s, l, len(toks)),
+                             stored_bf16=cfg.x_dtype == "bf16")
         return {**stats, "compared": [(s, l, len(t)) for s, l, t in jobs]}

@@ -46,7 +46,7 @@ def test_failed_fill_rolls_back_and_next_forward_recovers():
                 r = moe.route(vals[s], synth.router_weights(cfg, l), cfg.k, cfg.gating)
                 ref = moe.experts_and_combine(vals[s], r["ids"], r["gates"], cfg.E, cfg.wdtype, cfg.H, cfg.I,
                                               lambda e, l=l: st.pool_blob(l, e))
-                assert_close(got[s][l], ref, "bf16", "step %d layer %d" % (s, l))
+                assert_close(got[s][l], ref, "bf16", "step %d layer %d" % (s, l), stored_bf16=True)
 
 
 def test_routing_timeout_changes_nothing():
@@ -119,4 +119,4 @@ def test_fused_ffn_wait_gives_up_and_is_reported():
                 r = moe.route(vals[s], synth.router_weights(cfg, l), cfg.k, cfg.gating)
                 ref = moe.experts_and_combine(vals[s], r["ids"], r["gates"], cfg.E, cfg.wdtype, cfg.H, cfg.I,
                                               lambda e, l=l: st.pool_blob(l, e))
-                assert_close(got[s][l], ref, "bf16", "step %d layer %d" % (s, l))
+                assert_close(got[s][l], ref, "bf16", "step %d layer %d" % (s, l), stored_bf16=True)

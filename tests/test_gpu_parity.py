@@ -192,7 +192,7 @@ def test_expert_ffn_and_combine_parity(wd, H, I, T, E, k, shared):
             ref = moe.swiglu_ffn(xv[pair // k][None], wg, wu, wdn)[0]
             assert_close(y[q], ref, wd, "y pair %d expert %d" % (pair, e))
     ref_out = moe.experts_and_combine(xv, ids, gates.astype(np.float64), E, wd, H, I, lambda e: blobs[e], sh)
-    assert_close(out.float().cpu().numpy(), ref_out, wd, "combined out")
+    assert_close(out.float().cpu().numpy(), ref_out, wd, "combined out", stored_bf16=wd != "f32")
 
 
 # ------------------------------------------------------------- forwards --
@@ -230,7 +230,8 @@ def _check_run(cfg, stack, vals, outs, ids, ref, steps):
         if s >= last:
             continue
         for l in range(cfg.L):
-            assert_close(o[l], ref["out"][(s, l)], cfg.wdtype, "step %d layer %d" % (s, l))
+            assert_close(o[l], ref["out"][(s, l)], cfg.wdtype, "step %d layer %d" % (s, l),
+                         stored_bf16=cfg.x_dtype == "bf16")
 
 
 def test_config1_tiny_forward_parity():
@@ -326,7 +327,7 @@ def test_resize_grow_and_shrink_mid_run():
                 if s % 10 == 9:
                     o = moe.experts_and_combine(vals[s], r["ids"], r["gates"], cfg.E, cfg.wdtype, cfg.H,
                                                 cfg.I, lambda e, l=l: st.pool_blob(l, e))
-                    assert_close(got[s][l], o, cfg.wdtype, "step %d layer %d" % (s, l))
+                    assert_close(got[s][l], o, cfg.wdtype, "step %d layer %d" % (s, l), stored_bf16=cfg.x_dtype == "bf16")
         assert [tuple(t) for t in st.trace()] == trace_tuples(ref_l.trace)
         assert st.stats()["capacity"] == 17
 
@@ -368,7 +369,7 @@ def test_forwards_on_alternating_streams():
         ref = oracle_run(cfg, st, vals)
         for s in range(cfg.tokens):
             for l in range(cfg.L):
-                assert_close(got[s][l], ref["out"][(s, l)], "bf16", "step %d layer %d" % (s, l))
+                assert_close(got[s][l], ref["out"][(s, l)], "bf16", "step %d layer %d" % (s, l), stored_bf16=True)
 
 
 def test_empty_forward_changes_nothing():

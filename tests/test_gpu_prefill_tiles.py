@@ -91,7 +91,7 @@ def test_step_level_prefill_gemms_every_y_row():
     out = torch.empty((T, H), dtype=torch.bfloat16, device=DEV)
     ft.ft_combine(y, g_dev, inv_dev, T, H, K, True, True, out)
     ref = moe.experts_and_combine(x_f, r["ids"], r["gates"], E, "bf16", H, I, lambda e: blobs[e], blobs[E])
-    assert_close(out.float().cpu().numpy(), ref, "bf16", "combined output")
+    assert_close(out.float().cpu().numpy(), ref, "bf16", "combined output", stored_bf16=True)
 
 
 @pytest.mark.parametrize("wdtype", ["bf16", "nvfp4"])

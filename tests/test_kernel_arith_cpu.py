@@ -74,3 +74,50 @@ def test_bf16_hi_lo_split_keeps_h_within_2_pow_minus_17():
     # adds the next 9 bits, since |h - hi| is at most half an ulp of hi
     assert np.all(np.abs(hi.astype(np.float64) - h) <= 2.0 ** -8 * np.abs(h.astype(np.float64)))
     assert np.max(err / np.maximum(np.abs(h.astype(np.float64)), 1e-300)) > 2.0 ** -19   # the bound is nearly reached
+
+
+def test_nvfp4_expansion_writes_each_swizzled_chunk_once():
+    # The NVFP4 prefill GEMM expands one stage (a B tile of 256 rows x 64 K elements) with
+    # 128 threads, item = thread + 128 i (i < 4), row rr = item >> 1, half hf = item & 1:
+    # it reads 16 code bytes at rr*32 + hf*16 of the raw tile and two scale bytes at
+    # rr*16 + (kb & 3)*4 + 2*hf of the scale block, and writes chunk c = 4*hf + j (j < 4)
+    # of row rr at rr*128 + ((c ^ (rr & 7)) * 16): the 128-byte swizzle the MMA descriptor
+    # reads (TMA writes bf16 tiles the same way).  Every chunk of the 32 KB tile must be
+    # written exactly once, at the address the swizzle gives K elements 8c .. 8c+7, and
+    # every read must stay inside the 8 KB code tile and the 4 KB scale block.
+    written = {}
+    raw_reads, scale_reads = set(), set()
+    for thread in range(128):
+        for i in range(4):
+            item = thread + 128 * i
+            rr, hf = item >> 1, item & 1
+            raw_reads.add(rr * 32 + hf * 16)
+            for kb in range(4):
+                off = rr * 16 + (kb & 3) * 4 + 2 * hf
+                assert 0 <= off and off + 2 <= 256 * 16
+                scale_reads.add(off)
+            for j in range(4):
+                c = 4 * hf + j
+                addr = rr * 128 + ((c ^ (rr & 7)) * 16)
+                assert addr not in written
+                written[addr] = (rr, c)
+    assert sorted(written) == list(range(0, 256 * 128, 16))
+    for addr, (rr, c) in written.items():
+        # the swizzle places chunk c of row rr at 16-byte position c ^ (rr % 8) of the row
+        assert addr // 128 == rr and (addr % 128) // 16 == c ^ (rr % 8)
+    assert sorted(raw_reads) == list(range(0, 256 * 32, 16))      # each 16-byte code group once
+    assert len(scale_reads) == 256 * 2 * 4                        # two scales per item, per stage
+
+
+def test_nvfp4_expansion_element_order():
+    # Code byte b of a half-row holds K elements 2b (low nibble) and 2b+1 (high nibble); word j
+    # (bytes 4j .. 4j+3) becomes output chunk j, whose 16-byte bf16 words are the pairs of bytes
+    # 4j, 4j+1, 4j+2, 4j+3 in order: so chunk c of the row holds K elements 8c .. 8c+7 and the
+    # 16-element block scale of elements 16s .. 16s+15 is block s (j < 2: s = 2 hf, else 2 hf + 1).
+    for hf in range(2):
+        for j in range(4):
+            c = 4 * hf + j
+            elems = [2 * (4 * j + b) + n for b in range(4) for n in range(2)]   # within the half
+            assert [32 * hf + e for e in elems] == list(range(8 * c, 8 * c + 8))
+            block = 2 * hf + (0 if j < 2 else 1)
+            assert all((32 * hf + e) // 16 == block for e in elems)

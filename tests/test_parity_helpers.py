@@ -68,3 +68,28 @@ def test_float_bound_accepts_rounding_and_rejects_a_planted_error():
         assert_close(ref * 1.01, ref, "bf16")             # a 1% scale error: relative L2 1e-2
     with pytest.raises(AssertionError):
         assert_close(bf16_like, ref, "f32")               # bf16 rounding is far outside the fp32 bound
+
+
+def test_bf16_storage_allowance():
+    # The allowance for bf16-stored outputs is half an ulp of the stored value, checked here
+    # against the generator's bf16 rounding (round to nearest even): the exact values stored
+    # as bf16 pass the max-abs bound with it even where an outlier's own rounding exceeds
+    # 2e-2 * rms, and a real error on top of the rounding still fails.
+    import synth
+    from gpu_util import bf16_half_ulp
+    rng = np.random.default_rng(1)
+    ref = rng.standard_normal(20000)
+    ref[7] = 9.9                                  # an outlier at ~10 rms: its rounding is ~0.03 rms
+    stored = (synth.round_bf16(ref.astype(np.float32)).astype(np.uint32) << 16).view(np.float32)
+    assert np.all(np.abs(stored - ref) <= bf16_half_ulp(ref))        # half an ulp bounds RNE
+    assert np.abs(stored[7] - ref[7]) > 2e-2 * np.sqrt(np.mean(ref * ref))   # the bound alone fails here
+    assert_close(stored, ref, "bf16", stored_bf16=True)
+    with pytest.raises(AssertionError):
+        assert_close(stored, ref, "bf16")
+    bad = stored.astype(np.float64)
+    bad[11] += 0.05 * np.sqrt(np.mean(ref * ref))
+    with pytest.raises(AssertionError):
+        assert_close(bad, ref, "bf16", stored_bf16=True)
+    # the half ulp: 2^(e-8) for |v| in [2^e, 2^(e+1))
+    assert bf16_half_ulp(1.0) == 2.0 ** -8 and bf16_half_ulp(1.99) == 2.0 ** -8 and bf16_half_ulp(2.0) == 2.0 ** -7
+    assert bf16_half_ulp(-0.75) == 2.0 ** -9 and bf16_half_ulp(0.0) == 0.0
