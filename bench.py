@@ -90,12 +90,20 @@ def headline_config(world):
 TRAFFIC = {
     "gemv_bf16": {"sources": ["moe_expert_offload_top_b200/csrc/decode_gemv.cuh",
                               "moe_expert_offload_top_b200/csrc/expert_decode.cu"],
-                  "sha256": None, "ratio": None, "capture": None},
+                  "sha256": "dbebf6db6b2b1d148770f5fa47b7c9163955ea7c74973d38dd0a9d3edb2a4264", "ratio": 1.00316,
+                  "capture": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 8 gate/up launches of "
+                             "kernel_driver --workload dsv4flash-decode-bf16 --layers 1 --experts 16 --steps 8 "
+                             "--perf (7 experts per launch, as here), 1.00316 of their algorithmic bytes; scaled "
+                             "to the average launch here"},
     "gemv_int4": {"sources": ["moe_expert_offload_top_b200/csrc/decode_gemv.cuh",
                               "moe_expert_offload_top_b200/csrc/gemv_int4_mma.cu"],
                   "sha256": None, "ratio": None, "capture": None},
     "gemm": {"sources": ["moe_expert_offload_top_b200/csrc/grouped_gemm_sm100.cu"],
-             "sha256": None, "ratio": None, "capture": None},
+             "sha256": "0507ce91301990d38f67cede0ff1f116891de1794c23254f95a46243e0b318f6", "ratio": 1.03732,
+             "capture": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the gate/up and down launches of "
+                        "kernel_driver --workload dsv4flash-prefill-bf16 --layers 1 --experts 64 --tokens 8192 "
+                        "--steps 2 --perf (768 pairs per expert, compute-bound like the sweep), 1.03732 of their "
+                        "algorithmic bytes; scaled to the swept forward's bytes"},
 }
 
 
