@@ -227,11 +227,12 @@ FT_API int ft_moe_set_fused_routing(ft_moe* h, int enabled);
  * the combine.  The per-output arithmetic is the same, so the outputs are bit-identical. */
 FT_API int ft_moe_set_fused_ffn(ft_moe* h, int enabled);
 
-/* int4 decode GEMV (per-pass launch shape): 1 (default) = on the tensor cores
- * (mma.sync with bf16 operands and fp32 accumulation; the down projection's input h is
- * carried as two bf16 halves, 16 mantissa bits), 0 = fp32 multiply-adds on the CUDA
- * cores.  Both are within the stated bound of the oracle; their outputs differ in the
- * last bits (summation order).  ft_expert_ffn_decode always uses the tensor cores. */
+/* int4 decode GEMV (per-pass launch shape): 1 (default) = on the int8 tensor cores
+ * (mma.sync m16n8k32: the nibbles as signed bytes 16 q, the inputs x and h as 16-bit block
+ * fixed point in two bytes, exact int32 products per 128-element group, scaled and summed
+ * in fp32), 0 = fp32 multiply-adds on the CUDA cores.  Both are within the stated bound of
+ * the oracle; their outputs differ in the last bits.  ft_expert_ffn_decode always uses the
+ * tensor cores. */
 FT_API int ft_moe_set_int4_tensor_cores(ft_moe* h, int enabled);
 
 /* Host-side fault injection for tests of failure handling (no GPU fault is made).
@@ -439,7 +440,13 @@ FT_API int ft_permute(const int* ids, int T, int top_k, int E, int* counts, int*
  *     y[q] = W_down h[q]                          (y: [T*k + T][H] f32, device)
  *   x: [T][H] device, f32 for FT_W_F32, else bf16.  max_pairs_per_expert: the largest
  *   pair count of one entry (sizes the per-CTA token staging; larger values are
- *   processed in chunks of 8).  Rows of h / y that no entry owns are not written. */
+ *   processed in chunks of 8).  Rows of h / y that no entry owns are not written.
+ *   FT_W_INT4_G128 (the int8 tensor-core GEMV): the tokens and, between the two passes,
+ *   the entries' h rows are rewritten as 16-bit block fixed point (a signed and an
+ *   unsigned byte per value, then a float scale), the tokens in the first
+ *   T * (2H + 16) bytes of y before the down pass writes y, the h rows in place; so after
+ *   the call h holds that form, not the fp32 values, and rows of y that no entry owns may
+ *   hold those bytes. */
 FT_API int ft_expert_ffn_decode(const void* x, int T, int H, int I, int top_k, int wdtype,
                          const void* const* blobs, const int* experts, int n_list,
                          int max_pairs_per_expert, const int* offsets, const int* perm, float* h,

@@ -102,6 +102,7 @@ struct ft_moe {
   int* d_perm = nullptr;
   int* d_inv = nullptr;
   float* d_h = nullptr;
+  void* d_xs = nullptr;           // int4 stacks: the forward's tokens as sliced rows (tensor-core GEMV)
   float* d_y = nullptr;
   int* h_ids = nullptr;            // routing ids on the host: h_box + 2
   int* h_box = nullptr;            // mapped pinned {seq, device error word, ids[T*k]}
@@ -225,6 +226,8 @@ void free_scratch(ft_moe* h) {
   cudaFree(h->d_logits); cudaFree(h->d_ids); cudaFree(h->d_gates); cudaFree(h->d_counts);
   cudaFree(h->d_offsets); cudaFree(h->d_perm); cudaFree(h->d_inv); cudaFree(h->d_h);
   cudaFree(h->d_y);
+  cudaFree(h->d_xs);
+  h->d_xs = nullptr;
   cudaFree(h->d_ax);
   h->d_ax = nullptr;
   h->maps_dirty = true;
@@ -253,7 +256,8 @@ int ensure_scratch(ft_moe* h, int T) {
             cudaHostAlloc(&h->h_box, sizeof(int) * (2 + pairs), cudaHostAllocMapped) == cudaSuccess &&
             cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->d_box), h->h_box, 0) == cudaSuccess &&
             ((h->wdtype != FT_W_BF16 && h->wdtype != FT_W_NVFP4) ||
-             cudaMalloc(&h->d_ax, sizeof(uint16_t) * rows * h->H) == cudaSuccess);
+             cudaMalloc(&h->d_ax, sizeof(uint16_t) * rows * h->H) == cudaSuccess) &&
+            (h->wdtype != FT_W_INT4_G128 || cudaMalloc(&h->d_xs, ftk::int4_sliced_x_bytes(T, h->H)) == cudaSuccess);
   if (!ok) {
     cudaGetLastError();
     free_scratch(h);
@@ -921,14 +925,14 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
       stage_mark(se, SE_G0, s);
       FT_CUDA_B(ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, ready, max_pairs, h->d_offsets,
                                         h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr, h->d_err,
-                                        h->int4_tensor != 0));
+                                        h->int4_tensor != 0, h->d_xs));
       stage_mark(se, SE_DA, s);
       rc = wait_fills();
       if (rc) return bail(rc, h->err);
       stage_mark(se, SE_G2, s);
       FT_CUDA_B(ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, later, max_pairs, h->d_offsets,
                                         h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G3] : nullptr, h->d_err,
-                                        h->int4_tensor != 0));
+                                        h->int4_tensor != 0, h->d_xs));
       if (se) se->split = 1;
       h->perf.kernel_launches += 2;
     } else {
@@ -939,7 +943,7 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
       stage_mark(se, SE_G0, s);
       FT_CUDA_B(ftk::launch_ffn_decode(x, T, h->H, h->I, k, h->wdtype, list, max_pairs, h->d_offsets,
                                         h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G1] : nullptr, h->d_err,
-                                        h->int4_tensor != 0));
+                                        h->int4_tensor != 0, h->d_xs));
     }
     stage_mark(se, SE_D1, s);
     rc = record_use();

@@ -116,11 +116,11 @@ static cudaError_t launch_pass(int nt, int rpw, int rows, cudaStream_t s, const 
 cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdtype,
                               const ExpertList& list, int max_pairs_per_expert, const int* offsets,
                               const int* perm, float* h, float* y, cudaStream_t s,
-                              cudaEvent_t between, int* err, bool int4_tensor) {
+                              cudaEvent_t between, int* err, bool int4_tensor, void* int4_xs) {
   (void)err;
   if (list.n <= 0 || T <= 0) return cudaSuccess;
   if (wdtype == WT_INT4 && int4_tensor)
-    return launch_ffn_int4_mma(x, T, H, I, k, list, offsets, perm, h, y, s, between, max_pairs_per_expert);
+    return launch_ffn_int4_mma(x, T, H, I, k, list, offsets, perm, h, y, s, between, max_pairs_per_expert, int4_xs);
   int nt = max_pairs_per_expert < T ? max_pairs_per_expert : T;
   if (nt < 1) nt = 1;
   auto bytes_of = [&](int K) -> size_t {

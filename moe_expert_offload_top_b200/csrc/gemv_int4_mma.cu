@@ -1,54 +1,36 @@
-// K3 for decode with int4 (group-128) expert weights, on the tensor cores.
+// K3 for decode with int4 (group-128) expert weights, on the int8 tensor cores.
 //
 // Method ("FreeToken linux", "FreeToken's MoE memory handling"): each selected expert
 // runs from its cache slot; h = silu(W_gate x) * (W_up x), y = W_down h, with int4
 // weights w = q * s (q a two's-complement nibble, s the bf16 scale of 128 consecutive
 // reduction-axis elements of one row; the low nibble of a byte holds the even element).
 //
-// Why tensor cores for a matrix-vector product.  On the FP32 pipes an int4 weight costs
-// about five instructions (unpack, widen, offset, multiply-add), so the GEMV is bound by
-// instruction issue, not by HBM.  Here the unpack is about one instruction per weight
-// and the multiply-adds go to mma.sync.m16n8k16 (bf16 in, fp32 accumulate), which also
-// covers up to 8 tokens of an expert at once.  The operands stay in registers:
-// tcgen05.mma would take the dequantised weights from shared memory, i.e. twice the
-// HBM bytes again through shared memory, for an M of at most 8 tokens.
+// Integer products, exact.  A nibble q moved into the high half of a byte reads, as a
+// signed int8, 16 q: (w << 4) & 0xF0F0F0F0 gives the even elements of a 32-bit word and
+// w & 0xF0F0F0F0 the odd ones, three instructions per eight weights and no offset to
+// remove.  The inputs (the token x for gate/up, h for down) are written, once per launch,
+// as 16-bit block fixed point: X = round(v * 2^(14 - E)) with E the exponent of the
+// largest |v| of the row (|X| < 2^15; for a bf16 x every element within 2^7 of the
+// largest is exact, and the error of any element is below 2^-15 of the largest), split
+// into a signed high byte and an unsigned low byte, X = 256 hi + lo.
+// mma.sync.m16n8k32 multiplies the 16 q bytes with the hi bytes (s8 x s8) and the lo bytes
+// (s8 x u8) into int32 accumulators, exactly: each 128-element group gives
+// S = 256 D_hi + D_lo = 16 sum(q X).  The group's partial is float(S) times its weight
+// scale s, summed in fp32; the row's result is that sum times 2^(E - 14) / 16.
 //
-// Tile: a CTA owns NM 16-row weight tiles of one expert: gate and up rows of the same
-// 16 (or 32) h columns, or 16*NM consecutive rows of W_down.  Its 4 warps split the
-// reduction axis into contiguous ranges of 128-element groups; their partial sums are
-// added in warp order through shared memory.
+// Fragments (m16n8k32, 8-bit).  Lane (g, t) = (lane / 4, lane % 4) holds 16 bytes (32
+// nibbles, elements 32t .. 32t+31) of weight rows g and g+8 per group.  Word j of that
+// chunk is elements k0 .. k0+7 (k0 = 32t + 8j): its even elements form A register a0 (row
+// g) / a1 (row g+8) and its odd elements a2 / a3 of MMA j.  The reduction index of the MMA
+// is therefore a permutation of the physical one, and the inputs are stored in the same
+// permutation: in every block of 8 elements, the even ones first, then the odd ones.
 //
-// Memory pipeline.  Every lane copies the bytes it will itself use (its two rows of
-// each tile, 16 bytes per row per group, and its 64 bytes of the input vector) into its
-// own slots of a shared-memory ring with cp.async, S groups ahead of the group it
-// computes, and reads them back with 16-byte shared loads: the loads in flight do not
-// hold registers, and no barrier is needed (a thread's cp.async.wait_group covers its
-// own copies).  The scales of the CTA's rows are staged in shared memory once.  The
-// down pass copies its weights (and scales) before griddepcontrol.wait, so they stream
-// while the gate/up grid finishes; only its inputs h wait for it.
-//
-// Fragments.  Lane (g, t) = (lane / 4, lane % 4).  For one 128-element group, lane
-// (g, t) holds 16 bytes (32 nibbles, elements 32t .. 32t+31) of rows g and g+8.  Word j
-// of that chunk holds elements k0 .. k0+7 (k0 = 32t + 8j); the pair (k0+n, k0+n+4) of
-// nibbles n and n+4 becomes one bf16x2 register: ((w >> 4n) & 0x000F000F) ^ 0x43084308
-// is the bf16 pair (136 + q).  This is the exponent-bias (magic number) integer-to-
-// float conversion: the 4-bit integer is written into the low mantissa bits of a float
-// whose exponent makes one mantissa step worth 1 (bf16 128.0 = 0x4300), and flipping
-// bit 3 maps the two's-complement nibble q to q + 8, so the float reads 128 + q + 8
-// (the conversion described for int4 -> fp16 by Kim et al., "Who Says Elephants Can't
-// Run: Bringing Large Scale MoE Models into Cloud Scale Production", 2022, here with a
-// bf16 exponent).  The MMA's reduction index is a permutation of the physical one (the
-// same for weights and inputs): MMA 2j takes pairs n = 0, 1, MMA 2j+1 pairs n = 2, 3,
-// and the input fragment is built from the same element pairs with byte permutes.  The
-// offset 136 is removed per group by one MMA against a constant fragment of -136 (shared
-// by the CTA's tiles), so each group's partial sum is sum(q x) as far as fp32
-// accumulation goes; it is then scaled by the group's s and accumulated.
-//
-// Down projection: its input h is fp32.  The gate/up kernel stores each h value as two
-// bf16 (hi = bf16(h), lo = bf16(h - hi)) in the same row of the h buffer, so h keeps 16
-// bits of mantissa (relative error 2^-17).  The down MMAs take hi and lo as separate
-// columns of the input fragment (columns 0-3: hi of up to 4 tokens, 4-7: their lo), so
-// one MMA covers both, and the two columns are added at the end.
+// Memory pipeline (as before): every lane copies the bytes it uses itself (16 bytes of
+// rows g and g+8 of each tile, 32 + 32 bytes of its input column's hi and lo bytes) into
+// its own slots of a shared-memory ring with cp.async, kStages - 1 groups ahead; the down
+// pass copies its weights before griddepcontrol.wait.  Scales of the CTA's rows are staged
+// in shared memory once.  The 4 warps of a CTA split the reduction axis and add their
+// partial sums in warp order.
 #include "decode_gemv.cuh"
 #include "sm100_sync.cuh"
 
@@ -63,76 +45,149 @@ constexpr int kQThreads = 32 * kQWarps;
 #ifndef FT_INT4_STAGES
 #define FT_INT4_STAGES 4
 #endif
-#ifndef FT_INT4_GU_TILES
-#define FT_INT4_GU_TILES 2
-#endif
 #ifndef FT_INT4_DOWN_TILES
 #define FT_INT4_DOWN_TILES 2
 #endif
-constexpr int kStages = FT_INT4_STAGES;          // groups of copies in flight per lane
-constexpr int kGuTiles = FT_INT4_GU_TILES;       // gate/up: 16-row tiles per CTA (gate, up: even)
-constexpr int kDownTiles = FT_INT4_DOWN_TILES;   // down: 16-row tiles per CTA
-constexpr uint32_t kNeg136x2 = 0xC308C308u;      // bf16 pair (-136, -136)
+constexpr int kStages = FT_INT4_STAGES;
+constexpr int kDownTiles = FT_INT4_DOWN_TILES;
+constexpr int kNtok = 8;                 // tokens (MMA columns) per pass
+constexpr int kPrepThreads = 256;
 
-// d (16x8 f32) = A (16x16 bf16) * B (16x8 bf16) + c.
-FT_DEVICE void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                        uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+// d (16x8 s32) += A (16x32 s8) * B (32x8, s8 or u8).
+FT_DEVICE void mma_s8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+FT_DEVICE void mma_s8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Nibbles n and n+4 of w as the bf16 pair (136 + q_n, 136 + q_{n+4}).
-FT_DEVICE uint32_t nib2(uint32_t w, int n) { return ((w >> (4 * n)) & 0x000F000Fu) ^ 0x43084308u; }
-
 FT_DEVICE uint32_t word_of(const uint4& v, int j) { return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w; }
+// 16 q of the even / odd nibbles of w as four signed bytes.
+FT_DEVICE uint32_t even16q(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
+FT_DEVICE uint32_t odd16q(uint32_t w) { return w & 0xF0F0F0F0u; }
 
-// Input pairs (e_n, e_{n+4}), n = 0..3, of 8 consecutive bf16 elements held in v.
-FT_DEVICE void in_pairs(const uint4& v, uint32_t (&p)[4]) {
-  p[0] = __byte_perm(v.x, v.z, 0x5410);
-  p[1] = __byte_perm(v.x, v.z, 0x7632);
-  p[2] = __byte_perm(v.y, v.w, 0x5410);
-  p[3] = __byte_perm(v.y, v.w, 0x7632);
-}
-
-// 16-byte asynchronous copy global -> shared; bytes = 0 writes zeros and reads nothing.
 FT_DEVICE void cp16(void* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(bytes)
-               : "memory");
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(bytes) : "memory");
 }
 FT_DEVICE void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 FT_DEVICE void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Shared-memory layout of one CTA (dynamic): the scales of its rows, the partial sums of
-// its warps, and per warp a ring of kStages groups of (2 NM weight chunks + 4 input
-// chunks) x 32 lanes x 16 bytes, stored chunk-major so that a warp's 16-byte shared
-// accesses are contiguous.
+// ---------------------------------------------------------------- the inputs --
+// A sliced row of K inputs: [hi bytes: K][lo bytes: K][f: float = 2^(E - 14) / 16][12 bytes],
+// bytes in the even-then-odd order of every block of 8 elements.
+__host__ __device__ constexpr size_t sliced_row_bytes(int K) { return 2 * (size_t)K + 16; }
+
+// Block maximum of |v| over 256 threads (all call it).
+FT_DEVICE float block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float m = 0.f;
+  for (int i = 0; i < kPrepThreads / 32; ++i) m = fmaxf(m, red[i]);
+  __syncthreads();
+  return m;
+}
+
+// Writes the 8 values v (elements 8b .. 8b+7 of a row) as bytes of X = round(v * scale):
+// hi bytes (signed) and lo bytes (unsigned), even elements first.
+FT_DEVICE void slice8(const float (&v)[8], float scale, unsigned char* hi, unsigned char* lo, int b) {
+  uint32_t h[2] = {0u, 0u}, l[2] = {0u, 0u};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    int X = __float2int_rn(v[e] * scale);
+    X = max(-32767, min(32767, X));
+    const int pos = (e & 1) ? 4 + (e >> 1) : (e >> 1);   // even elements first, then odd
+    h[pos >> 2] |= (uint32_t)((X >> 8) & 0xFF) << (8 * (pos & 3));
+    l[pos >> 2] |= (uint32_t)(X & 0xFF) << (8 * (pos & 3));
+  }
+  *reinterpret_cast<uint2*>(hi + 8 * b) = make_uint2(h[0], h[1]);
+  *reinterpret_cast<uint2*>(lo + 8 * b) = make_uint2(l[0], l[1]);
+}
+
+// The T tokens of x (bf16 [T][H]) as sliced rows; grid T, kPrepThreads threads.
+__global__ void __launch_bounds__(kPrepThreads) int4_prep_x_kernel(const uint16_t* __restrict__ x, int H,
+                                                                   unsigned char* __restrict__ xs) {
+  __shared__ float red[kPrepThreads / 32];
+  const uint16_t* row = x + (size_t)blockIdx.x * H;
+  unsigned char* out = xs + (size_t)blockIdx.x * sliced_row_bytes(H);
+  float m = 0.f;
+  for (int i = threadIdx.x; i < H; i += kPrepThreads) m = fmaxf(m, fabsf(bf16_to_f32(row[i])));
+  m = block_max(m, red);
+  // E = exponent of the largest |v|; the scale 2^(14 - E) is exact, so is v * scale
+  const int E = m > 0.f ? ((int)((__float_as_uint(m) >> 23) & 0xFF) - 127) : 0;
+  const float scale = ldexpf(1.f, 14 - E);
+  for (int b = threadIdx.x; b < H / 8; b += kPrepThreads) {
+    const uint4 q = *reinterpret_cast<const uint4*>(row + 8 * b);
+    const float v[8] = {bf16lo(q.x), bf16hi(q.x), bf16lo(q.y), bf16hi(q.y),
+                        bf16lo(q.z), bf16hi(q.z), bf16lo(q.w), bf16hi(q.w)};
+    slice8(v, scale, out, out + H, b);
+  }
+  if (threadIdx.x == 0) *reinterpret_cast<float*>(out + 2 * (size_t)H) = ldexpf(1.f, E - 14) * 0.0625f;
+}
+
+// The h rows of the list's pairs (fp32 [rows][I] written by the gate/up pass), sliced in
+// place: row q becomes [hi I][lo I][f] within its 4I bytes.  Grid (n_list, rows_max).
+__global__ void __launch_bounds__(kPrepThreads) int4_prep_h_kernel(const __grid_constant__ ExpertList list, int T,
+                                                                   int k, int I, const int* __restrict__ offsets,
+                                                                   float* __restrict__ hbuf) {
+  __shared__ float red[kPrepThreads / 32];
+  extern __shared__ float vals[];   // I floats
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int e = list.expert[blockIdx.x];
+  const int q0 = e >= 0 ? offsets[e] : T * k;
+  const int n = e >= 0 ? offsets[e + 1] - q0 : T;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if ((int)blockIdx.y >= n) return;   // the same for the whole CTA
+  float* row = hbuf + (size_t)(q0 + blockIdx.y) * I;
+  float m = 0.f;
+  for (int i = threadIdx.x; i < I; i += kPrepThreads) {
+    const float v = __ldcg(row + i);
+    vals[i] = v;
+    m = fmaxf(m, fabsf(v));
+  }
+  m = block_max(m, red);   // its barriers also order every read of the row before the writes
+  const int E = m > 0.f ? ((int)((__float_as_uint(m) >> 23) & 0xFF) - 127) : 0;
+  const float scale = ldexpf(1.f, 14 - E);
+  unsigned char* out = reinterpret_cast<unsigned char*>(row);
+  for (int b = threadIdx.x; b < I / 8; b += kPrepThreads) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = vals[8 * b + i];
+    slice8(v, scale, out, out + I, b);
+  }
+  if (threadIdx.x == 0) *reinterpret_cast<float*>(out + 2 * (size_t)I) = ldexpf(1.f, E - 14) * 0.0625f;
+}
+
+// ------------------------------------------------------------------ the GEMV --
+// Per CTA: the scales of its rows, the warps' partial sums, and per warp a ring of kStages
+// groups of (2 NM weight chunks + 4 input chunks) x 32 lanes x 16 bytes (chunk-major).
 template <int NM>
 struct Int4Smem {
   static constexpr int kChunks = 2 * NM + 4;
-  __host__ __device__ static constexpr size_t ring_off() { return 0; }
   __host__ __device__ static constexpr size_t ring_bytes() { return (size_t)kQWarps * kStages * kChunks * 32 * 16; }
   __host__ __device__ static constexpr size_t red_off() { return ring_bytes(); }
   __host__ __device__ static constexpr size_t red_bytes() { return (size_t)kQWarps * NM * 16 * 8 * sizeof(float); }
   __host__ __device__ static constexpr size_t scale_off() { return red_off() + red_bytes(); }
-  __host__ __device__ static constexpr size_t bytes(int nb) { return scale_off() + (size_t)NM * 16 * nb * sizeof(uint16_t); }
+  __host__ __device__ static constexpr size_t bytes(int nb) { return scale_off() + (size_t)NM * 16 * nb * 2; }
 };
 
-// MODE 0: gate/up + SwiGLU into h (bf16 hi/lo per value); MODE 1: down into y (f32).
-// Grid (ceil(rows / rows per CTA), list.n), 128 threads, Int4Smem<NM>::bytes(nb) of dynamic
-// shared memory.
+// MODE 0: gate/up + SwiGLU into h (fp32, sliced by int4_prep_h_kernel); MODE 1: down into y.
+// xs: the sliced token rows (MODE 0).  Grid (ceil(rows / rows per CTA), list.n), 128 threads.
 template <int MODE, int NM>
 __global__ void __launch_bounds__(kQThreads)
-int4_mma_kernel(const uint16_t* __restrict__ x, int T, int H, int I, int k, const __grid_constant__ ExpertList list,
-                const int* __restrict__ offsets, const int* __restrict__ perm, float* __restrict__ hbuf,
-                float* __restrict__ ybuf) {
+int4_i8_kernel(const unsigned char* __restrict__ xs, int T, int H, int I, int k, const __grid_constant__ ExpertList list,
+               const int* __restrict__ offsets, const int* __restrict__ perm, float* __restrict__ hbuf,
+               float* __restrict__ ybuf) {
   constexpr bool GU = MODE == 0;
-  constexpr int NTOK = GU ? 8 : 4;          // tokens per pass (down: hi and lo take two columns each)
   using L = Int4Smem<NM>;
   extern __shared__ __align__(16) unsigned char smem[];
-  uint4* ring = reinterpret_cast<uint4*>(smem + L::ring_off());
+  uint4* ring = reinterpret_cast<uint4*>(smem);
   float (*red)[NM][16][8] = reinterpret_cast<float (*)[NM][16][8]>(smem + L::red_off());
   uint16_t* ssc = reinterpret_cast<uint16_t*>(smem + L::scale_off());   // [NM][16][nb]
 
@@ -145,8 +200,8 @@ int4_mma_kernel(const uint16_t* __restrict__ x, int T, int H, int I, int k, cons
   const size_t mat = (size_t)H * I;
   const uint16_t* sc = reinterpret_cast<const uint16_t*>(blob + 3 * mat / 2);
   const size_t row_bytes = (size_t)K / 2;
-  const int nb = K / 128;                                       // scale groups per row
-  // tile m: matrix wm[m], first row rbase[m]
+  const int nb = K / 128;
+  const size_t srow = sliced_row_bytes(K);   // a sliced input row (x rows; h rows are 4 I bytes apart)
   const uint8_t* wm[NM];
   int rbase[NM];
 #pragma unroll
@@ -154,7 +209,7 @@ int4_mma_kernel(const uint16_t* __restrict__ x, int T, int H, int I, int k, cons
     wm[m] = GU ? blob + (m & 1) * (mat / 2) : blob + mat;
     rbase[m] = GU ? row0 + 16 * (m >> 1) : row0 + 16 * m;
   }
-  const uint8_t* wsrcA[NM];   // this lane's rows g and g+8 of each tile (clamped to the matrix)
+  const uint8_t* wsrcA[NM];
   const uint8_t* wsrcB[NM];
 #pragma unroll
   for (int m = 0; m < NM; ++m) {
@@ -162,25 +217,22 @@ int4_mma_kernel(const uint16_t* __restrict__ x, int T, int H, int I, int k, cons
     wsrcB[m] = wm[m] + (size_t)min(rbase[m] + g + 8, rows - 1) * row_bytes + t * 16;
   }
   const int b0 = warp * nb / kQWarps, b1 = (warp + 1) * nb / kQWarps, nblk = b1 - b0;
-  uint4* myring = ring + (size_t)warp * kStages * L::kChunks * 32 + lane;   // chunk c of stage s: [(s*kChunks + c)*32]
+  uint4* myring = ring + (size_t)warp * kStages * L::kChunks * 32 + lane;
 
-  const int q0 = e >= 0 ? offsets[e] : T * k;   // offsets is written before this grid (routing)
+  const int q0 = e >= 0 ? offsets[e] : T * k;
   const int q1 = e >= 0 ? offsets[e + 1] : T * k + T;
   if (GU) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (q1 <= q0 || row0 >= rows) {                // the same for the whole CTA
+  if (q1 <= q0 || row0 >= rows) {
     if (!GU) asm volatile("griddepcontrol.wait;" ::: "memory");
     return;
   }
-
-  // scales of the CTA's rows (rows past the matrix repeat its last row; never stored)
   for (int i = threadIdx.x; i < NM * 16 * nb; i += kQThreads) {
     const int m = i / (16 * nb), r = (i / nb) % 16, b = i % nb;
     const uint16_t* sm_m = GU ? sc + (m & 1) * (mat / 128) : sc + 2 * (mat / 128);
     const int rb = GU ? row0 + 16 * (m >> 1) : row0 + 16 * m;
     ssc[i] = __ldg(sm_m + (size_t)min(rb + r, rows - 1) * nb + b);
   }
-
-  auto issue_w = [&](int i) {   // weight chunks of local group i into stage i % kStages
+  auto issue_w = [&](int i) {
     uint4* st = myring + (size_t)(i % kStages) * L::kChunks * 32;
     const size_t off = (size_t)(b0 + i) * 64;
 #pragma unroll
@@ -189,39 +241,33 @@ int4_mma_kernel(const uint16_t* __restrict__ x, int T, int H, int I, int k, cons
       cp16(st + (2 * m + 1) * 32, wsrcB[m] + off, 16);
     }
   };
-  // input chunks: 64 bytes of this lane's column for local group i (zeros where the
-  // column has no token)
-  auto issue_x = [&](int i, const uint16_t* src, bool valid) {
+  // this lane's input column, group i: 32 hi bytes (elements 32t .. 32t+31), 32 lo bytes
+  auto issue_x = [&](int i, const unsigned char* src, bool valid) {
     uint4* st = myring + (size_t)(i % kStages) * L::kChunks * 32 + 2 * NM * 32;
-    const uint16_t* p = valid ? src + (size_t)(b0 + i) * 128 + 32 * t : x;
+    const size_t off = (size_t)(b0 + i) * 128 + 32 * t;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) cp16(st + j * 32, valid ? p + 8 * j : x, valid ? 16u : 0u);
+    for (int p = 0; p < 2; ++p)
+#pragma unroll
+      for (int hl = 0; hl < 2; ++hl)
+        cp16(st + (2 * hl + p) * 32, valid ? src + (size_t)hl * K + off + 16 * p : xs, valid ? 16u : 0u);
   };
 
-  bool first_chunk = true;
-  for (int c0 = q0; c0 < q1; c0 += NTOK) {
-    const int nt = min(NTOK, q1 - c0);
-    // this lane's input column: GU token g; down hi (g < 4) or lo (g >= 4) of token g % 4
-    const int col_tok = GU ? g : (g & 3);
-    const bool valid = col_tok < nt;
-    // prologue: weight copies of the first kStages-1 groups (down: before waiting for the
-    // gate/up grid, whose h it reads), then the inputs of those groups
+  bool first = true;
+  for (int c0 = q0; c0 < q1; c0 += kNtok) {
+    const int nt = min(kNtok, q1 - c0);
+    const bool valid = g < nt;
 #pragma unroll
     for (int i = 0; i < kStages - 1; ++i) {
       if (i < nblk) issue_w(i);
       cp_commit();
     }
-    if (!GU && first_chunk) asm volatile("griddepcontrol.wait;" ::: "memory");
-    first_chunk = false;
-    const uint16_t* src = x;
+    if (!GU && first) asm volatile("griddepcontrol.wait;" ::: "memory");
+    first = false;
+    const unsigned char* src = xs;
     if (valid) {
-      const int q = c0 + col_tok;
-      if constexpr (GU) {
-        const int tok = e >= 0 ? perm[q] / k : q - T * k;
-        src = x + (size_t)tok * H;
-      } else {
-        src = reinterpret_cast<const uint16_t*>(hbuf + (size_t)q * I) + (g >> 2) * I;   // hi, or lo
-      }
+      const int q = c0 + g;
+      if constexpr (GU) src = xs + (size_t)(e >= 0 ? perm[q] / k : q - T * k) * srow;
+      else src = reinterpret_cast<const unsigned char*>(hbuf + (size_t)q * I);
     }
 #pragma unroll
     for (int i = 0; i < kStages - 1; ++i) {
@@ -233,47 +279,48 @@ int4_mma_kernel(const uint16_t* __restrict__ x, int T, int H, int I, int k, cons
     float acc[NM][4];
 #pragma unroll
     for (int m = 0; m < NM; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
-
     for (int i = 0; i < nblk; ++i) {
-      const int nx = i + kStages - 1;   // the group whose copies go out now
+      const int nx = i + kStages - 1;
       if (nx < nblk) {
         issue_w(nx);
         issue_x(nx, src, valid);
       }
       cp_commit();
-      cp_wait<kStages - 1>();           // group i has landed (this lane's copies)
+      cp_wait<kStages - 1>();
       const uint4* st = myring + (size_t)(i % kStages) * L::kChunks * 32;
-      uint4 wa[NM], wb[NM], xv[4];
+      uint4 wa[NM], wb[NM], xh[2], xl[2];
 #pragma unroll
       for (int m = 0; m < NM; ++m) { wa[m] = st[(2 * m) * 32]; wb[m] = st[(2 * m + 1) * 32]; }
+      xh[0] = st[(2 * NM + 0) * 32]; xh[1] = st[(2 * NM + 1) * 32];
+      xl[0] = st[(2 * NM + 2) * 32]; xl[1] = st[(2 * NM + 3) * 32];
+      int dh[NM][4], dl[NM][4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) xv[j] = st[(2 * NM + j) * 32];
-      float d[NM][4], db[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int m = 0; m < NM; ++m)
 #pragma unroll
-      for (int m = 0; m < NM; ++m) d[m][0] = d[m][1] = d[m][2] = d[m][3] = 0.f;
+        for (int r = 0; r < 4; ++r) dh[m][r] = dl[m][r] = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        uint32_t b[4];
-        in_pairs(xv[j], b);
+        // B of MMA j: this lane's 8 input bytes of word j (even elements, then odd ones)
+        const uint32_t bh0 = word_of(xh[j >> 1], 2 * (j & 1)), bh1 = word_of(xh[j >> 1], 2 * (j & 1) + 1);
+        const uint32_t bl0 = word_of(xl[j >> 1], 2 * (j & 1)), bl1 = word_of(xl[j >> 1], 2 * (j & 1) + 1);
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
           const uint32_t a = word_of(wa[m], j), c = word_of(wb[m], j);
-          mma16816(d[m], nib2(a, 0), nib2(c, 0), nib2(a, 1), nib2(c, 1), b[0], b[1]);
-          mma16816(d[m], nib2(a, 2), nib2(c, 2), nib2(a, 3), nib2(c, 3), b[2], b[3]);
+          const uint32_t a0 = even16q(a), a1 = even16q(c), a2 = odd16q(a), a3 = odd16q(c);
+          mma_s8s8(dh[m], a0, a1, a2, a3, bh0, bh1);
+          mma_s8u8(dl[m], a0, a1, a2, a3, bl0, bl1);
         }
-        mma16816(db, kNeg136x2, kNeg136x2, kNeg136x2, kNeg136x2, b[0], b[1]);
-        mma16816(db, kNeg136x2, kNeg136x2, kNeg136x2, kNeg136x2, b[2], b[3]);
       }
-      // d: rows g (d[0], d[1]) and g+8 (d[2], d[3]), columns 2t and 2t+1
+      // dh/dl: rows g (0, 1) and g+8 (2, 3), columns 2t and 2t+1
       const int blk = b0 + i;
 #pragma unroll
       for (int m = 0; m < NM; ++m) {
         const float s0 = bf16_to_f32(ssc[(m * 16 + g) * nb + blk]);
         const float s1 = bf16_to_f32(ssc[(m * 16 + g + 8) * nb + blk]);
-        acc[m][0] = fmaf(s0, d[m][0] + db[0], acc[m][0]);
-        acc[m][1] = fmaf(s0, d[m][1] + db[1], acc[m][1]);
-        acc[m][2] = fmaf(s1, d[m][2] + db[2], acc[m][2]);
-        acc[m][3] = fmaf(s1, d[m][3] + db[3], acc[m][3]);
+        acc[m][0] = fmaf(s0, (float)(256 * dh[m][0] + dl[m][0]), acc[m][0]);
+        acc[m][1] = fmaf(s0, (float)(256 * dh[m][1] + dl[m][1]), acc[m][1]);
+        acc[m][2] = fmaf(s1, (float)(256 * dh[m][2] + dl[m][2]), acc[m][2]);
+        acc[m][3] = fmaf(s1, (float)(256 * dh[m][3] + dl[m][3]), acc[m][3]);
       }
     }
     cp_wait<0>();
@@ -286,28 +333,26 @@ int4_mma_kernel(const uint16_t* __restrict__ x, int T, int H, int I, int k, cons
     }
     __syncthreads();
     {
-      const int r = threadIdx.x >> 3, col = threadIdx.x & 7;   // 128 threads: one (row, column) of a tile
+      const int r = threadIdx.x >> 3, col = threadIdx.x & 7;   // one (row, column) of a tile per thread
       auto wsum = [&](int m, int cc) {
         return ((red[0][m][r][cc] + red[1][m][r][cc]) + red[2][m][r][cc]) + red[3][m][r][cc];
       };
-      if constexpr (GU) {
+      if (col < nt) {
+        const int q = c0 + col;
+        // the column's input row: 2^(E - 14) / 16 after its bytes
+        const float f = GU ? *reinterpret_cast<const float*>(xs + (size_t)(e >= 0 ? perm[q] / k : q - T * k) * srow + 2 * (size_t)K)
+                           : __ldcg(reinterpret_cast<const float*>(reinterpret_cast<const unsigned char*>(hbuf + (size_t)q * I) + 2 * (size_t)K));
+        if constexpr (GU) {
 #pragma unroll
-        for (int p = 0; p < NM / 2; ++p) {
-          const int row = rbase[2 * p] + r;
-          if (col < nt && row < rows) {
-            const float hv = silu(wsum(2 * p, col)) * wsum(2 * p + 1, col);
-            const uint16_t hi = f32_to_bf16(hv);
-            uint16_t* hrow = reinterpret_cast<uint16_t*>(hbuf + (size_t)(c0 + col) * I);
-            hrow[row] = hi;
-            hrow[I + row] = f32_to_bf16(hv - bf16_to_f32(hi));
+          for (int p = 0; p < NM / 2; ++p) {
+            const int row = rbase[2 * p] + r;
+            if (row < rows) hbuf[(size_t)q * I + row] = silu(wsum(2 * p, col) * f) * (wsum(2 * p + 1, col) * f);
           }
-        }
-      } else {
-        if (col < nt) {
+        } else {
 #pragma unroll
           for (int m = 0; m < NM; ++m) {
             const int row = rbase[m] + r;
-            if (row < rows) ybuf[(size_t)(c0 + col) * H + row] = wsum(m, col) + wsum(m, col + 4);
+            if (row < rows) ybuf[(size_t)q * H + row] = wsum(m, col) * f;
           }
         }
       }
@@ -317,13 +362,15 @@ int4_mma_kernel(const uint16_t* __restrict__ x, int T, int H, int I, int k, cons
 }
 
 template <typename... KArgs, typename... Args>
-cudaError_t launch_smem(void (*kern)(KArgs...), dim3 grid, size_t smem, cudaStream_t s, bool dependent,
-                        Args... args) {
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool dependent,
+                      Args... args) {
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kQThreads);
+  cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -336,20 +383,34 @@ cudaError_t launch_smem(void (*kern)(KArgs...), dim3 grid, size_t smem, cudaStre
 
 }  // namespace
 
+size_t int4_sliced_x_bytes(int T, int H) { return (size_t)T * sliced_row_bytes(H); }
+
 cudaError_t launch_ffn_int4_mma(const void* x, int T, int H, int I, int k, const ExpertList& list, const int* offsets,
                                 const int* perm, float* h, float* y, cudaStream_t s, cudaEvent_t between,
-                                int /*max_pairs_per_expert*/) {
+                                int max_pairs_per_expert, void* xsliced) {
   if (list.n <= 0 || T <= 0) return cudaSuccess;
   if (H % 128 || I % 128) return cudaErrorInvalidValue;
-  const uint16_t* xb = static_cast<const uint16_t*>(x);
-  const unsigned gu_ctas = (unsigned)((I + 16 * (kGuTiles / 2) - 1) / (16 * (kGuTiles / 2)));
-  cudaError_t e = launch_smem(int4_mma_kernel<0, kGuTiles>, dim3(gu_ctas, list.n), Int4Smem<kGuTiles>::bytes(H / 128),
-                              s, false, xb, T, H, I, k, list, offsets, perm, h, y);
+  // the sliced tokens go to xsliced, or to the front of y (y is written only by the down pass,
+  // after the gate/up pass has read them)
+  unsigned char* xs = static_cast<unsigned char*>(xsliced ? xsliced : static_cast<void*>(y));
+  cudaError_t e = launch_ex(int4_prep_x_kernel, dim3(T), dim3(kPrepThreads), 0, s, false,
+                            static_cast<const uint16_t*>(x), H, xs);
+  if (e != cudaSuccess) return e;
+  e = launch_ex(int4_i8_kernel<0, 2>, dim3(I / 16, list.n), dim3(kQThreads), Int4Smem<2>::bytes(H / 128), s, false,
+                static_cast<const unsigned char*>(xs), T, H, I, k, list, offsets, perm, h, y);
   if (e != cudaSuccess) return e;
   if (between) cudaEventRecord(between, s);
+  int has_shared = 0;
+  for (int i = 0; i < list.n; ++i) has_shared |= list.expert[i] < 0;
+  int rows_max = max_pairs_per_expert < 1 ? T * k : max_pairs_per_expert;
+  if (has_shared && T > rows_max) rows_max = T;
+  e = launch_ex(int4_prep_h_kernel, dim3(list.n, rows_max), dim3(kPrepThreads), (size_t)I * sizeof(float), s, true,
+                list, T, k, I, offsets, h);
+  if (e != cudaSuccess) return e;
   const unsigned down_ctas = (unsigned)((H + 16 * kDownTiles - 1) / (16 * kDownTiles));
-  return launch_smem(int4_mma_kernel<1, kDownTiles>, dim3(down_ctas, list.n), Int4Smem<kDownTiles>::bytes(I / 128),
-                     s, true, xb, T, H, I, k, list, offsets, perm, h, y);
+  return launch_ex(int4_i8_kernel<1, kDownTiles>, dim3(down_ctas, list.n), dim3(kQThreads),
+                   Int4Smem<kDownTiles>::bytes(I / 128), s, true, static_cast<const unsigned char*>(xs), T, H, I, k,
+                   list, offsets, perm, h, y);
 }
 
 }  // namespace ftk

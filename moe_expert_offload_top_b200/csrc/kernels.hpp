@@ -43,18 +43,26 @@ cudaError_t launch_permute(const int* ids, int T, int k, int E, int* counts, int
 // K3 (decode): per list entry, gate/up + SwiGLU of its tokens into h [pairs][I] fp32,
 // then the down projection into y [pairs][H] fp32.  Pairs are positions in the
 // permutation (routed) or T*k + t (shared expert).  `between` (optional) is recorded
-// on s between the two launches.
-// int4 weights run on the tensor cores (launch_ffn_int4_mma) unless int4_tensor is false;
-// h then holds each value as bf16 hi and lo halves (the row's first and second I uint16).
+// on s between the gate/up and the down passes.
+// int4 weights run on the int8 tensor cores (launch_ffn_int4_mma) unless int4_tensor is
+// false; the h rows of the list's pairs are then left as sliced inputs (see below), and
+// int4_xs (int4_sliced_x_bytes(T, H) bytes) receives the sliced tokens, or, when null, the
+// front of y does (before the down pass writes y).
 cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdtype,
                               const ExpertList& list, int max_pairs_per_expert, const int* offsets,
                               const int* perm, float* h, float* y, cudaStream_t s,
-                              cudaEvent_t between = nullptr, int* err = nullptr, bool int4_tensor = true);
-// K3 (decode) for int4 group-128 weights with mma.sync (gemv_int4_mma.cu); x bf16.
-// max_pairs_per_expert: the most pairs one entry owns (sizes per-CTA input staging).
+                              cudaEvent_t between = nullptr, int* err = nullptr, bool int4_tensor = true,
+                              void* int4_xs = nullptr);
+// K3 (decode) for int4 group-128 weights on the int8 tensor cores (gemv_int4_mma.cu); x bf16.
+// The tokens and, after the gate/up pass, the h rows of the list's pairs are written as
+// 16-bit block fixed point split into a signed and an unsigned byte per value (a sliced row:
+// hi bytes, lo bytes, then a float), the tokens into xsliced (or the front of y when null), the
+// h rows in place.  max_pairs_per_expert: the most pairs one entry owns.
 cudaError_t launch_ffn_int4_mma(const void* x, int T, int H, int I, int k, const ExpertList& list, const int* offsets,
                                 const int* perm, float* h, float* y, cudaStream_t s, cudaEvent_t between,
-                                int max_pairs_per_expert);
+                                int max_pairs_per_expert, void* xsliced);
+// Bytes of the sliced tokens of launch_ffn_int4_mma.
+size_t int4_sliced_x_bytes(int T, int H);
 // K3 + K5 (decode) in one launch (ffn_fused.cuh): gate/up + SwiGLU into h, down into y
 // and, with `combine`, out[t] = sum_j gates[t][j] * y[inv[t*k+j]] (+ shared) for the
 // entries of `list`.  The combine of a launch covers every pair of the forward, so

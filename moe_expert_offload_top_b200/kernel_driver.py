@@ -1,7 +1,7 @@
 """Runs a named workload at reduced size through the C ABI, for kernel profiling.
 
     python -m moe_expert_offload_top_b200.kernel_driver --workload NAME
-        [--layers L] [--experts E] [--slots C] [--steps S] [--batch B] [--tokens T]
+        [--layers L] [--experts E] [--slots C] [--steps S] [--batch B] [--tokens T] [--wdtype W] [--perf]
 
 The workload keeps its shapes (hidden, intermediate, top-k, gating, weight format,
 shared expert) and token process; --layers / --experts shrink the pool so that a
@@ -33,6 +33,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=12)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--tokens", type=int, default=None, help="prefill: tokens per forward")
+    ap.add_argument("--wdtype", default=None, choices=["f32", "bf16", "int4", "nvfp4"],
+                    help="another weight format for the workload's shapes")
     ap.add_argument("--perf", action="store_true",
                     help="stage timing on: also print the algorithmic bytes and flops per FFN launch")
     a = ap.parse_args(argv)
@@ -43,7 +45,7 @@ def main(argv=None):
     T = (a.tokens or base.tokens) if prefill else a.batch
     n_tok = T * a.steps if prefill else max(base.tokens, T * a.steps)
     cfg = dataclasses.replace(base, L=a.layers, E=E, k=k, C=a.slots or a.layers * E, tokens=n_tok,
-                              batches=(T,), resize_to=None)
+                              batches=(T,), resize_to=None, wdtype=a.wdtype or base.wdtype)
     with GpuStack(cfg, max_tokens=T) as st:
         vals, x = st.tokens(T)
         out = torch.empty((cfg.L, T, cfg.H), dtype=st.xdt, device=st.device)

@@ -121,3 +121,69 @@ def test_nvfp4_expansion_element_order():
             assert [32 * hf + e for e in elems] == list(range(8 * c, 8 * c + 8))
             block = 2 * hf + (0 if j < 2 else 1)
             assert all((32 * hf + e) // 16 == block for e in elems)
+
+
+def test_int4_nibbles_as_signed_bytes_16q():
+    # The int8 tensor-core GEMV: (w << 4) & 0xF0F0F0F0 puts the even nibbles, w & 0xF0F0F0F0 the
+    # odd ones, in the high halves of four bytes; read as signed int8 each byte is 16 q for the
+    # two's-complement nibble q of its element (element 2i: low nibble of byte i).
+    rng = np.random.default_rng(3)
+    words = np.concatenate([rng.integers(0, 2 ** 32, 8192, dtype=np.uint64).astype(np.uint32),
+                            np.array([0, 0xFFFFFFFF, 0x88888888, 0x77777777, 0x80808080], dtype=np.uint32)])
+    even = ((words.astype(np.uint64) << 4) & 0xF0F0F0F0).astype(np.uint32)
+    odd = words & np.uint32(0xF0F0F0F0)
+    nib = np.stack([(words >> np.uint32(4 * e)) & np.uint32(15) for e in range(8)], axis=1).astype(np.int64)
+    q = np.where(nib >= 8, nib - 16, nib)                       # element e of the word
+    ev_bytes = even.view(np.int8).reshape(-1, 4).astype(np.int64)   # little-endian: byte i
+    od_bytes = odd.view(np.int8).reshape(-1, 4).astype(np.int64)
+    assert np.array_equal(ev_bytes, 16 * q[:, 0::2])
+    assert np.array_equal(od_bytes, 16 * q[:, 1::2])
+
+
+def _slice_rows(v):
+    # the prep kernels' rule: E = exponent of max |v|, X = rint(v * 2^(14 - E)) clamped to
+    # +-32767, hi = X >> 8 (signed), lo = X & 255, f = 2^(E - 14) / 16
+    m = np.max(np.abs(v))
+    E = int(np.frexp(np.float32(m))[1]) - 1 if m > 0 else 0
+    X = np.clip(np.rint(v.astype(np.float64) * 2.0 ** (14 - E)), -32767, 32767).astype(np.int64)
+    return X, X >> 8, X & 255, E
+
+
+def test_int4_input_slices_block_fixed_point():
+    rng = np.random.default_rng(4)
+    for trial in range(20):
+        scale = 10.0 ** rng.uniform(-6, 6)
+        v = synth.round_bf16((rng.standard_normal(7168) * scale).astype(np.float32))
+        v = _bf16_bits_to_f32(v).astype(np.float64)
+        v[rng.integers(0, 7168, 5)] *= 0.0                          # exact zeros too
+        X, hi, lo, E = _slice_rows(v)
+        assert np.all(hi >= -128) and np.all(hi <= 127) and np.all(lo >= 0) and np.all(lo <= 255)
+        assert np.array_equal(256 * hi + lo, X)                     # the two bytes rebuild X
+        back = X * 2.0 ** (E - 14)
+        big = np.abs(v) >= 2.0 ** (E - 7)                           # within 2^7 of the largest
+        assert np.array_equal(back[big], v[big])                    # bf16 inputs there are exact
+        assert np.max(np.abs(back - v)) <= 2.0 ** (E - 15)          # any input: half a step
+    # fp32 inputs (h): the error of every element is at most half a step of 2^(E - 14)
+    h = rng.standard_normal(2048) * 3.7
+    X, hi, lo, E = _slice_rows(h)
+    assert np.max(np.abs(X * 2.0 ** (E - 14) - h)) <= 2.0 ** (E - 15)
+
+
+def test_int4_int8_mma_accumulators_fit_int32():
+    # one 128-element group: 4 MMAs of 32 products each into int32; the largest |16 q| is 128,
+    # the largest |hi| 128 and lo 255, so |256 D_hi + D_lo| < 2^31, and float(S) keeps 24 bits
+    d_hi = 128 * 128 * 128
+    d_lo = 128 * 128 * 255
+    assert 256 * d_hi + d_lo < 2 ** 31
+
+
+def test_int4_slice_permutation_matches_the_fragment_order():
+    # MMA j of a group takes, per lane t, A = even16q / odd16q of word j (elements 32t + 8j +
+    # {0,2,4,6} and +{1,3,5,7}); the sliced input stores every block of 8 elements even-first,
+    # so bytes 0-3 of block j are elements {0,2,4,6} and bytes 4-7 are {1,3,5,7}
+    def pos(e):
+        return e >> 1 if e % 2 == 0 else 4 + (e >> 1)
+    order = [None] * 8
+    for e in range(8):
+        order[pos(e)] = e
+    assert order == [0, 2, 4, 6, 1, 3, 5, 7]
