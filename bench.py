@@ -463,7 +463,8 @@ def int4_leg(args, dev, peaks, peak_src, link_h2d):
                        "h2d_bytes_per_step": r["h2d_bytes_per_step"], "d2h_bytes_per_step": r["d2h_bytes_per_step"]},
                "gpu_launches": int(r["perf_dev"]["kernel_launches"]), "clocks": r["clocks"],
                "roofline": gemv_roofline(r["perf"], peaks, peak_src, "gemv_int4",
-                                         "int4_mma_kernel<0> (int4 g128 expert gate/up + SwiGLU, mma.sync, decode)"),
+                                         "int4_prep_x_kernel + int4_i8_kernel<0> (int4 g128 expert gate/up + SwiGLU, "
+                                         "int8 mma.sync m16n8k32, decode)"),
                "cache": cache_summary(r["st"], link_h2d),
                "cold_start": {"value": args.warmup / r["cold_dt"], "unit": "tokens/s",
                               "miss_rate": r["cold_st"]["misses"] / max(r["cold_st"]["routed"], 1)},

@@ -25,12 +25,14 @@
 // is therefore a permutation of the physical one, and the inputs are stored in the same
 // permutation: in every block of 8 elements, the even ones first, then the odd ones.
 //
-// Memory pipeline (as before): every lane copies the bytes it uses itself (16 bytes of
-// rows g and g+8 of each tile, 32 + 32 bytes of its input column's hi and lo bytes) into
-// its own slots of a shared-memory ring with cp.async, kStages - 1 groups ahead; the down
-// pass copies its weights before griddepcontrol.wait.  Scales of the CTA's rows are staged
-// in shared memory once.  The 4 warps of a CTA split the reduction axis and add their
-// partial sums in warp order.
+// Memory pipeline: every lane copies the bytes it uses itself (16 bytes of rows g and g+8
+// of each tile; for the lanes of a token column, 32 + 32 bytes of its hi and lo bytes) into
+// its own slots of a shared-memory ring with cp.async, S - 1 groups ahead.  A stage holds
+// the weight chunks and the input bytes of only the columns the launch uses (ncols <= 8,
+// the most pairs of one expert), so that at batch 1 nearly all of the ring is weights; S
+// is chosen per launch so that four CTAs fit on an SM.  The down pass copies its weights
+// before griddepcontrol.wait.  Scales of the CTA's rows are staged in shared memory once.
+// The 4 warps of a CTA split the reduction axis and add their partial sums in warp order.
 #include "decode_gemv.cuh"
 #include "sm100_sync.cuh"
 
@@ -42,13 +44,9 @@ using namespace gemv;
 
 constexpr int kQWarps = 4;
 constexpr int kQThreads = 32 * kQWarps;
-#ifndef FT_INT4_STAGES
-#define FT_INT4_STAGES 4
-#endif
 #ifndef FT_INT4_DOWN_TILES
 #define FT_INT4_DOWN_TILES 2
 #endif
-constexpr int kStages = FT_INT4_STAGES;
 constexpr int kDownTiles = FT_INT4_DOWN_TILES;
 constexpr int kNtok = 8;                 // tokens (MMA columns) per pass
 constexpr int kPrepThreads = 256;
@@ -70,8 +68,18 @@ FT_DEVICE uint32_t word_of(const uint4& v, int j) { return j == 0 ? v.x : j == 1
 FT_DEVICE uint32_t even16q(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
 FT_DEVICE uint32_t odd16q(uint32_t w) { return w & 0xF0F0F0F0u; }
 
-FT_DEVICE void cp16(void* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(bytes) : "memory");
+FT_DEVICE void cp16s(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+FT_DEVICE uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+FT_DEVICE uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
 }
 FT_DEVICE void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -114,6 +122,7 @@ FT_DEVICE void slice8(const float (&v)[8], float scale, unsigned char* hi, unsig
 __global__ void __launch_bounds__(kPrepThreads) int4_prep_x_kernel(const uint16_t* __restrict__ x, int H,
                                                                    unsigned char* __restrict__ xs) {
   __shared__ float red[kPrepThreads / 32];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the gate/up pass's weight copies
   const uint16_t* row = x + (size_t)blockIdx.x * H;
   unsigned char* out = xs + (size_t)blockIdx.x * sliced_row_bytes(H);
   float m = 0.f;
@@ -165,31 +174,37 @@ __global__ void __launch_bounds__(kPrepThreads) int4_prep_h_kernel(const __grid_
 }
 
 // ------------------------------------------------------------------ the GEMV --
-// Per CTA: the scales of its rows, the warps' partial sums, and per warp a ring of kStages
-// groups of (2 NM weight chunks + 4 input chunks) x 32 lanes x 16 bytes (chunk-major).
-template <int NM>
+// Per CTA: per warp a ring of S stages, then the warps' partial sums, then the scales of
+// its rows (per group and tile, the bf16 scales of rows g and g+8 in one word).  A stage is 2 NM weight chunks x 32 lanes x 16 bytes (chunk-major), then the
+// input bytes of ncols columns, 256 bytes each: pieces 0-7 the 128 hi bytes of the group,
+// 8-15 the lo bytes, piece p of column c at slot p ^ c so that the 8 columns' lanes read
+// without bank conflicts.
+template <int NM, int S>
 struct Int4Smem {
-  static constexpr int kChunks = 2 * NM + 4;
-  __host__ __device__ static constexpr size_t ring_bytes() { return (size_t)kQWarps * kStages * kChunks * 32 * 16; }
-  __host__ __device__ static constexpr size_t red_off() { return ring_bytes(); }
+  __host__ __device__ static constexpr size_t wbytes() { return (size_t)2 * NM * 32 * 16; }
+  __host__ __device__ static constexpr size_t stage_bytes(int ncols) { return wbytes() + (size_t)ncols * 256; }
+  __host__ __device__ static constexpr size_t red_off(int ncols) { return (size_t)kQWarps * S * stage_bytes(ncols); }
   __host__ __device__ static constexpr size_t red_bytes() { return (size_t)kQWarps * NM * 16 * 8 * sizeof(float); }
-  __host__ __device__ static constexpr size_t scale_off() { return red_off() + red_bytes(); }
-  __host__ __device__ static constexpr size_t bytes(int nb) { return scale_off() + (size_t)NM * 16 * nb * 2; }
+  __host__ __device__ static constexpr size_t scale_off(int ncols) { return red_off(ncols) + red_bytes(); }
+  __host__ __device__ static constexpr size_t bytes(int nb, int ncols) {
+    return scale_off(ncols) + (size_t)NM * 16 * nb * 2;
+  }
 };
 
 // MODE 0: gate/up + SwiGLU into h (fp32, sliced by int4_prep_h_kernel); MODE 1: down into y.
-// xs: the sliced token rows (MODE 0).  Grid (ceil(rows / rows per CTA), list.n), 128 threads.
-template <int MODE, int NM>
-__global__ void __launch_bounds__(kQThreads)
+// xs: the sliced token rows (MODE 0).  ncols (1..8): token columns per pass, at least the
+// most pairs of any listed expert for one pass per expert.  Grid (ceil(rows / rows per CTA),
+// list.n), 128 threads, Int4Smem<NM, S>::bytes(K / 128, ncols) bytes of shared memory.
+template <int MODE, int NM, int S>
+__global__ void __launch_bounds__(kQThreads, 4)
 int4_i8_kernel(const unsigned char* __restrict__ xs, int T, int H, int I, int k, const __grid_constant__ ExpertList list,
                const int* __restrict__ offsets, const int* __restrict__ perm, float* __restrict__ hbuf,
-               float* __restrict__ ybuf) {
+               float* __restrict__ ybuf, int ncols) {
   constexpr bool GU = MODE == 0;
-  using L = Int4Smem<NM>;
+  using L = Int4Smem<NM, S>;
   extern __shared__ __align__(16) unsigned char smem[];
-  uint4* ring = reinterpret_cast<uint4*>(smem);
-  float (*red)[NM][16][8] = reinterpret_cast<float (*)[NM][16][8]>(smem + L::red_off());
-  uint16_t* ssc = reinterpret_cast<uint16_t*>(smem + L::scale_off());   // [NM][16][nb]
+  float (*red)[NM][16][8] = reinterpret_cast<float (*)[NM][16][8]>(smem + L::red_off(ncols));
+  uint32_t* ssc = reinterpret_cast<uint32_t*>(smem + L::scale_off(ncols));   // [nb][NM][8]: rows g | g+8 << 16
 
   const int e = list.expert[blockIdx.y];
   const uint8_t* blob = list.blob[blockIdx.y];
@@ -202,66 +217,64 @@ int4_i8_kernel(const unsigned char* __restrict__ xs, int T, int H, int I, int k,
   const size_t row_bytes = (size_t)K / 2;
   const int nb = K / 128;
   const size_t srow = sliced_row_bytes(K);   // a sliced input row (x rows; h rows are 4 I bytes apart)
-  const uint8_t* wm[NM];
-  int rbase[NM];
-#pragma unroll
-  for (int m = 0; m < NM; ++m) {
-    wm[m] = GU ? blob + (m & 1) * (mat / 2) : blob + mat;
-    rbase[m] = GU ? row0 + 16 * (m >> 1) : row0 + 16 * m;
-  }
-  const uint8_t* wsrcA[NM];
-  const uint8_t* wsrcB[NM];
-#pragma unroll
-  for (int m = 0; m < NM; ++m) {
-    wsrcA[m] = wm[m] + (size_t)min(rbase[m] + g, rows - 1) * row_bytes + t * 16;
-    wsrcB[m] = wm[m] + (size_t)min(rbase[m] + g + 8, rows - 1) * row_bytes + t * 16;
-  }
   const int b0 = warp * nb / kQWarps, b1 = (warp + 1) * nb / kQWarps, nblk = b1 - b0;
-  uint4* myring = ring + (size_t)warp * kStages * L::kChunks * 32 + lane;
+  int rbase[NM];
+  const uint8_t* wsrc[2 * NM];   // this lane's 16 bytes of rows g ([2m]) and g+8 ([2m+1]) of tile m, group b0
+#pragma unroll
+  for (int m = 0; m < NM; ++m) {
+    const uint8_t* wm = GU ? blob + (m & 1) * (mat / 2) : blob + mat;
+    rbase[m] = GU ? row0 + 16 * (m >> 1) : row0 + 16 * m;
+    wsrc[2 * m] = wm + (size_t)min(rbase[m] + g, rows - 1) * row_bytes + t * 16 + (size_t)b0 * 64;
+    wsrc[2 * m + 1] = wm + (size_t)min(rbase[m] + g + 8, rows - 1) * row_bytes + t * 16 + (size_t)b0 * 64;
+  }
+  // shared addresses: weight chunk c of stage st at ring_w + st * sbytes + 512 c; piece p of
+  // input column c at ring_x + st * sbytes + 256 c + 16 (p ^ c)
+  const uint32_t sbytes = (uint32_t)L::stage_bytes(ncols);
+  const uint32_t ring_w = smem_u32(smem) + (uint32_t)warp * S * sbytes + (uint32_t)lane * 16;
+  const uint32_t ring_x = smem_u32(smem) + (uint32_t)warp * S * sbytes + (uint32_t)L::wbytes();
+  const uint32_t ssc_s = smem_u32(ssc) + (uint32_t)g * 4;
 
   const int q0 = e >= 0 ? offsets[e] : T * k;
   const int q1 = e >= 0 ? offsets[e + 1] : T * k + T;
   if (GU) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (q1 <= q0 || row0 >= rows) {
-    if (!GU) asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     return;
   }
-  for (int i = threadIdx.x; i < NM * 16 * nb; i += kQThreads) {
-    const int m = i / (16 * nb), r = (i / nb) % 16, b = i % nb;
+  for (int i = threadIdx.x; i < nb * NM * 8; i += kQThreads) {
+    const int b = i / (NM * 8), m = (i / 8) % NM, r = i % 8;
     const uint16_t* sm_m = GU ? sc + (m & 1) * (mat / 128) : sc + 2 * (mat / 128);
     const int rb = GU ? row0 + 16 * (m >> 1) : row0 + 16 * m;
-    ssc[i] = __ldg(sm_m + (size_t)min(rb + r, rows - 1) * nb + b);
+    const uint32_t s_lo = __ldg(sm_m + (size_t)min(rb + r, rows - 1) * nb + b);
+    const uint32_t s_hi = __ldg(sm_m + (size_t)min(rb + r + 8, rows - 1) * nb + b);
+    ssc[i] = s_lo | (s_hi << 16);
   }
-  auto issue_w = [&](int i) {
-    uint4* st = myring + (size_t)(i % kStages) * L::kChunks * 32;
-    const size_t off = (size_t)(b0 + i) * 64;
+  auto issue_w = [&](int i, uint32_t st_off) {
 #pragma unroll
-    for (int m = 0; m < NM; ++m) {
-      cp16(st + (2 * m) * 32, wsrcA[m] + off, 16);
-      cp16(st + (2 * m + 1) * 32, wsrcB[m] + off, 16);
-    }
+    for (int c = 0; c < 2 * NM; ++c) cp16s(ring_w + st_off + 512 * c, wsrc[c] + (size_t)i * 64);
   };
-  // this lane's input column, group i: 32 hi bytes (elements 32t .. 32t+31), 32 lo bytes
-  auto issue_x = [&](int i, const unsigned char* src, bool valid) {
-    uint4* st = myring + (size_t)(i % kStages) * L::kChunks * 32 + 2 * NM * 32;
-    const size_t off = (size_t)(b0 + i) * 128 + 32 * t;
-#pragma unroll
-    for (int p = 0; p < 2; ++p)
-#pragma unroll
-      for (int hl = 0; hl < 2; ++hl)
-        cp16(st + (2 * hl + p) * 32, valid ? src + (size_t)hl * K + off + 16 * p : xs, valid ? 16u : 0u);
+  // the input column of lane g, group b0 + i: 32 hi bytes (elements 32t .. 32t+31), 32 lo bytes
+  const uint32_t xo[4] = {(uint32_t)(g * 256 + 16 * ((2 * t) ^ g)), (uint32_t)(g * 256 + 16 * ((2 * t + 1) ^ g)),
+                          (uint32_t)(g * 256 + 16 * ((8 + 2 * t) ^ g)), (uint32_t)(g * 256 + 16 * ((9 + 2 * t) ^ g))};
+  auto issue_x = [&](int i, uint32_t st_off, const unsigned char* src) {
+    const unsigned char* p = src + (size_t)(b0 + i) * 128 + 32 * t;
+    cp16s(ring_x + st_off + xo[0], p);
+    cp16s(ring_x + st_off + xo[1], p + 16);
+    cp16s(ring_x + st_off + xo[2], p + K);
+    cp16s(ring_x + st_off + xo[3], p + K + 16);
   };
 
   bool first = true;
-  for (int c0 = q0; c0 < q1; c0 += kNtok) {
-    const int nt = min(kNtok, q1 - c0);
+  for (int c0 = q0; c0 < q1; c0 += ncols) {
+    const int nt = min(ncols, q1 - c0);
     const bool valid = g < nt;
-#pragma unroll
-    for (int i = 0; i < kStages - 1; ++i) {
-      if (i < nblk) issue_w(i);
+#pragma unroll 1
+    for (int i = 0; i < S - 1; ++i) {
+      if (i < nblk) issue_w(i, i * sbytes);
       cp_commit();
     }
-    if (!GU && first) asm volatile("griddepcontrol.wait;" ::: "memory");
+    // before this point: only the weights, scales and routing (ready before the kernel before)
+    if (first) asm volatile("griddepcontrol.wait;" ::: "memory");
     first = false;
     const unsigned char* src = xs;
     if (valid) {
@@ -269,30 +282,38 @@ int4_i8_kernel(const unsigned char* __restrict__ xs, int T, int H, int I, int k,
       if constexpr (GU) src = xs + (size_t)(e >= 0 ? perm[q] / k : q - T * k) * srow;
       else src = reinterpret_cast<const unsigned char*>(hbuf + (size_t)q * I);
     }
-#pragma unroll
-    for (int i = 0; i < kStages - 1; ++i) {
-      if (i < nblk) issue_x(i, src, valid);
+#pragma unroll 1
+    for (int i = 0; i < S - 1; ++i) {
+      if (valid && i < nblk) issue_x(i, i * sbytes, src);
       cp_commit();
     }
     __syncthreads();   // the scales are staged
+    // lanes past the pass's columns read column 0 (copied by lanes 0-3); their MMA columns are
+    // discarded
+    const int gx = valid ? g : 0;
+    const uint32_t xr0 = ring_x + gx * 256 + 16 * ((2 * t) ^ gx), xr1 = ring_x + gx * 256 + 16 * ((2 * t + 1) ^ gx);
+    const uint32_t xr2 = ring_x + gx * 256 + 16 * ((8 + 2 * t) ^ gx), xr3 = ring_x + gx * 256 + 16 * ((9 + 2 * t) ^ gx);
 
     float acc[NM][4];
 #pragma unroll
     for (int m = 0; m < NM; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
+    uint32_t st_off = 0, wst_off = (S - 1) * sbytes;
+    const uint32_t ring_bytes = S * sbytes;
+#pragma unroll 1
     for (int i = 0; i < nblk; ++i) {
-      const int nx = i + kStages - 1;
+      const int nx = i + S - 1;
       if (nx < nblk) {
-        issue_w(nx);
-        issue_x(nx, src, valid);
+        issue_w(nx, wst_off);
+        if (valid) issue_x(nx, wst_off, src);
       }
       cp_commit();
-      cp_wait<kStages - 1>();
-      const uint4* st = myring + (size_t)(i % kStages) * L::kChunks * 32;
-      uint4 wa[NM], wb[NM], xh[2], xl[2];
+      cp_wait<S - 1>();
+      __syncwarp();   // lanes 0-3's input copies are complete for the lanes that read them
+      uint4 wv[2 * NM];
 #pragma unroll
-      for (int m = 0; m < NM; ++m) { wa[m] = st[(2 * m) * 32]; wb[m] = st[(2 * m + 1) * 32]; }
-      xh[0] = st[(2 * NM + 0) * 32]; xh[1] = st[(2 * NM + 1) * 32];
-      xl[0] = st[(2 * NM + 2) * 32]; xl[1] = st[(2 * NM + 3) * 32];
+      for (int c = 0; c < 2 * NM; ++c) wv[c] = lds128(ring_w + st_off + 512 * c);
+      const uint4 xh0 = lds128(xr0 + st_off), xh1 = lds128(xr1 + st_off);
+      const uint4 xl0 = lds128(xr2 + st_off), xl1 = lds128(xr3 + st_off);
       int dh[NM][4], dl[NM][4];
 #pragma unroll
       for (int m = 0; m < NM; ++m)
@@ -301,27 +322,31 @@ int4_i8_kernel(const unsigned char* __restrict__ xs, int T, int H, int I, int k,
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         // B of MMA j: this lane's 8 input bytes of word j (even elements, then odd ones)
-        const uint32_t bh0 = word_of(xh[j >> 1], 2 * (j & 1)), bh1 = word_of(xh[j >> 1], 2 * (j & 1) + 1);
-        const uint32_t bl0 = word_of(xl[j >> 1], 2 * (j & 1)), bl1 = word_of(xl[j >> 1], 2 * (j & 1) + 1);
+        const uint4& xh = j < 2 ? xh0 : xh1;
+        const uint4& xl = j < 2 ? xl0 : xl1;
+        const uint32_t bh0 = word_of(xh, 2 * (j & 1)), bh1 = word_of(xh, 2 * (j & 1) + 1);
+        const uint32_t bl0 = word_of(xl, 2 * (j & 1)), bl1 = word_of(xl, 2 * (j & 1) + 1);
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
-          const uint32_t a = word_of(wa[m], j), c = word_of(wb[m], j);
+          const uint32_t a = word_of(wv[2 * m], j), c = word_of(wv[2 * m + 1], j);
           const uint32_t a0 = even16q(a), a1 = even16q(c), a2 = odd16q(a), a3 = odd16q(c);
           mma_s8s8(dh[m], a0, a1, a2, a3, bh0, bh1);
           mma_s8u8(dl[m], a0, a1, a2, a3, bl0, bl1);
         }
       }
       // dh/dl: rows g (0, 1) and g+8 (2, 3), columns 2t and 2t+1
-      const int blk = b0 + i;
+      const uint32_t srow_s = ssc_s + (uint32_t)(b0 + i) * (NM * 32);
 #pragma unroll
       for (int m = 0; m < NM; ++m) {
-        const float s0 = bf16_to_f32(ssc[(m * 16 + g) * nb + blk]);
-        const float s1 = bf16_to_f32(ssc[(m * 16 + g + 8) * nb + blk]);
+        const uint32_t sp = lds32(srow_s + 32 * m);
+        const float s0 = __uint_as_float(sp << 16), s1 = __uint_as_float(sp & 0xFFFF0000u);
         acc[m][0] = fmaf(s0, (float)(256 * dh[m][0] + dl[m][0]), acc[m][0]);
         acc[m][1] = fmaf(s0, (float)(256 * dh[m][1] + dl[m][1]), acc[m][1]);
         acc[m][2] = fmaf(s1, (float)(256 * dh[m][2] + dl[m][2]), acc[m][2]);
         acc[m][3] = fmaf(s1, (float)(256 * dh[m][3] + dl[m][3]), acc[m][3]);
       }
+      st_off = st_off + sbytes == ring_bytes ? 0 : st_off + sbytes;
+      wst_off = wst_off + sbytes == ring_bytes ? 0 : wst_off + sbytes;
     }
     cp_wait<0>();
 #pragma unroll
@@ -385,6 +410,31 @@ cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
 
 size_t int4_sliced_x_bytes(int T, int H) { return (size_t)T * sliced_row_bytes(H); }
 
+namespace {
+// Stages of the ring for a pass of ncols token columns: the most (up to 5) with which four
+// CTAs fit on an SM (56 KB each, of the SM's 228 KB less 1 KB reserved per CTA).
+template <int NM>
+int int4_stages(int nb, int ncols) {
+  constexpr size_t kBudget = 56 * 1024;
+  return Int4Smem<NM, 5>::bytes(nb, ncols) <= kBudget ? 5 : Int4Smem<NM, 4>::bytes(nb, ncols) <= kBudget ? 4 : 3;
+}
+
+template <int MODE, int NM, typename... Args>
+cudaError_t launch_i8(int S, int nb, int ncols, dim3 grid, cudaStream_t s, bool dependent, Args... args) {
+  switch (S) {
+    case 5:
+      return launch_ex(int4_i8_kernel<MODE, NM, 5>, grid, dim3(kQThreads), Int4Smem<NM, 5>::bytes(nb, ncols), s, dependent,
+                       args..., ncols);
+    case 4:
+      return launch_ex(int4_i8_kernel<MODE, NM, 4>, grid, dim3(kQThreads), Int4Smem<NM, 4>::bytes(nb, ncols), s, dependent,
+                       args..., ncols);
+    default:
+      return launch_ex(int4_i8_kernel<MODE, NM, 3>, grid, dim3(kQThreads), Int4Smem<NM, 3>::bytes(nb, ncols), s, dependent,
+                       args..., ncols);
+  }
+}
+}  // namespace
+
 cudaError_t launch_ffn_int4_mma(const void* x, int T, int H, int I, int k, const ExpertList& list, const int* offsets,
                                 const int* perm, float* h, float* y, cudaStream_t s, cudaEvent_t between,
                                 int max_pairs_per_expert, void* xsliced) {
@@ -393,24 +443,24 @@ cudaError_t launch_ffn_int4_mma(const void* x, int T, int H, int I, int k, const
   // the sliced tokens go to xsliced, or to the front of y (y is written only by the down pass,
   // after the gate/up pass has read them)
   unsigned char* xs = static_cast<unsigned char*>(xsliced ? xsliced : static_cast<void*>(y));
-  cudaError_t e = launch_ex(int4_prep_x_kernel, dim3(T), dim3(kPrepThreads), 0, s, false,
-                            static_cast<const uint16_t*>(x), H, xs);
-  if (e != cudaSuccess) return e;
-  e = launch_ex(int4_i8_kernel<0, 2>, dim3(I / 16, list.n), dim3(kQThreads), Int4Smem<2>::bytes(H / 128), s, false,
-                static_cast<const unsigned char*>(xs), T, H, I, k, list, offsets, perm, h, y);
-  if (e != cudaSuccess) return e;
-  if (between) cudaEventRecord(between, s);
   int has_shared = 0;
   for (int i = 0; i < list.n; ++i) has_shared |= list.expert[i] < 0;
   int rows_max = max_pairs_per_expert < 1 ? T * k : max_pairs_per_expert;
   if (has_shared && T > rows_max) rows_max = T;
+  const int ncols = rows_max < kNtok ? rows_max : kNtok;
+  cudaError_t e = launch_ex(int4_prep_x_kernel, dim3(T), dim3(kPrepThreads), 0, s, false,
+                            static_cast<const uint16_t*>(x), H, xs);
+  if (e != cudaSuccess) return e;
+  e = launch_i8<0, 2>(int4_stages<2>(H / 128, ncols), H / 128, ncols, dim3(I / 16, list.n), s, true,
+                      static_cast<const unsigned char*>(xs), T, H, I, k, list, offsets, perm, h, y);
+  if (e != cudaSuccess) return e;
+  if (between) cudaEventRecord(between, s);
   e = launch_ex(int4_prep_h_kernel, dim3(list.n, rows_max), dim3(kPrepThreads), (size_t)I * sizeof(float), s, true,
                 list, T, k, I, offsets, h);
   if (e != cudaSuccess) return e;
   const unsigned down_ctas = (unsigned)((H + 16 * kDownTiles - 1) / (16 * kDownTiles));
-  return launch_ex(int4_i8_kernel<1, kDownTiles>, dim3(down_ctas, list.n), dim3(kQThreads),
-                   Int4Smem<kDownTiles>::bytes(I / 128), s, true, static_cast<const unsigned char*>(xs), T, H, I, k,
-                   list, offsets, perm, h, y);
+  return launch_i8<1, kDownTiles>(int4_stages<kDownTiles>(I / 128, ncols), I / 128, ncols, dim3(down_ctas, list.n), s,
+                                  true, static_cast<const unsigned char*>(xs), T, H, I, k, list, offsets, perm, h, y);
 }
 
 }  // namespace ftk
