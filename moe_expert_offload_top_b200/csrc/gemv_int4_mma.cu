@@ -30,9 +30,14 @@
 // its own slots of a shared-memory ring with cp.async, S - 1 groups ahead.  A stage holds
 // the weight chunks and the input bytes of only the columns the launch uses (ncols <= 8,
 // the most pairs of one expert), so that at batch 1 nearly all of the ring is weights; S
-// is chosen per launch so that four CTAs fit on an SM.  The down pass copies its weights
-// before griddepcontrol.wait.  Scales of the CTA's rows are staged in shared memory once.
-// The 4 warps of a CTA split the reduction axis and add their partial sums in warp order.
+// is chosen per launch so that the CTAs of 16 warps fit on an SM (the register limit).  Both
+// passes copy their first weight groups before griddepcontrol.wait.  Scales of the CTA's
+// rows are staged in shared memory once.  The W warps of a CTA split the reduction axis and
+// add their partial sums in warp order: W = 4 for gate/up (16 rows of gate and of up per
+// CTA), W = 1 for down (32 rows per one-warp CTA, so that at batch 1 the 8 x 224 CTAs of a
+// top-8 forward at H = 7168 are resident at once).  Lanes past the pass's token columns read
+// column 0's input bytes, so the loop has no branch on the column; their MMA columns are
+// discarded.
 #include "decode_gemv.cuh"
 #include "sm100_sync.cuh"
 
@@ -42,8 +47,16 @@ namespace {
 
 using namespace gemv;
 
-constexpr int kQWarps = 4;
-constexpr int kQThreads = 32 * kQWarps;
+#ifndef FT_INT4_WARPS_PER_SM
+#define FT_INT4_WARPS_PER_SM 16
+#endif
+constexpr int kWarpsPerSm = FT_INT4_WARPS_PER_SM;   // resident warps per SM: caps the registers
+#ifndef FT_INT4_GU_WARPS
+#define FT_INT4_GU_WARPS 4
+#endif
+#ifndef FT_INT4_DOWN_WARPS
+#define FT_INT4_DOWN_WARPS 1
+#endif
 #ifndef FT_INT4_DOWN_TILES
 #define FT_INT4_DOWN_TILES 2
 #endif
@@ -179,12 +192,12 @@ __global__ void __launch_bounds__(kPrepThreads) int4_prep_h_kernel(const __grid_
 // input bytes of ncols columns, 256 bytes each: pieces 0-7 the 128 hi bytes of the group,
 // 8-15 the lo bytes, piece p of column c at slot p ^ c so that the 8 columns' lanes read
 // without bank conflicts.
-template <int NM, int S>
+template <int NM, int S, int W>
 struct Int4Smem {
   __host__ __device__ static constexpr size_t wbytes() { return (size_t)2 * NM * 32 * 16; }
   __host__ __device__ static constexpr size_t stage_bytes(int ncols) { return wbytes() + (size_t)ncols * 256; }
-  __host__ __device__ static constexpr size_t red_off(int ncols) { return (size_t)kQWarps * S * stage_bytes(ncols); }
-  __host__ __device__ static constexpr size_t red_bytes() { return (size_t)kQWarps * NM * 16 * 8 * sizeof(float); }
+  __host__ __device__ static constexpr size_t red_off(int ncols) { return (size_t)W * S * stage_bytes(ncols); }
+  __host__ __device__ static constexpr size_t red_bytes() { return (size_t)W * NM * 16 * 8 * sizeof(float); }
   __host__ __device__ static constexpr size_t scale_off(int ncols) { return red_off(ncols) + red_bytes(); }
   __host__ __device__ static constexpr size_t bytes(int nb, int ncols) {
     return scale_off(ncols) + (size_t)NM * 16 * nb * 2;
@@ -195,13 +208,13 @@ struct Int4Smem {
 // xs: the sliced token rows (MODE 0).  ncols (1..8): token columns per pass, at least the
 // most pairs of any listed expert for one pass per expert.  Grid (ceil(rows / rows per CTA),
 // list.n), 128 threads, Int4Smem<NM, S>::bytes(K / 128, ncols) bytes of shared memory.
-template <int MODE, int NM, int S>
-__global__ void __launch_bounds__(kQThreads, 4)
+template <int MODE, int NM, int S, int W>
+__global__ void __launch_bounds__(32 * W, kWarpsPerSm / W)
 int4_i8_kernel(const unsigned char* __restrict__ xs, int T, int H, int I, int k, const __grid_constant__ ExpertList list,
                const int* __restrict__ offsets, const int* __restrict__ perm, float* __restrict__ hbuf,
                float* __restrict__ ybuf, int ncols) {
   constexpr bool GU = MODE == 0;
-  using L = Int4Smem<NM, S>;
+  using L = Int4Smem<NM, S, W>;
   extern __shared__ __align__(16) unsigned char smem[];
   float (*red)[NM][16][8] = reinterpret_cast<float (*)[NM][16][8]>(smem + L::red_off(ncols));
   uint32_t* ssc = reinterpret_cast<uint32_t*>(smem + L::scale_off(ncols));   // [nb][NM][8]: rows g | g+8 << 16
@@ -217,7 +230,7 @@ int4_i8_kernel(const unsigned char* __restrict__ xs, int T, int H, int I, int k,
   const size_t row_bytes = (size_t)K / 2;
   const int nb = K / 128;
   const size_t srow = sliced_row_bytes(K);   // a sliced input row (x rows; h rows are 4 I bytes apart)
-  const int b0 = warp * nb / kQWarps, b1 = (warp + 1) * nb / kQWarps, nblk = b1 - b0;
+  const int b0 = warp * nb / W, b1 = (warp + 1) * nb / W, nblk = b1 - b0;
   int rbase[NM];
   const uint8_t* wsrc[2 * NM];   // this lane's 16 bytes of rows g ([2m]) and g+8 ([2m+1]) of tile m, group b0
 #pragma unroll
@@ -241,7 +254,7 @@ int4_i8_kernel(const unsigned char* __restrict__ xs, int T, int H, int I, int k,
     asm volatile("griddepcontrol.wait;" ::: "memory");
     return;
   }
-  for (int i = threadIdx.x; i < nb * NM * 8; i += kQThreads) {
+  for (int i = threadIdx.x; i < nb * NM * 8; i += 32 * W) {
     const int b = i / (NM * 8), m = (i / 8) % NM, r = i % 8;
     const uint16_t* sm_m = GU ? sc + (m & 1) * (mat / 128) : sc + 2 * (mat / 128);
     const int rb = GU ? row0 + 16 * (m >> 1) : row0 + 16 * m;
@@ -357,10 +370,13 @@ int4_i8_kernel(const unsigned char* __restrict__ xs, int T, int H, int I, int k,
       red[warp][m][g + 8][2 * t + 1] = acc[m][3];
     }
     __syncthreads();
-    {
-      const int r = threadIdx.x >> 3, col = threadIdx.x & 7;   // one (row, column) of a tile per thread
+    for (int rc = threadIdx.x; rc < 128; rc += 32 * W) {
+      const int r = rc >> 3, col = rc & 7;   // one (row, column) of a tile per thread
       auto wsum = [&](int m, int cc) {
-        return ((red[0][m][r][cc] + red[1][m][r][cc]) + red[2][m][r][cc]) + red[3][m][r][cc];
+        float v = red[0][m][r][cc];
+#pragma unroll
+        for (int w = 1; w < W; ++w) v += red[w][m][r][cc];
+        return v;
       };
       if (col < nt) {
         const int q = c0 + col;
@@ -411,26 +427,28 @@ cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
 size_t int4_sliced_x_bytes(int T, int H) { return (size_t)T * sliced_row_bytes(H); }
 
 namespace {
-// Stages of the ring for a pass of ncols token columns: the most (up to 5) with which four
-// CTAs fit on an SM (56 KB each, of the SM's 228 KB less 1 KB reserved per CTA).
-template <int NM>
+// Stages of the ring for a pass of ncols token columns: the most (up to 5) with which
+// kWarpsPerSm / W CTAs fit on an SM (of its 228 KB, less 1 KB reserved per CTA).
+template <int NM, int W>
 int int4_stages(int nb, int ncols) {
-  constexpr size_t kBudget = 56 * 1024;
-  return Int4Smem<NM, 5>::bytes(nb, ncols) <= kBudget ? 5 : Int4Smem<NM, 4>::bytes(nb, ncols) <= kBudget ? 4 : 3;
+  constexpr size_t kBudget = 228 * 1024 / (kWarpsPerSm / W) - 1024;
+  return Int4Smem<NM, 5, W>::bytes(nb, ncols) <= kBudget   ? 5
+         : Int4Smem<NM, 4, W>::bytes(nb, ncols) <= kBudget ? 4
+                                                           : 3;
 }
 
-template <int MODE, int NM, typename... Args>
-cudaError_t launch_i8(int S, int nb, int ncols, dim3 grid, cudaStream_t s, bool dependent, Args... args) {
-  switch (S) {
+template <int MODE, int NM, int W, typename... Args>
+cudaError_t launch_i8(int nb, int ncols, dim3 grid, cudaStream_t s, bool dependent, Args... args) {
+  switch (int4_stages<NM, W>(nb, ncols)) {
     case 5:
-      return launch_ex(int4_i8_kernel<MODE, NM, 5>, grid, dim3(kQThreads), Int4Smem<NM, 5>::bytes(nb, ncols), s, dependent,
-                       args..., ncols);
+      return launch_ex(int4_i8_kernel<MODE, NM, 5, W>, grid, dim3(32 * W), Int4Smem<NM, 5, W>::bytes(nb, ncols), s,
+                       dependent, args..., ncols);
     case 4:
-      return launch_ex(int4_i8_kernel<MODE, NM, 4>, grid, dim3(kQThreads), Int4Smem<NM, 4>::bytes(nb, ncols), s, dependent,
-                       args..., ncols);
+      return launch_ex(int4_i8_kernel<MODE, NM, 4, W>, grid, dim3(32 * W), Int4Smem<NM, 4, W>::bytes(nb, ncols), s,
+                       dependent, args..., ncols);
     default:
-      return launch_ex(int4_i8_kernel<MODE, NM, 3>, grid, dim3(kQThreads), Int4Smem<NM, 3>::bytes(nb, ncols), s, dependent,
-                       args..., ncols);
+      return launch_ex(int4_i8_kernel<MODE, NM, 3, W>, grid, dim3(32 * W), Int4Smem<NM, 3, W>::bytes(nb, ncols), s,
+                       dependent, args..., ncols);
   }
 }
 }  // namespace
@@ -451,16 +469,17 @@ cudaError_t launch_ffn_int4_mma(const void* x, int T, int H, int I, int k, const
   cudaError_t e = launch_ex(int4_prep_x_kernel, dim3(T), dim3(kPrepThreads), 0, s, false,
                             static_cast<const uint16_t*>(x), H, xs);
   if (e != cudaSuccess) return e;
-  e = launch_i8<0, 2>(int4_stages<2>(H / 128, ncols), H / 128, ncols, dim3(I / 16, list.n), s, true,
-                      static_cast<const unsigned char*>(xs), T, H, I, k, list, offsets, perm, h, y);
+  e = launch_i8<0, 2, FT_INT4_GU_WARPS>(H / 128, ncols, dim3(I / 16, list.n), s, true,
+                                       static_cast<const unsigned char*>(xs), T, H, I, k, list, offsets, perm, h, y);
   if (e != cudaSuccess) return e;
   if (between) cudaEventRecord(between, s);
   e = launch_ex(int4_prep_h_kernel, dim3(list.n, rows_max), dim3(kPrepThreads), (size_t)I * sizeof(float), s, true,
                 list, T, k, I, offsets, h);
   if (e != cudaSuccess) return e;
   const unsigned down_ctas = (unsigned)((H + 16 * kDownTiles - 1) / (16 * kDownTiles));
-  return launch_i8<1, kDownTiles>(int4_stages<kDownTiles>(I / 128, ncols), I / 128, ncols, dim3(down_ctas, list.n), s,
-                                  true, static_cast<const unsigned char*>(xs), T, H, I, k, list, offsets, perm, h, y);
+  return launch_i8<1, kDownTiles, FT_INT4_DOWN_WARPS>(I / 128, ncols, dim3(down_ctas, list.n), s, true,
+                                                     static_cast<const unsigned char*>(xs), T, H, I, k, list, offsets,
+                                                     perm, h, y);
 }
 
 }  // namespace ftk
