@@ -213,6 +213,32 @@ def aggregate(tokens, seconds, device=None):
     return t.item(), s.item()
 
 
+def host_memory_short(pool_bytes, replicas_on_node):
+    """None when this node's available memory holds the replicas' pinned pools (with 10%
+    to spare), else the reason.  Read before any rank allocates."""
+    try:
+        with open("/proc/meminfo") as f:
+            avail = next(int(l.split()[1]) * 1024 for l in f if l.startswith("MemAvailable:"))
+    except Exception:
+        return None
+    need = pool_bytes * replicas_on_node
+    if need <= 0.9 * avail:
+        return None
+    return ("host memory: %d replicas on this node need %.0f GB of pinned expert pool, %.0f GB available"
+            % (replicas_on_node, need / 1e9, avail / 1e9))
+
+
+def agree_any(flag, device=None):
+    """True on every rank if it is true on any rank (one collective, taken by all)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return flag
+    t = torch.tensor([1.0 if flag else 0.0], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item() > 0
+
+
 def barrier(device=None):
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
@@ -735,6 +761,16 @@ def run_ours(args):
     W, K = args.warmup, args.steps
     legs = set(ALL_LEGS if args.legs == "all" else [s for s in args.legs.split(",") if s])
     peaks, peak_src = measured_peaks()
+    short = host_memory_short(cfg.L * cfg.E * cfg.blob_bytes, int(os.environ.get("LOCAL_WORLD_SIZE", "1")))
+    if agree_any(short is not None, dev):
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": None, "unit": "tokens/s", "n_gpus": world,
+                              "config": headline_config(world),
+                              "error": short or "another rank's node is short of host memory"}), flush=True)
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+        return 1
     link_h2d, link_d2h = ft.ft_probe_host_link(256 << 20, 5)
     t0 = time.perf_counter()
     stack = GpuStack(cfg, device=dev)

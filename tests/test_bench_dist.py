@@ -28,7 +28,10 @@ def _rank_main(rank, world, port, q):
     r, w, lr = bench.dist_setup(world)
     bench.barrier()
     tokens, secs = bench.aggregate(100 * (r + 1), 0.5 + r, None)
-    q.put((r, w, lr, tokens, secs))
+    # the host-memory decision is taken by all ranks together: one short rank stops both
+    stop = bench.agree_any(r == 1, None)
+    go = bench.agree_any(False, None)
+    q.put((r, w, lr, tokens, secs, stop, go))
     dist.destroy_process_group()
 
 
@@ -43,9 +46,23 @@ def test_two_rank_aggregation_gloo():
         p.join(timeout=120)
     assert all(p.exitcode == 0 for p in procs)
     res = sorted(q.get(timeout=5) for _ in range(2))
-    for r, (rank, world, local, tokens, secs) in enumerate(res):
+    for r, (rank, world, local, tokens, secs, stop, go) in enumerate(res):
         assert (rank, world, local) == (r, 2, r)
         assert tokens == 300.0 and secs == 1.5      # sum of tokens, max of times
+        assert stop is True and go is False
+
+
+def test_host_memory_guard_for_replicas():
+    # N replicas on a node pin N copies of the expert pool; the bench stops before
+    # allocating when the node's available memory cannot hold them
+    sys.path.insert(0, ROOT)
+    import bench
+    with open("/proc/meminfo") as f:
+        avail = next(int(l.split()[1]) * 1024 for l in f if l.startswith("MemAvailable:"))
+    assert bench.host_memory_short(1 << 20, 2) is None
+    why = bench.host_memory_short(avail, 2)
+    assert why is not None and "2 replicas" in why
+    assert bench.agree_any(True) is True and bench.agree_any(False) is False
 
 
 def test_single_process_aggregation_is_identity():
