@@ -97,7 +97,11 @@ TRAFFIC = {
                              "to the average launch here"},
     "gemv_int4": {"sources": ["moe_expert_offload_top_b200/csrc/decode_gemv.cuh",
                               "moe_expert_offload_top_b200/csrc/gemv_int4_mma.cu"],
-                  "sha256": None, "ratio": None, "capture": None},
+                  "sha256": "bd18dc0e2198213de971cebd8a256259fce92eeeca2a76f1ffd465f819dbb2a5", "ratio": 1.0425,
+                  "capture": "ncu dram__bytes_read.sum + dram__bytes_write.sum of int4_prep_x_kernel + the gate/up "
+                             "int4_i8_kernel of two forwards of kernel_driver --workload int4-large-pool --layers 1 "
+                             "--experts 64 --steps 8 --perf (8 experts per launch, as here), 1.0425 of their "
+                             "algorithmic bytes; scaled to the average launch here"},
     "gemm": {"sources": ["moe_expert_offload_top_b200/csrc/grouped_gemm_sm100.cu"],
              "sha256": "0507ce91301990d38f67cede0ff1f116891de1794c23254f95a46243e0b318f6", "ratio": 1.03732,
              "capture": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the gate/up and down launches of "
