@@ -409,7 +409,11 @@ FT_API int ft_probe_host_memory(size_t bytes, int threads, int iters, double* gb
  * by z (descending, ties to the lower index).  gates[t][j] = softmax or sigmoid of
  * the selected logits, normalised over the k selected.
  *   x: [T][H] (x_is_bf16 ? bf16 : f32), router_w: [E][H] f32, logits: [T][E] f32
- *   (written), ids: [T][k] int32, gates: [T][k] f32. */
+ *   (written), ids: [T][k] int32, gates: [T][k] f32.
+ * Above 64 tokens the logits come from the forward's tiled router: each logit sums an fp32
+ * partial per 32 elements of H (increasing H) into its accumulator, in H order.  With
+ * H % 32 == 0 and 16-byte aligned x and router_w it streams the K steps through shared
+ * memory with cp.async; otherwise a one-step kernel computes the same sums, bit for bit. */
 FT_API int ft_router_topk(const void* x, int x_is_bf16, const float* router_w, int T, int H, int E,
                    int top_k, int gating, float* logits, int* ids, float* gates, void* stream);
 

@@ -1396,8 +1396,10 @@ int ft_router_topk(const void* x, int x_is_bf16, const float* router_w, int T, i
       top_k > FT_MAX_TOPK || (T > 0 && (!x || !router_w || !logits || !ids || !gates)))
     return FT_ERR_INVALID;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (ftk::launch_router_logits(x, x_is_bf16 != 0, router_w, T, H, E, logits, s) != cudaSuccess)
-    return FT_ERR_CUDA;
+  // the forward's choice: the tiled router above 64 tokens
+  const cudaError_t le = T > 64 ? ftk::launch_router_logits_tiled(x, x_is_bf16 != 0, router_w, T, H, E, logits, s)
+                                : ftk::launch_router_logits(x, x_is_bf16 != 0, router_w, T, H, E, logits, s);
+  if (le != cudaSuccess) return FT_ERR_CUDA;
   if (ftk::launch_topk_gates(logits, T, E, top_k, gating, ids, gates, s) != cudaSuccess)
     return FT_ERR_CUDA;
   return FT_OK;

@@ -141,10 +141,13 @@ __global__ void topk_gates_kernel(const float* __restrict__ z, int T, int E, int
   }
 }
 
-// Many tokens: CTA tile of 64 tokens x 64 experts, K step 16 through shared
-// memory, 256 threads each owning a 4 x 4 block of logits (fp32 FMAs in a fixed
-// order along H).
-constexpr int RT = 64, RE = 64, RK = 16;
+// Many tokens: CTA tile of 64 tokens x 64 experts, K step 32 through shared
+// memory, 256 threads each owning a 4 x 4 block of logits.  Each logit sums in two
+// levels, in a fixed order: a fresh fp32 partial of the 32 products of a K step (fmaf
+// in increasing H), added to the logit's accumulator step by step.  The error then grows
+// with 32 + H/32 terms rather than H (at H = 7168 a single running sum missed the 2e-6
+// relative bound against the float64 sum).
+constexpr int RT = 64, RE = 64, RK = 32;
 template <typename XT>
 __global__ void __launch_bounds__(256)
 router_logits_tiled_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T, int H, int E,
@@ -168,6 +171,7 @@ router_logits_tiled_kernel(const XT* __restrict__ x, const float* __restrict__ w
       ws[c][r] = wv;
     }
     __syncthreads();
+    float part[4][4] = {};
 #pragma unroll
     for (int c = 0; c < RK; ++c) {
       float a[4], b[4];
@@ -176,8 +180,12 @@ router_logits_tiled_kernel(const XT* __restrict__ x, const float* __restrict__ w
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(a[i], b[j], part[i][j]);
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
     __syncthreads();
   }
 #pragma unroll
@@ -185,6 +193,118 @@ router_logits_tiled_kernel(const XT* __restrict__ x, const float* __restrict__ w
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int t = t0 + ty * 4 + i, e = e0 + tx * 4 + j;
+      if (t < T && e < E) z[(size_t)t * E + e] = acc[i][j];
+    }
+}
+
+// Many tokens, pipelined: the same 64 x 64 CTA tile, K steps of 32 elements through a
+// 3-stage cp.async ring (x rows as stored, bf16 or fp32; router rows fp32).  Thread (tx, ty)
+// = (tid % 16, tid / 16) owns logits (t0 + ty + 16 i, e0 + tx + 16 j), i, j < 4, so the 16
+// lanes of a half-warp read 16 consecutive router rows; rows are padded by 16 bytes so that
+// those 16-byte reads fall on distinct banks.  The two-level sum of router_logits_tiled_kernel
+// (a partial per K step of 32, then the accumulator), bit for bit.  Needs H % 32 == 0 and
+// 16-byte aligned x and w.
+constexpr int PT = 64, PE = 64, PK = 32, PS = 3;
+template <typename XT>
+struct RouterPipe {
+  static constexpr int kXRow = PK * (int)sizeof(XT) + 16;   // bytes of one x row in a stage
+  static constexpr int kWRow = PK * 4 + 16;
+  static constexpr int kFRow = PK * 4 + 16;                  // bf16 x: the step's rows widened to fp32
+  static constexpr int kStage = PT * kXRow + PE * kWRow;
+  static constexpr int kBytes = PS * kStage + (sizeof(XT) == 2 ? PT * kFRow : 0);
+};
+
+template <typename XT>
+__global__ void __launch_bounds__(256)
+router_logits_pipe_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T, int H, int E,
+                          float* __restrict__ z) {
+  using P = RouterPipe<XT>;
+  extern __shared__ __align__(16) unsigned char rsm[];
+  const int t0 = blockIdx.x * PT, e0 = blockIdx.y * PE;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int nk = H / PK;
+  const uint32_t base = (uint32_t)__cvta_generic_to_shared(rsm);
+  // the 16-byte pieces this thread copies per stage: x rows (PK * sizeof(XT) / 16 pieces
+  // each) and router rows (8 pieces each)
+  constexpr int XP = PK * (int)sizeof(XT) / 16, WP = PK * 4 / 16;
+  auto issue = [&](int ks, int st) {
+    const uint32_t sx = base + st * P::kStage, sw = sx + PT * P::kXRow;
+    for (int i = threadIdx.x; i < PT * XP; i += 256) {
+      const int r = i / XP, c = i % XP;
+      const XT* src = x + (size_t)min(t0 + r, T - 1) * H + (size_t)ks * PK + c * (16 / (int)sizeof(XT));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sx + r * P::kXRow + c * 16), "l"(src) : "memory");
+    }
+    for (int i = threadIdx.x; i < PE * WP; i += 256) {
+      const int r = i / WP, c = i % WP;
+      const float* src = w + (size_t)min(e0 + r, E - 1) * H + (size_t)ks * PK + c * 4;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sw + r * P::kWRow + c * 16), "l"(src) : "memory");
+    }
+  };
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int s = 0; s < PS - 1; ++s) {
+    if (s < nk) issue(s, s);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  for (int ks = 0; ks < nk; ++ks) {
+    asm volatile("cp.async.wait_group %0;" ::"n"(PS - 2) : "memory");
+    __syncthreads();   // stage ks is in for every thread; stage ks - 1 is no longer read
+    if (ks + PS - 1 < nk) issue(ks + PS - 1, (ks + PS - 1) % PS);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    const unsigned char* sx = rsm + (ks % PS) * P::kStage;
+    const unsigned char* sw = sx + PT * P::kXRow;
+    if constexpr (sizeof(XT) == 2) {
+      // widen the step's x rows once (8 per thread) instead of in each of the 16 threads
+      // that read an element; the barrier at the top of the next step keeps them until all
+      // threads are done with them
+      unsigned char* sf = rsm + PS * P::kStage;
+      const int r = threadIdx.x >> 2, c = (threadIdx.x & 3) * 8;
+      const uint4 v = *reinterpret_cast<const uint4*>(sx + r * P::kXRow + c * 2);
+      float4* d = reinterpret_cast<float4*>(sf + r * P::kFRow + c * 4);
+      d[0] = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
+      d[1] = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
+      __syncthreads();
+      sx = sf;
+    }
+    float part[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) part[i][j] = 0.f;
+#pragma unroll
+    for (int kq = 0; kq < PK; kq += 4) {
+      float a[4][4], b[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = *reinterpret_cast<const float4*>(sx + (ty + 16 * i) * (sizeof(XT) == 2 ? P::kFRow : P::kXRow) + kq * 4);
+        a[i][0] = v.x; a[i][1] = v.y; a[i][2] = v.z; a[i][3] = v.w;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 v = *reinterpret_cast<const float4*>(sw + (tx + 16 * j) * P::kWRow + kq * 4);
+        b[j][0] = v.x; b[j][1] = v.y; b[j][2] = v.z; b[j][3] = v.w;
+      }
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) part[i][j] = fmaf(a[i][kk], b[j][kk], part[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = t0 + ty + 16 * i, e = e0 + tx + 16 * j;
       if (t < T && e < E) z[(size_t)t * E + e] = acc[i][j];
     }
 }
@@ -402,6 +522,22 @@ route_decode_kernel(const XT* __restrict__ x, const float* __restrict__ w, int T
 cudaError_t launch_router_logits_tiled(const void* x, bool x_bf16, const float* w_router, int T, int H,
                                        int E, float* logits, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
+  const bool aligned = ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w_router)) & 15) == 0;
+  if (H % PK == 0 && aligned) {
+    dim3 pgrid((T + PT - 1) / PT, (E + PE - 1) / PE);
+    if (x_bf16) {
+      auto kern = router_logits_pipe_kernel<uint16_t>;
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RouterPipe<uint16_t>::kBytes);
+      if (e != cudaSuccess) return e;
+      kern<<<pgrid, 256, RouterPipe<uint16_t>::kBytes, s>>>(static_cast<const uint16_t*>(x), w_router, T, H, E, logits);
+    } else {
+      auto kern = router_logits_pipe_kernel<float>;
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RouterPipe<float>::kBytes);
+      if (e != cudaSuccess) return e;
+      kern<<<pgrid, 256, RouterPipe<float>::kBytes, s>>>(static_cast<const float*>(x), w_router, T, H, E, logits);
+    }
+    return cudaGetLastError();
+  }
   dim3 grid((T + RT - 1) / RT, (E + RE - 1) / RE);
   if (x_bf16)
     router_logits_tiled_kernel<uint16_t><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(x), w_router, T, H,

@@ -54,6 +54,36 @@ def test_router_topk_parity(T, H, E, k, gating, xbf16):
     assert np.max(np.abs(g.cpu().numpy()[ok] - gr[ok])) <= 2e-6
 
 
+@pytest.mark.parametrize("T,H,E,xbf16", [(4096, 4096, 256, True), (150, 7168, 200, True), (97, 512, 64, False)])
+def test_tiled_router_pipelined_equals_one_step(T, H, E, xbf16):
+    # Above 64 tokens the logits come from the tiled router.  Its cp.async pipeline runs on
+    # 16-byte aligned x; an x one element off that alignment takes the one-step kernel.
+    # Both sum an fp32 partial per 32 elements of H into each logit in H order: bit for bit equal.
+    x = synth.normal_f32(11, 8, 0, 0, T * H).reshape(T, H)
+    w = synth.normal_f32(11, 4, 0, 0, E * H, 0.02).reshape(E, H)
+    if xbf16:
+        xd, xv = _bf16_dev(x)
+    else:
+        xd, xv = torch.from_numpy(np.ascontiguousarray(x)).to(DEV), x
+    pad = torch.empty(T * H + 8, dtype=xd.dtype, device=DEV)
+    xm = pad[1:1 + T * H].view(T, H)   # 2 or 4 bytes past a 16-byte boundary
+    xm.copy_(xd)
+    assert xd.data_ptr() % 16 == 0 and xm.data_ptr() % 16 != 0
+    wd = torch.from_numpy(w).to(DEV)
+    za = torch.full((T, E), float("nan"), device=DEV)
+    zb = torch.full((T, E), float("nan"), device=DEV)
+    ids = torch.empty((T, 4), dtype=torch.int32, device=DEV)
+    g = torch.empty((T, 4), device=DEV)
+    ft.ft_router_topk(xd, xbf16, wd, T, H, E, 4, "sigmoid", za, ids, g)
+    ft.ft_router_topk(xm, xbf16, wd, T, H, E, 4, "sigmoid", zb, ids, g)
+    torch.cuda.synchronize()
+    a, b = za.cpu().numpy(), zb.cpu().numpy()
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    rows = np.random.default_rng(T).choice(T, min(T, 64), replace=False)   # the oracle on a sample
+    zr = moe.router_logits(xv[rows], w)
+    assert np.max(np.abs(a[rows] - zr)) <= 2e-6 * max(1.0, np.abs(zr).max())
+
+
 @pytest.mark.parametrize("T,H,E,k,gating,xbf16", [
     (1, 256, 16, 2, "softmax", False), (1, 2048, 128, 8, "softmax", True), (1, 4096, 256, 6, "sigmoid", True),
     (8, 7168, 256, 8, "sigmoid", True), (32, 7168, 256, 8, "sigmoid", True), (64, 512, 256, 16, "softmax", True),
@@ -147,6 +177,9 @@ def test_permute_parity(T, k, E):
     ("bf16", 2048, 768, 1, 128, 8, False), ("bf16", 2048, 768, 3, 16, 8, True),
     ("bf16", 1024, 512, 37, 6, 3, True), ("int4", 1024, 512, 1, 16, 4, False),
     ("int4", 7168, 2048, 2, 8, 8, False), ("int4", 1024, 256, 19, 5, 2, True),
+    # int4: 9 groups of 128 on the gate/up reduction axis split 2/2/2/3 over the 4 warps; 5
+    # token columns per pass (4 ring stages)
+    ("int4", 1152, 384, 5, 6, 3, True),
     ("nvfp4", 2048, 768, 1, 16, 8, False), ("nvfp4", 1024, 512, 3, 8, 4, True), ("nvfp4", 256, 96, 12, 4, 2, True),
 ])
 def test_expert_ffn_and_combine_parity(wd, H, I, T, E, k, shared):
