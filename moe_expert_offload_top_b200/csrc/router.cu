@@ -209,9 +209,8 @@ template <typename XT>
 struct RouterPipe {
   static constexpr int kXRow = PK * (int)sizeof(XT) + 16;   // bytes of one x row in a stage
   static constexpr int kWRow = PK * 4 + 16;
-  static constexpr int kFRow = PK * 4 + 16;                  // bf16 x: the step's rows widened to fp32
   static constexpr int kStage = PT * kXRow + PE * kWRow;
-  static constexpr int kBytes = PS * kStage + (sizeof(XT) == 2 ? PT * kFRow : 0);
+  static constexpr int kBytes = PS * kStage;
 };
 
 template <typename XT>
@@ -256,19 +255,6 @@ router_logits_pipe_kernel(const XT* __restrict__ x, const float* __restrict__ w,
     asm volatile("cp.async.commit_group;" ::: "memory");
     const unsigned char* sx = rsm + (ks % PS) * P::kStage;
     const unsigned char* sw = sx + PT * P::kXRow;
-    if constexpr (sizeof(XT) == 2) {
-      // widen the step's x rows once (8 per thread) instead of in each of the 16 threads
-      // that read an element; the barrier at the top of the next step keeps them until all
-      // threads are done with them
-      unsigned char* sf = rsm + PS * P::kStage;
-      const int r = threadIdx.x >> 2, c = (threadIdx.x & 3) * 8;
-      const uint4 v = *reinterpret_cast<const uint4*>(sx + r * P::kXRow + c * 2);
-      float4* d = reinterpret_cast<float4*>(sf + r * P::kFRow + c * 4);
-      d[0] = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
-      d[1] = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
-      __syncthreads();
-      sx = sf;
-    }
     float part[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -279,8 +265,14 @@ router_logits_pipe_kernel(const XT* __restrict__ x, const float* __restrict__ w,
       float a[4][4], b[4][4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float4 v = *reinterpret_cast<const float4*>(sx + (ty + 16 * i) * (sizeof(XT) == 2 ? P::kFRow : P::kXRow) + kq * 4);
-        a[i][0] = v.x; a[i][1] = v.y; a[i][2] = v.z; a[i][3] = v.w;
+        const unsigned char* row = sx + (ty + 16 * i) * P::kXRow;
+        if constexpr (sizeof(XT) == 2) {
+          const uint2 v = *reinterpret_cast<const uint2*>(row + kq * 2);
+          a[i][0] = bf16lo(v.x); a[i][1] = bf16hi(v.x); a[i][2] = bf16lo(v.y); a[i][3] = bf16hi(v.y);
+        } else {
+          const float4 v = *reinterpret_cast<const float4*>(row + kq * 4);
+          a[i][0] = v.x; a[i][1] = v.y; a[i][2] = v.z; a[i][3] = v.w;
+        }
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
