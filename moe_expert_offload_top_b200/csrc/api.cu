@@ -102,7 +102,7 @@ struct ft_moe {
   int* d_perm = nullptr;
   int* d_inv = nullptr;
   float* d_h = nullptr;
-  void* d_xs = nullptr;           // int4 stacks: the forward's tokens as sliced rows (tensor-core GEMV)
+  void* d_xs = nullptr;           // int4 / NVFP4 stacks: the forward's tokens as sliced rows (tensor-core GEMV)
   float* d_y = nullptr;
   int* h_ids = nullptr;            // routing ids on the host: h_box + 2
   int* h_box = nullptr;            // mapped pinned {seq, device error word, ids[T*k]}
@@ -126,7 +126,7 @@ struct ft_moe {
   cudaEvent_t xs_ev = nullptr;    // orders a forward after the previous stream's work
   int last_T = 0;
   int fused_ffn = 0;              // decode FFN + combine as one launch (ffn_decode_fused_kernel)
-  int int4_tensor = 1;            // int4 decode GEMV on the tensor cores (mma.sync)
+  int int4_tensor = 1;            // int4 / NVFP4 decode GEMV on the tensor cores (mma.sync)
   int* d_ctl = nullptr;           // work counters of the fused decode FFN
   int* h_hold = nullptr;          // mapped pinned flag that releases hold_kernel (stage timing)
   int* d_hold = nullptr;
@@ -257,7 +257,8 @@ int ensure_scratch(ft_moe* h, int T) {
             cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->d_box), h->h_box, 0) == cudaSuccess &&
             ((h->wdtype != FT_W_BF16 && h->wdtype != FT_W_NVFP4) ||
              cudaMalloc(&h->d_ax, sizeof(uint16_t) * rows * h->H) == cudaSuccess) &&
-            (h->wdtype != FT_W_INT4_G128 || cudaMalloc(&h->d_xs, ftk::int4_sliced_x_bytes(T, h->H)) == cudaSuccess);
+            ((h->wdtype != FT_W_INT4_G128 && h->wdtype != FT_W_NVFP4) ||
+             cudaMalloc(&h->d_xs, ftk::int4_sliced_x_bytes(T, h->H)) == cudaSuccess);
   if (!ok) {
     cudaGetLastError();
     free_scratch(h);

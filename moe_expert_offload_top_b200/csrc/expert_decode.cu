@@ -121,6 +121,8 @@ cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdt
   if (list.n <= 0 || T <= 0) return cudaSuccess;
   if (wdtype == WT_INT4 && int4_tensor)
     return launch_ffn_int4_mma(x, T, H, I, k, list, offsets, perm, h, y, s, between, max_pairs_per_expert, int4_xs);
+  if (wdtype == WT_NVFP4 && int4_tensor && H % 128 == 0 && I % 128 == 0)   // whole groups of 128
+    return launch_ffn_nvfp4_mma(x, T, H, I, k, list, offsets, perm, h, y, s, between, max_pairs_per_expert, int4_xs);
   int nt = max_pairs_per_expert < T ? max_pairs_per_expert : T;
   if (nt < 1) nt = 1;
   auto bytes_of = [&](int K) -> size_t {

@@ -39,13 +39,14 @@
 // column 0's input bytes, so the loop has no branch on the column; their MMA columns are
 // discarded.
 #include "decode_gemv.cuh"
-#include "sm100_sync.cuh"
+#include "gemv_ring.cuh"
 
 namespace ftk {
 
 namespace {
 
 using namespace gemv;
+using namespace ring;
 
 #ifndef FT_INT4_WARPS_PER_SM
 #define FT_INT4_WARPS_PER_SM 16
@@ -62,7 +63,6 @@ constexpr int kWarpsPerSm = FT_INT4_WARPS_PER_SM;   // resident warps per SM: ca
 #endif
 constexpr int kDownTiles = FT_INT4_DOWN_TILES;
 constexpr int kNtok = 8;                 // tokens (MMA columns) per pass
-constexpr int kPrepThreads = 256;
 
 // d (16x8 s32) += A (16x32 s8) * B (32x8, s8 or u8).
 FT_DEVICE void mma_s8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -76,44 +76,14 @@ FT_DEVICE void mma_s8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-FT_DEVICE uint32_t word_of(const uint4& v, int j) { return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w; }
 // 16 q of the even / odd nibbles of w as four signed bytes.
 FT_DEVICE uint32_t even16q(uint32_t w) { return (w << 4) & 0xF0F0F0F0u; }
 FT_DEVICE uint32_t odd16q(uint32_t w) { return w & 0xF0F0F0F0u; }
-
-FT_DEVICE void cp16s(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-FT_DEVICE uint4 lds128(uint32_t a) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
-  return v;
-}
-FT_DEVICE uint32_t lds32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
-FT_DEVICE void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-FT_DEVICE void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // ---------------------------------------------------------------- the inputs --
 // A sliced row of K inputs: [hi bytes: K][lo bytes: K][f: float = 2^(E - 14) / 16][12 bytes],
 // bytes in the even-then-odd order of every block of 8 elements.
 __host__ __device__ constexpr size_t sliced_row_bytes(int K) { return 2 * (size_t)K + 16; }
-
-// Block maximum of |v| over 256 threads (all call it).
-FT_DEVICE float block_max(float v, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float m = 0.f;
-  for (int i = 0; i < kPrepThreads / 32; ++i) m = fmaxf(m, red[i]);
-  __syncthreads();
-  return m;
-}
 
 // Writes the 8 values v (elements 8b .. 8b+7 of a row) as bytes of X = round(v * scale):
 // hi bytes (signed) and lo bytes (unsigned), even elements first.
@@ -142,7 +112,7 @@ __global__ void __launch_bounds__(kPrepThreads) int4_prep_x_kernel(const uint16_
   for (int i = threadIdx.x; i < H; i += kPrepThreads) m = fmaxf(m, fabsf(bf16_to_f32(row[i])));
   m = block_max(m, red);
   // E = exponent of the largest |v|; the scale 2^(14 - E) is exact, so is v * scale
-  const int E = m > 0.f ? ((int)((__float_as_uint(m) >> 23) & 0xFF) - 127) : 0;
+  const int E = exponent_of(m);
   const float scale = ldexpf(1.f, 14 - E);
   for (int b = threadIdx.x; b < H / 8; b += kPrepThreads) {
     const uint4 q = *reinterpret_cast<const uint4*>(row + 8 * b);
@@ -174,7 +144,7 @@ __global__ void __launch_bounds__(kPrepThreads) int4_prep_h_kernel(const __grid_
     m = fmaxf(m, fabsf(v));
   }
   m = block_max(m, red);   // its barriers also order every read of the row before the writes
-  const int E = m > 0.f ? ((int)((__float_as_uint(m) >> 23) & 0xFF) - 127) : 0;
+  const int E = exponent_of(m);
   const float scale = ldexpf(1.f, 14 - E);
   unsigned char* out = reinterpret_cast<unsigned char*>(row);
   for (int b = threadIdx.x; b < I / 8; b += kPrepThreads) {
@@ -400,26 +370,6 @@ int4_i8_kernel(const unsigned char* __restrict__ xs, int T, int H, int I, int k,
     }
     __syncthreads();
   }
-}
-
-template <typename... KArgs, typename... Args>
-cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool dependent,
-                      Args... args) {
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = dependent ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
 }  // namespace

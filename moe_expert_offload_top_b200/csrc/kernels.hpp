@@ -44,10 +44,11 @@ cudaError_t launch_permute(const int* ids, int T, int k, int E, int* counts, int
 // then the down projection into y [pairs][H] fp32.  Pairs are positions in the
 // permutation (routed) or T*k + t (shared expert).  `between` (optional) is recorded
 // on s between the gate/up and the down passes.
-// int4 weights run on the int8 tensor cores (launch_ffn_int4_mma) unless int4_tensor is
-// false; the h rows of the list's pairs are then left as sliced inputs (see below), and
-// int4_xs (int4_sliced_x_bytes(T, H) bytes) receives the sliced tokens, or, when null, the
-// front of y does (before the down pass writes y).
+// Packed weights run on the tensor cores unless int4_tensor is false: int4 on the int8
+// ones (launch_ffn_int4_mma), NVFP4 on the f16 ones (launch_ffn_nvfp4_mma).  The h rows of
+// the list's pairs are then left as sliced inputs (see below), and int4_xs
+// (int4_sliced_x_bytes(T, H) bytes) receives the sliced tokens, or, when null, the front of
+// y does (before the down pass writes y).
 cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdtype,
                               const ExpertList& list, int max_pairs_per_expert, const int* offsets,
                               const int* perm, float* h, float* y, cudaStream_t s,
@@ -61,8 +62,15 @@ cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdt
 cudaError_t launch_ffn_int4_mma(const void* x, int T, int H, int I, int k, const ExpertList& list, const int* offsets,
                                 const int* perm, float* h, float* y, cudaStream_t s, cudaEvent_t between,
                                 int max_pairs_per_expert, void* xsliced);
-// Bytes of the sliced tokens of launch_ffn_int4_mma.
+// Bytes of the sliced tokens of launch_ffn_int4_mma and launch_ffn_nvfp4_mma.
 size_t int4_sliced_x_bytes(int T, int H);
+// K3 (decode) for NVFP4 weights on the f16 tensor cores (gemv_nvfp4_mma.cu); x bf16.  The
+// tokens and, after the gate/up pass, the h rows of the list's pairs are written as f16 rows
+// with a per-row power-of-two scale (then a float: the scale's inverse), the tokens into
+// xsliced (or the front of y when null), the h rows in place.
+cudaError_t launch_ffn_nvfp4_mma(const void* x, int T, int H, int I, int k, const ExpertList& list, const int* offsets,
+                                 const int* perm, float* h, float* y, cudaStream_t s, cudaEvent_t between,
+                                 int max_pairs_per_expert, void* xsliced);
 // K3 + K5 (decode) in one launch (ffn_fused.cuh): gate/up + SwiGLU into h, down into y
 // and, with `combine`, out[t] = sum_j gates[t][j] * y[inv[t*k+j]] (+ shared) for the
 // entries of `list`.  The combine of a launch covers every pair of the forward, so

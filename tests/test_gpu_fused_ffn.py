@@ -132,11 +132,12 @@ def test_per_pass_kernels_split_around_the_fill_wait():
         assert np.array_equal(oa, ob)
 
 
-@pytest.mark.parametrize("batch", [1, 8])
-def test_int4_tensor_core_gemv_against_cuda_cores_and_oracle(batch):
-    # the int4 decode GEMV on mma.sync and on the fp32 pipes: the same routing and cache
-    # trace, outputs that differ only by summation order, both within the oracle's bound
-    cfg = synth.MoeConfig("int4-tc", L=2, E=32, H=1024, I=512, k=8, gating="sigmoid", wdtype="int4",
+@pytest.mark.parametrize("wdtype,batch", [("int4", 1), ("int4", 8), ("nvfp4", 1), ("nvfp4", 8)])
+def test_int4_tensor_core_gemv_against_cuda_cores_and_oracle(wdtype, batch):
+    # the packed-weight decode GEMV on mma.sync (int4: int8 products; NVFP4: f16 products)
+    # and on the fp32 pipes: the same routing and cache trace, outputs that differ only by
+    # summation order (and, for NVFP4, h rounded to f16), both within the oracle's bound
+    cfg = synth.MoeConfig("%s-tc" % wdtype, L=2, E=32, H=1024, I=512, k=8, gating="sigmoid", wdtype=wdtype,
                           shared=True, C=64, tokens=16 * batch, batches=(batch,), process="ar1", mode="decode")
     a = _run(cfg, fused=False, batch=batch, oracle=True, int4_tensor=True)
     b = _run(cfg, fused=False, batch=batch, int4_tensor=False)
@@ -151,4 +152,4 @@ def test_int4_tensor_core_gemv_against_cuda_cores_and_oracle(batch):
     last = steps if div is None else div // (cfg.L * batch)
     for s in range(last):
         for l in range(cfg.L):
-            assert_close(a["outs"][s][l], ref["out"][(s, l)], "int4", "step %d layer %d" % (s, l), stored_bf16=True)
+            assert_close(a["outs"][s][l], ref["out"][(s, l)], wdtype, "step %d layer %d" % (s, l), stored_bf16=True)

@@ -187,3 +187,89 @@ def test_int4_slice_permutation_matches_the_fragment_order():
     for e in range(8):
         order[pos(e)] = e
     assert order == [0, 2, 4, 6, 1, 3, 5, 7]
+
+
+# ------------------------------------------------ NVFP4 decode on the f16 tensor cores --
+
+def _mma_m16n8k16(a_regs, b_regs):
+    """One mma.sync.m16n8k16 from per-lane fragments, as the PTX fragment layout defines
+    them: a_regs[lane] = 4 pairs (a0..a3), b_regs[lane] = 2 pairs (b0, b1); returns D (16 x 8)."""
+    A = np.zeros((16, 16))
+    B = np.zeros((16, 8))
+    for lane in range(32):
+        g, t = lane >> 2, lane & 3
+        a0, a1, a2, a3 = a_regs[lane]
+        A[g, 2 * t:2 * t + 2] = a0
+        A[g + 8, 2 * t:2 * t + 2] = a1
+        A[g, 2 * t + 8:2 * t + 10] = a2
+        A[g + 8, 2 * t + 8:2 * t + 10] = a3
+        b0, b1 = b_regs[lane]
+        B[2 * t:2 * t + 2, g] = b0
+        B[2 * t + 8:2 * t + 10, g] = b1
+    return A @ B
+
+
+def test_nvfp4_mma_fragments_give_the_group_dot_products():
+    # One 128-element group of 16 weight rows and 8 token columns through the kernel's
+    # assignment: lane (g, t) holds code bytes 16t .. 16t+15 of rows g and g+8 (elements
+    # 32t .. 32t+31); MMA j takes bytes 2j (a0 / a1) and 2j+1 (a2 / a3) times block scale
+    # 2t + j // 4, and input elements 32t + 4j .. +3 of column g (b0, b1).  The 8 MMAs must
+    # sum to the plain dot products.
+    rng = np.random.default_rng(7)
+    e2 = np.array([_e2m1(c) for c in range(16)])
+    codes = rng.integers(0, 16, (16, 128))
+    scodes = rng.integers(0, 0x7F, (16, 8))                    # e4m3, no NaN
+    sv = np.array([[_e4m3(c) for c in row] for row in scodes])
+    w = e2[codes] * np.repeat(sv, 16, axis=1)                 # value of each weight
+    x = rng.standard_normal((128, 8)).astype(np.float16).astype(np.float64)
+    D = np.zeros((16, 8))
+    for j in range(8):
+        a_regs, b_regs = [], []
+        for lane in range(32):
+            g, t = lane >> 2, lane & 3
+            def pair(r, byte):
+                e0 = 32 * t + 2 * byte                         # low nibble: the even element
+                s = sv[r, 2 * t + j // 4]
+                return np.array([e2[codes[r, e0]] * s, e2[codes[r, e0 + 1]] * s])
+            a_regs.append((pair(g, 2 * j), pair(g + 8, 2 * j), pair(g, 2 * j + 1), pair(g + 8, 2 * j + 1)))
+            k0 = 32 * t + 4 * j
+            b_regs.append((x[k0:k0 + 2, g], x[k0 + 2:k0 + 4, g]))
+        D += _mma_m16n8k16(a_regs, b_regs)
+    assert np.allclose(D, w @ x, rtol=1e-12, atol=1e-12)
+
+
+def test_nvfp4_input_slots_distinct_and_bank_conflict_free():
+    # piece u (16 bytes) of lane (g, t) sits at slot (4u + t) ^ (4 (g & 1)) of column g's 256
+    # bytes: one slot per piece, and the 8 lanes of a quarter-warp reading piece u hit 8
+    # different 16-byte bank groups (a column's 256 bytes wrap the 128 bytes of banks twice)
+    for g in range(8):
+        slots = sorted((4 * u + t) ^ (4 * (g & 1)) for u in range(4) for t in range(4))
+        assert slots == list(range(16))
+    for u in range(4):
+        for g0 in range(0, 8, 2):
+            groups = {((g * 256 + 16 * ((4 * u + t) ^ (4 * (g & 1)))) % 128) // 16 for g in (g0, g0 + 1) for t in range(4)}
+            assert len(groups) == 8
+
+
+def test_nvfp4_inputs_as_f16_rows_with_a_power_of_two_scale():
+    # x' = x * 2^(14 - E), E the exponent of the row's largest |x|: |x'| < 2^15 (f16 holds it);
+    # a bf16 x is exact in f16 wherever |x| >= 2^(E - 28) (f16 normals); an fp32 h rounds to
+    # 11 significant bits there (relative error at most 2^-11, half an ulp)
+    rng = np.random.default_rng(8)
+    for trial in range(20):
+        scale = 10.0 ** rng.uniform(-8, 8)
+        v = _bf16_bits_to_f32(synth.round_bf16((rng.standard_normal(4096) * scale).astype(np.float32)))
+        v = v.astype(np.float64)
+        m = np.max(np.abs(v))
+        E = int(np.frexp(np.float32(m))[1]) - 1
+        xs = v * 2.0 ** (14 - E)
+        assert np.max(np.abs(xs)) < 2.0 ** 15
+        f16 = xs.astype(np.float16).astype(np.float64)
+        normal = np.abs(v) >= 2.0 ** (E - 28)
+        assert np.array_equal(f16[normal], xs[normal])
+        h = rng.standard_normal(2048) * scale
+        E = int(np.frexp(np.float32(np.max(np.abs(h))))[1]) - 1
+        hs = (h * 2.0 ** (14 - E)).astype(np.float32).astype(np.float64)
+        hf = hs.astype(np.float16).astype(np.float64)
+        big = np.abs(hs) >= 2.0 ** -14
+        assert np.all(np.abs(hf[big] - hs[big]) <= 2.0 ** -11 * np.abs(hs[big]))

@@ -2,7 +2,7 @@
 may not allocate device memory (their intermediate rows live in the library's
 static device array).  Checked through the C ABI against the allocating entry
 points (ft_expert_ffn_decode with caller scratch, then ft_combine) on two calls
-in a row, for bf16 and int4 weights: both run the same kernels on the same
+in a row, for bf16, int4 and NVFP4 weights: both run the same kernels on the same
 inputs, so the outputs must agree bit for bit.  Also checked: its size limit
 and its check of the shared-expert entry."""
 import numpy as np
@@ -57,7 +57,7 @@ def _no_alloc(a):
     return out
 
 
-@pytest.mark.parametrize("wdtype", ["bf16", "int4"])
+@pytest.mark.parametrize("wdtype", ["bf16", "int4", "nvfp4"])
 def test_no_alloc_entry_matches_the_allocating_path_twice(wdtype):
     first, second = _inputs(21, wdtype), _inputs(22, wdtype)
     for a in (first, second):          # two calls in a row share the static scratch
