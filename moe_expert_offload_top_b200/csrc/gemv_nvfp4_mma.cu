@@ -137,8 +137,8 @@ __global__ void __launch_bounds__(kPrepThreads) nvfp4_prep_h_kernel(const __grid
 }
 
 // ------------------------------------------------------------------ the GEMV --
-// Per CTA: per warp a ring of S stages, the warps' partial sums, and the block scales of its
-// rows.  A stage is 2 NM weight chunks x 32 lanes x 16 bytes (chunk-major), then the input
+// Per CTA: per warp a ring of S stages (the warps' partial sums reuse its bytes once every
+// warp has drained its ring), and the block scales of its rows.  A stage is 2 NM weight chunks x 32 lanes x 16 bytes (chunk-major), then the input
 // bytes of ncols columns, 256 bytes each (128 f16 of the group): lane (g, t)'s piece u
 // (elements 32t + 8u .. +7) at slot (4u + t) ^ (4 (g & 1)), so that the 8 lanes of a
 // quarter-warp read 8 distinct bank groups.  The scales are words [nb][NM][8 g][4 t]: the
@@ -147,9 +147,11 @@ template <int NM, int S, int W>
 struct Fp4Smem {
   __host__ __device__ static constexpr size_t wbytes() { return (size_t)2 * NM * 32 * 16; }
   __host__ __device__ static constexpr size_t stage_bytes(int ncols) { return wbytes() + (size_t)ncols * 256; }
-  __host__ __device__ static constexpr size_t red_off(int ncols) { return (size_t)W * S * stage_bytes(ncols); }
+  __host__ __device__ static constexpr size_t ring_bytes(int ncols) { return (size_t)W * S * stage_bytes(ncols); }
   __host__ __device__ static constexpr size_t red_bytes() { return (size_t)W * NM * 16 * 8 * sizeof(float); }
-  __host__ __device__ static constexpr size_t scale_off(int ncols) { return red_off(ncols) + red_bytes(); }
+  __host__ __device__ static constexpr size_t scale_off(int ncols) {
+    return ring_bytes(ncols) > red_bytes() ? ring_bytes(ncols) : red_bytes();
+  }
   __host__ __device__ static constexpr size_t bytes(int nb, int ncols) {
     return scale_off(ncols) + (size_t)nb * NM * 32 * 4;
   }
@@ -167,7 +169,7 @@ nvfp4_mma_kernel(const unsigned char* __restrict__ xs, int T, int H, int I, int 
   constexpr bool GU = MODE == 0;
   using L = Fp4Smem<NM, S, W>;
   extern __shared__ __align__(16) unsigned char smem[];
-  float (*red)[NM][16][8] = reinterpret_cast<float (*)[NM][16][8]>(smem + L::red_off(ncols));
+  float (*red)[NM][16][8] = reinterpret_cast<float (*)[NM][16][8]>(smem);   // over the ring
   uint32_t* ssc = reinterpret_cast<uint32_t*>(smem + L::scale_off(ncols));
 
   const int e = list.expert[blockIdx.y];
@@ -301,6 +303,7 @@ nvfp4_mma_kernel(const unsigned char* __restrict__ xs, int T, int H, int I, int 
       wst_off = wst_off + sbytes == ring_bytes ? 0 : wst_off + sbytes;
     }
     cp_wait<0>();
+    __syncthreads();   // every warp's ring is drained: the partial sums may overwrite it
     // acc: rows g (0, 1) and g+8 (2, 3), columns 2t and 2t+1
 #pragma unroll
     for (int m = 0; m < NM; ++m) {
