@@ -29,7 +29,8 @@ The one JSON line (rank 0) carries:
     cache from 15% to 30%; "prefill" of the headline shapes (4096 tokens through the 8
     layers with whole-layer double buffering over PCIe, the same with every expert
     resident, a tensor-pipe sweep of one resident layer at 16k/32k/64k tokens, and one
-    layer with NVFP4 weights, every expert resident); "shrink": decode
+    layer with NVFP4 weights, every expert resident, with its decode GEMVs at batch 1 and
+    8 on the tensor cores and on the fp32 pipes); "shrink": decode
     tokens/s before and after shrinking the cache from 58% to 40% of the experts ("this
     tool runs datacenter AI on your PC", the cache shrink demo).
 --impl reference times the CPU oracle alone on the headline workload.
@@ -700,6 +701,7 @@ def nvfp4_prefill(args, dev, peaks, x, bf16_ms_per_layer, gemm_figures):
         torch.cuda.synchronize(dev)
         perf = ft.ft_moe_perf(stack.h)
         ft.ft_moe_set_stage_timing(stack.h, 0)
+        decode = nvfp4_decode_gemv(stack, x, dev, peaks)
     finally:
         stack.close()
     return {"workload": "%s: 1 layer, E=%d, H=%d, I=%d, top-%d %s + shared expert, NVFP4 weights, %d N(0,1) "
@@ -708,7 +710,46 @@ def nvfp4_prefill(args, dev, peaks, x, bf16_ms_per_layer, gemm_figures):
             "vs_bf16_resident_ms_per_layer": 1e3 * dt / bf16_ms_per_layer,
             "grouped_gemm": dict(gemm_figures(perf), kernel="grouped_gemm_kernel<0,1>+<1,1> (NVFP4 tiles expanded "
                                                            "to bf16 in shared memory, tcgen05 kind::f16)"),
-            "stages_ms_per_layer": {k2: v / 1e3 for k2, v in stage_us(perf).items()}, "pool_setup_s": setup_s}
+            "stages_ms_per_layer": {k2: v / 1e3 for k2, v in stage_us(perf).items()}, "pool_setup_s": setup_s,
+            "decode_gemv": decode}
+
+
+def nvfp4_decode_gemv(stack, x, dev, peaks, steps=16):
+    """Decode on the same resident NVFP4 layer (every expert in its slot, so no fills): the
+    expert GEMVs per launch, stage-timed, on the f16 tensor cores and on the fp32 pipes, at
+    batch 1 and 8; the tokens are rows of the prefill prompt."""
+    import torch
+
+    import moe_expert_offload_top_b200 as ft
+    ft.ft_moe_set_mode(stack.h, 0)
+    stream = torch.cuda.current_stream(dev)
+    res = {"peak_gbs": peaks["hbm_gbs"]}
+    for batch in (1, 8):
+        out = torch.empty((1, batch, stack.cfg.H), dtype=torch.bfloat16, device=dev)
+        row = {}
+        for name, on in (("tensor_cores", 1), ("fp32_pipes", 0)):
+            ft.ft_moe_set_int4_tensor_cores(stack.h, on)
+            for s in range(3):
+                stack.forward(0, x[s * batch:(s + 1) * batch], out[0], stream)
+            ft.ft_moe_sync(stack.h)
+            torch.cuda.synchronize(dev)
+            ft.ft_moe_reset_perf(stack.h)
+            ft.ft_moe_set_stage_timing(stack.h, 1)
+            for s in range(3, 3 + steps):
+                stack.forward(0, x[s * batch:(s + 1) * batch], out[0], stream)
+            torch.cuda.synchronize(dev)
+            p = ft.ft_moe_perf(stack.h)
+            ft.ft_moe_set_stage_timing(stack.h, 0)
+            n = max(p["ffn_gate_up_launches"], 1)
+            gu = p["ffn_gate_up_bytes"] / (p["ffn_gate_up_ms"] * 1e-3) / 1e9
+            dn = p["ffn_down_bytes"] / (p["ffn_down_ms"] * 1e-3) / 1e9
+            row[name] = {"gate_up_us": 1e3 * p["ffn_gate_up_ms"] / n, "gate_up_gbs": gu,
+                         "gate_up_frac": gu / peaks["hbm_gbs"], "down_us": 1e3 * p["ffn_down_ms"] / n,
+                         "down_gbs": dn, "down_frac": dn / peaks["hbm_gbs"],
+                         "gate_up_bytes_per_launch": p["ffn_gate_up_bytes"] / n, "launches": n}
+        res["batch_%d" % batch] = row
+    ft.ft_moe_set_int4_tensor_cores(stack.h, 1)
+    return res
 
 
 # -------------------------------------------------------------- shrink leg --
