@@ -181,6 +181,9 @@ def test_permute_parity(T, k, E):
     # token columns per pass (4 ring stages)
     ("int4", 1152, 384, 5, 6, 3, True),
     ("nvfp4", 2048, 768, 1, 16, 8, False), ("nvfp4", 1024, 512, 3, 8, 4, True), ("nvfp4", 256, 96, 12, 4, 2, True),
+    # NVFP4 on the tensor cores: more pairs per expert than one pass of 8 columns (the shared
+    # expert's 19); 9 groups split 2/2/2/3 over the gate/up warps with 5 columns per pass
+    ("nvfp4", 1024, 256, 19, 5, 2, True), ("nvfp4", 1152, 384, 5, 6, 3, True),
 ])
 def test_expert_ffn_and_combine_parity(wd, H, I, T, E, k, shared):
     cfg = synth.MoeConfig("t", 1, E, H, I, k, "sigmoid", wd, shared, E, T, (T,), "iid", "decode")
