@@ -412,10 +412,12 @@ FT_API int ft_probe_host_memory(size_t bytes, int threads, int iters, double* gb
  * the selected logits, normalised over the k selected.
  *   x: [T][H] (x_is_bf16 ? bf16 : f32), router_w: [E][H] f32, logits: [T][E] f32
  *   (written), ids: [T][k] int32, gates: [T][k] f32.
- * Above 64 tokens the logits come from the forward's tiled router: each logit sums an fp32
- * partial per 32 elements of H (increasing H) into its accumulator, in H order.  With
- * H % 32 == 0 and 16-byte aligned x and router_w it streams the K steps through shared
- * memory with cp.async; otherwise a one-step kernel computes the same sums, bit for bit. */
+ * Above 64 tokens the logits come from the forward's tiled router: each logit sums a partial
+ * per 32 elements of H into its accumulator, in H order.  With H % 32 == 0 and 16-byte
+ * aligned x and router_w the K steps stream through shared memory with cp.async: bf16 x on
+ * the tf32 tensor cores (bf16 is exact in tf32; each router weight is split into tf32 hi + lo,
+ * within 2^-21 of it), fp32 x on the fp32 pipes.  Otherwise a one-step kernel on the fp32
+ * pipes computes the fp32-pipe sums, bit for bit. */
 FT_API int ft_router_topk(const void* x, int x_is_bf16, const float* router_w, int T, int H, int E,
                    int top_k, int gating, float* logits, int* ids, float* gates, void* stream);
 

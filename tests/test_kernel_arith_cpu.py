@@ -273,3 +273,58 @@ def test_nvfp4_inputs_as_f16_rows_with_a_power_of_two_scale():
         hf = hs.astype(np.float16).astype(np.float64)
         big = np.abs(hs) >= 2.0 ** -14
         assert np.all(np.abs(hf[big] - hs[big]) <= 2.0 ** -11 * np.abs(hs[big]))
+
+
+# ------------------------------------------------------- many-token router on tf32 MMAs --
+
+def _tf32_rna(v):
+    """fp32 -> tf32 (10 explicit mantissa bits), round to nearest, ties away from zero."""
+    b = np.asarray(v, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x1000) & 0xFFFFE000
+    return b.astype(np.uint32).view(np.float32)
+
+
+def _tf32_trunc(v):
+    """The bits the MMA reads of an fp32 operand: the top 10 explicit mantissa bits."""
+    return (np.asarray(v, dtype=np.float32).view(np.uint32) & np.uint32(0xFFFFE000)).view(np.float32)
+
+
+def test_router_tf32_split_is_within_2_pow_minus_21():
+    # w = hi + lo with hi = tf32(w) and lo = w - hi (exact in fp32); the MMA reads lo's top
+    # 11 significant bits, so hi + trunc(lo) is within 2^-21 |w|; a bf16 x is exact in tf32
+    rng = np.random.default_rng(9)
+    w = np.concatenate([rng.standard_normal(200000) * s for s in (1e-3, 0.02, 3.0)]).astype(np.float32)
+    hi = _tf32_rna(w)
+    lo = (w - hi).astype(np.float32)
+    assert np.array_equal(hi.astype(np.float64) + lo.astype(np.float64), w.astype(np.float64))   # exact split
+    got = hi.astype(np.float64) + _tf32_trunc(lo).astype(np.float64)
+    assert np.all(np.abs(got - w) <= 2.0 ** -21 * np.abs(w.astype(np.float64)))
+    x = _bf16_bits_to_f32(synth.round_bf16(rng.standard_normal(100000).astype(np.float32)))
+    assert np.array_equal(_tf32_trunc(x), x)
+
+
+def test_router_tf32_fragments_give_the_tile_logits():
+    # one warp's 32 tokens x 32 experts over one k8 step, through the kernel's assignment
+    # (a0 = x[g][t], a1 = x[g+8][t], a2 = x[g][t+4], a3 = x[g+8][t+4] of m-tile i; b0 = w[n][t],
+    # b1 = w[n][t+4] with n = 8j + g; d_c -> token 16i + g + 8 (c >> 1), expert 8j + 2t + (c & 1))
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((32, 8))
+    w = rng.standard_normal((32, 8))
+    z = np.full((32, 32), np.nan)
+    for i in range(2):
+        for j in range(4):
+            A = np.zeros((16, 8))
+            B = np.zeros((8, 8))
+            for lane in range(32):
+                g, t = lane >> 2, lane & 3
+                a = (x[16 * i + g, t], x[16 * i + g + 8, t], x[16 * i + g, t + 4], x[16 * i + g + 8, t + 4])
+                A[g, t], A[g + 8, t], A[g, t + 4], A[g + 8, t + 4] = a          # the PTX A layout
+                n = 8 * j + g
+                B[t, g], B[t + 4, g] = w[n, t], w[n, t + 4]                      # the PTX B layout
+            D = A @ B
+            for lane in range(32):
+                g, t = lane >> 2, lane & 3
+                d = (D[g, 2 * t], D[g, 2 * t + 1], D[g + 8, 2 * t], D[g + 8, 2 * t + 1])   # the PTX D layout
+                for c in range(4):
+                    z[16 * i + g + 8 * (c >> 1), 8 * j + 2 * t + (c & 1)] = d[c]
+    assert np.allclose(z, x @ w.T, rtol=1e-12, atol=1e-12)
