@@ -158,8 +158,10 @@ def test_fused_decode_routing_after_wider_call():
 
 
 @pytest.mark.parametrize("T,k,E", [(1, 2, 16), (7, 8, 128), (33, 6, 256), (300, 8, 256), (4096, 6, 256),
-                                   (5, 16, 16), (0, 2, 16)])
+                                   (5, 16, 16), (0, 2, 16), (128, 8, 16), (129, 8, 16), (3000, 5, 7)])
 def test_permute_parity(T, k, E):
+    # up to 1024 pairs: one CTA; more: one CTA per chunk of 1024 (128 x 8 is exactly one chunk,
+    # 129 x 8 leaves 8 pairs in a second one; few experts put many equal keys in every warp)
     rng = np.random.default_rng(T * 31 + k)
     ids = np.array([rng.choice(E, k, replace=False) for _ in range(T)], dtype=np.int32).reshape(T, k)
     if T > 20:
