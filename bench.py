@@ -91,10 +91,10 @@ def headline_config(world):
 TRAFFIC = {
     "gemv_bf16": {"sources": ["moe_expert_offload_top_b200/csrc/decode_gemv.cuh",
                               "moe_expert_offload_top_b200/csrc/expert_decode.cu"],
-                  "sha256": "020bbb275ac5b005d2a7a2240e68085817161ff8dc30355aa0826a419bfde9a0", "ratio": 1.00226,
+                  "sha256": "9cd1211ebda91b779c1d2e915539c28360cdb91dcac741dc28e5b2f8e593c40d", "ratio": 1.00208,
                   "capture": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 8 gate/up launches of "
                              "kernel_driver --workload dsv4flash-decode-bf16 --layers 1 --experts 16 --steps 8 "
-                             "--perf (7 experts per launch, as here), 1.00226 of their algorithmic bytes; scaled "
+                             "--perf (7 experts per launch, as here), 1.00208 of their algorithmic bytes; scaled "
                              "to the average launch here"},
     "gemv_int4": {"sources": ["moe_expert_offload_top_b200/csrc/decode_gemv.cuh",
                               "moe_expert_offload_top_b200/csrc/gemv_ring.cuh",

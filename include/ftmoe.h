@@ -227,14 +227,17 @@ FT_API int ft_moe_set_fused_routing(ft_moe* h, int enabled);
  * the combine.  The per-output arithmetic is the same, so the outputs are bit-identical. */
 FT_API int ft_moe_set_fused_ffn(ft_moe* h, int enabled);
 
-/* Packed-weight decode GEMV (per-pass launch shape): 1 (default) = on the tensor cores,
- * 0 = fp32 multiply-adds on the CUDA cores.  int4: the int8 tensor cores (mma.sync m16n8k32:
- * the nibbles as signed bytes 16 q, the inputs x and h as 16-bit block fixed point in two
- * bytes, exact int32 products per 128-element group, scaled and summed in fp32).  NVFP4 with
- * H and I multiples of 128: the f16 tensor cores (mma.sync m16n8k16: e2m1 code times e4m3
- * block scale formed exactly as f16, the inputs as f16 rows with a per-row power-of-two
- * scale, fp32 accumulators).  Both choices are within the stated bound of the oracle; their
- * outputs differ in the last bits.  ft_expert_ffn_decode always uses the tensor cores. */
+/* Decode GEMV for int4, NVFP4 and bf16 weights (per-pass launch shape): 1 (default) = on the
+ * tensor cores (mma.sync), 0 = fp32 multiply-adds on the CUDA cores.  int4: the int8 tensor
+ * cores (m16n8k32: the nibbles as signed bytes 16 q, the inputs x and h as 16-bit block fixed
+ * point in two bytes, exact int32 products per 128-element group, scaled and summed in fp32).
+ * NVFP4 with H and I multiples of 128: the f16 tensor cores (m16n8k16: e2m1 code times e4m3
+ * block scale formed exactly as f16, the inputs as f16 rows with a per-row power-of-two scale,
+ * fp32 accumulators).  bf16 with H and I multiples of 32 and 2 or more tokens: the bf16 tensor
+ * cores (m16n8k16: the weights as stored, x as stored, h as bf16 hi + lo halves, fp32
+ * accumulators); one token runs on the fp32 pipes, which stream the weights faster there.  Other shapes
+ * and formats use the fp32 pipes.  Both choices are within the stated bound of the oracle;
+ * their outputs differ in the last bits.  ft_expert_ffn_decode always uses the tensor cores. */
 FT_API int ft_moe_set_int4_tensor_cores(ft_moe* h, int enabled);
 
 /* Host-side fault injection for tests of failure handling (no GPU fault is made).
@@ -455,6 +458,9 @@ FT_API int ft_permute(const int* ids, int T, int top_k, int E, int* counts, int*
  *   T * (2H + 16) bytes of y before the down pass writes y, the h rows in place; so after
  *   the call h holds that form, not the fp32 values, and rows of y that no entry owns may
  *   hold those bytes.
+ *   FT_W_BF16 with H and I multiples of 32 and T >= 2 (the bf16 tensor-core GEMV): between the passes
+ *   the entries' h rows are rewritten in place as bf16 hi and lo halves ([I hi][I lo] in the
+ *   row's 4I bytes, 16 significant bits); x is read as it is.
  *   FT_W_NVFP4 with H and I multiples of 128 (the f16 tensor-core GEMV): likewise, with the
  *   tokens and h rows rewritten as f16 with a per-row power-of-two scale (then a float, the
  *   scale's inverse), the tokens in the first T * (2H + 16) bytes of y.  h rounds to 11

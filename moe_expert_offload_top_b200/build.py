@@ -18,7 +18,7 @@ LIB = os.path.join(HERE, "libftmoe.so")
 BUILD = os.path.join(ROOT, "_build")
 SOURCES = ["api.cu", "router.cu", "permute.cu", "expert_decode.cu", "grouped_gemm_sm100.cu", "noalloc.cu",
            "ffn_fused_f32.cu", "ffn_fused_bf16.cu", "ffn_fused_int4.cu", "ffn_fused_nvfp4.cu", "gemv_int4_mma.cu",
-           "gemv_nvfp4_mma.cu"]
+           "gemv_nvfp4_mma.cu", "gemv_bf16_mma.cu"]
 HEADERS = ["common.cuh", "kernels.hpp", "cache.hpp", "sm100_sync.cuh", "decode_gemv.cuh", "ffn_fused.cuh",
            "gemv_ring.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

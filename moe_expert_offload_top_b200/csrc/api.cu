@@ -935,7 +935,7 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
                                         h->d_perm, h->d_h, h->d_y, s, se ? se->ev[SE_G3] : nullptr, h->d_err,
                                         h->int4_tensor != 0, h->d_xs));
       if (se) se->split = 1;
-      h->perf.kernel_launches += 2;
+      h->perf.kernel_launches += ftk::ffn_decode_kernels(h->wdtype, h->int4_tensor != 0, h->H, h->I, T);
     } else {
       if (must_wait) {
         rc = wait_fills();
@@ -952,7 +952,9 @@ int ft_moe_forward(ft_moe* h, int layer, const void* x, int n_tokens, const floa
     FT_CUDA_B(ftk::launch_combine(h->d_y, h->d_gates, h->d_inv, T, h->H, k, h->has_shared != 0,
                                    xbf16, out, s));
     stage_mark(se, SE_C1, s);
-    h->perf.kernel_launches += 3;
+    // one FFN pass (the GEMMs: gate/up, down) and the combine
+    h->perf.kernel_launches +=
+        (use_gemm ? 2 : ftk::ffn_decode_kernels(h->wdtype, h->int4_tensor != 0, h->H, h->I, T)) + 1;
   }
   hold.release();
 #undef FT_CUDA_B

@@ -113,16 +113,47 @@ static cudaError_t launch_pass(int nt, int rpw, int rows, cudaStream_t s, const 
   }
 }
 
+// Which decode GEMV runs: the tensor-core kernels where their shapes allow, else the
+// per-row GEMV on the fp32 pipes.  bf16 uses the tensor cores from 2 tokens on: with one
+// token the per-row GEMV streams the weights faster (at dsv4flash shapes gate/up took 44.8
+// against 50.7 us per launch), with 8 it is 2.6 times slower.
+enum { kPathRows = 0, kPathInt4Mma = 1, kPathNvfp4Mma = 2, kPathBf16Mma = 3 };
+static int decode_path(int wdtype, bool tensor, int H, int I, int T) {
+  if (!tensor) return kPathRows;
+  if (wdtype == WT_INT4) return kPathInt4Mma;
+  if (wdtype == WT_NVFP4 && H % 128 == 0 && I % 128 == 0) return kPathNvfp4Mma;   // whole groups of 128
+  if (wdtype == WT_BF16 && T >= 2 && H % 32 == 0 && I % 32 == 0) return kPathBf16Mma;
+  return kPathRows;
+}
+
+int ffn_decode_kernels(int wdtype, bool int4_tensor, int H, int I, int T) {
+  switch (decode_path(wdtype, int4_tensor, H, I, T)) {
+    case kPathInt4Mma:
+    case kPathNvfp4Mma:
+      return 4;   // token slicing, gate/up, h slicing, down
+    case kPathBf16Mma:
+      return 3;   // gate/up, h split, down
+    default:
+      return 2;   // gate/up, down
+  }
+}
+
 cudaError_t launch_ffn_decode(const void* x, int T, int H, int I, int k, int wdtype,
                               const ExpertList& list, int max_pairs_per_expert, const int* offsets,
                               const int* perm, float* h, float* y, cudaStream_t s,
                               cudaEvent_t between, int* err, bool int4_tensor, void* int4_xs) {
   (void)err;
   if (list.n <= 0 || T <= 0) return cudaSuccess;
-  if (wdtype == WT_INT4 && int4_tensor)
-    return launch_ffn_int4_mma(x, T, H, I, k, list, offsets, perm, h, y, s, between, max_pairs_per_expert, int4_xs);
-  if (wdtype == WT_NVFP4 && int4_tensor && H % 128 == 0 && I % 128 == 0)   // whole groups of 128
-    return launch_ffn_nvfp4_mma(x, T, H, I, k, list, offsets, perm, h, y, s, between, max_pairs_per_expert, int4_xs);
+  switch (decode_path(wdtype, int4_tensor, H, I, T)) {
+    case kPathInt4Mma:
+      return launch_ffn_int4_mma(x, T, H, I, k, list, offsets, perm, h, y, s, between, max_pairs_per_expert, int4_xs);
+    case kPathNvfp4Mma:
+      return launch_ffn_nvfp4_mma(x, T, H, I, k, list, offsets, perm, h, y, s, between, max_pairs_per_expert, int4_xs);
+    case kPathBf16Mma:
+      return launch_ffn_bf16_mma(x, T, H, I, k, list, offsets, perm, h, y, s, between, max_pairs_per_expert);
+    default:
+      break;
+  }
   int nt = max_pairs_per_expert < T ? max_pairs_per_expert : T;
   if (nt < 1) nt = 1;
   auto bytes_of = [&](int K) -> size_t {

@@ -44,8 +44,9 @@ cudaError_t launch_permute(const int* ids, int T, int k, int E, int* counts, int
 // then the down projection into y [pairs][H] fp32.  Pairs are positions in the
 // permutation (routed) or T*k + t (shared expert).  `between` (optional) is recorded
 // on s between the gate/up and the down passes.
-// Packed weights run on the tensor cores unless int4_tensor is false: int4 on the int8
-// ones (launch_ffn_int4_mma), NVFP4 on the f16 ones (launch_ffn_nvfp4_mma).  The h rows of
+// Packed and bf16 weights run on the tensor cores unless int4_tensor is false: int4 on the
+// int8 ones (launch_ffn_int4_mma), NVFP4 on the f16 ones (launch_ffn_nvfp4_mma, H and I
+// multiples of 128), bf16 on the bf16 ones (launch_ffn_bf16_mma, H and I multiples of 32, T >= 2).  The h rows of
 // the list's pairs are then left as sliced inputs (see below), and int4_xs
 // (int4_sliced_x_bytes(T, H) bytes) receives the sliced tokens, or, when null, the front of
 // y does (before the down pass writes y).
@@ -71,6 +72,13 @@ size_t int4_sliced_x_bytes(int T, int H);
 cudaError_t launch_ffn_nvfp4_mma(const void* x, int T, int H, int I, int k, const ExpertList& list, const int* offsets,
                                  const int* perm, float* h, float* y, cudaStream_t s, cudaEvent_t between,
                                  int max_pairs_per_expert, void* xsliced);
+// K3 (decode) for bf16 weights on the bf16 tensor cores (gemv_bf16_mma.cu); x bf16.  After the
+// gate/up pass the h rows of the list's pairs are rewritten in place as bf16 hi and lo halves.
+cudaError_t launch_ffn_bf16_mma(const void* x, int T, int H, int I, int k, const ExpertList& list, const int* offsets,
+                                const int* perm, float* h, float* y, cudaStream_t s, cudaEvent_t between,
+                                int max_pairs_per_expert);
+// Kernels one launch_ffn_decode call launches for these arguments.
+int ffn_decode_kernels(int wdtype, bool int4_tensor, int H, int I, int T);
 // K3 + K5 (decode) in one launch (ffn_fused.cuh): gate/up + SwiGLU into h, down into y
 // and, with `combine`, out[t] = sum_j gates[t][j] * y[inv[t*k+j]] (+ shared) for the
 // entries of `list`.  The combine of a launch covers every pair of the forward, so

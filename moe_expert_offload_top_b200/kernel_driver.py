@@ -2,6 +2,7 @@
 
     python -m moe_expert_offload_top_b200.kernel_driver --workload NAME
         [--layers L] [--experts E] [--slots C] [--steps S] [--batch B] [--tokens T] [--wdtype W] [--perf]
+        [--fp32-pipes]
 
 The workload keeps its shapes (hidden, intermediate, top-k, gating, weight format,
 shared expert) and token process; --layers / --experts shrink the pool so that a
@@ -37,6 +38,8 @@ def main(argv=None):
                     help="another weight format for the workload's shapes")
     ap.add_argument("--perf", action="store_true",
                     help="stage timing on: also print the algorithmic bytes and flops per FFN launch")
+    ap.add_argument("--fp32-pipes", action="store_true",
+                    help="decode GEMV on the fp32 pipes instead of the tensor cores (int4, NVFP4, bf16)")
     a = ap.parse_args(argv)
     base = synth.CONFIGS[a.workload]
     E = a.experts or base.E
@@ -49,6 +52,8 @@ def main(argv=None):
     with GpuStack(cfg, max_tokens=T) as st:
         vals, x = st.tokens(T)
         out = torch.empty((cfg.L, T, cfg.H), dtype=st.xdt, device=st.device)
+        if a.fp32_pipes:
+            ft.ft_moe_set_int4_tensor_cores(st.h, 0)
         if a.perf:
             ft.ft_moe_set_stage_timing(st.h, 1)
         for s in range(a.steps):

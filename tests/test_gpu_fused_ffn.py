@@ -86,7 +86,7 @@ def test_many_tokens_gemv_path_fused():
     cfg = synth.MoeConfig("wide-gemv", L=1, E=16, H=1024, I=512, k=4, gating="softmax", wdtype="bf16",
                           shared=True, C=16, tokens=160, batches=(80,), process="iid", mode="decode")
     a = _run(cfg, fused=True, batch=80, gemm_threshold=1 << 30, oracle=True)
-    b = _run(cfg, fused=False, batch=80, gemm_threshold=1 << 30)
+    b = _run(cfg, fused=False, batch=80, gemm_threshold=1 << 30, int4_tensor=False)   # the same per-row arithmetic
     for oa, ob in zip(a["outs"], b["outs"]):
         assert np.array_equal(oa, ob)
     ref = a["ref"]
@@ -115,18 +115,22 @@ def test_resident_experts_run_before_the_fill_wait():
         assert np.array_equal(oa, ob)
 
 
-def test_per_pass_kernels_split_around_the_fill_wait():
-    # the default launch shape: forwards with both resident and copied experts run two
-    # gate/up + down pairs (five FFN launches with the combine), the others one pair
-    cfg = dataclasses.replace(synth.CONFIGS["decode-locality-bf16"], L=2, tokens=24, C=40)
-    fwd = cfg.L * cfg.tokens
-    a = _run(cfg, fused=False)
+@pytest.mark.parametrize("tensor,batch,per_pass", [(True, 1, 2), (True, 8, 3), (False, 8, 2)])
+def test_per_pass_kernels_split_around_the_fill_wait(tensor, batch, per_pass):
+    # the default launch shape: forwards with both resident and copied experts run two FFN
+    # passes (gate/up + down; on the bf16 tensor cores from 2 tokens on, with the h split
+    # between them), the others one, then the combine
+    cfg = dataclasses.replace(synth.CONFIGS["decode-locality-bf16"], L=2, tokens=24 * batch, C=40 if batch == 1 else 160,
+                              batches=(batch,))
+    fwd = cfg.L * (cfg.tokens // batch)
+    a = _run(cfg, fused=False, batch=batch, int4_tensor=tensor)
     p = a["perf"]
     assert p["forwards"] == fwd and p["ffn_fused_launches"] == 0
-    assert 4 * fwd < p["kernel_launches"] < 6 * fwd      # routing + 3, + 2 where split
-    b = _run(cfg, fused=False, stage_timing=True)
+    one = 1 + per_pass + 1                                # routing, one pass, combine
+    assert one * fwd < p["kernel_launches"] < (one + per_pass) * fwd     # + one pass where split
+    b = _run(cfg, fused=False, batch=batch, stage_timing=True, int4_tensor=tensor)
     q = b["perf"]
-    assert q["kernel_launches"] == 4 * fwd and q["ffn_gate_up_launches"] == fwd
+    assert q["kernel_launches"] == one * fwd and q["ffn_gate_up_launches"] == fwd
     assert q["ffn_gate_up_ms"] > 0 and q["ffn_down_ms"] > 0 and q["combine_ms"] > 0
     for oa, ob in zip(a["outs"], b["outs"]):
         assert np.array_equal(oa, ob)

@@ -328,3 +328,26 @@ def test_router_tf32_fragments_give_the_tile_logits():
                 for c in range(4):
                     z[16 * i + g + 8 * (c >> 1), 8 * j + 2 * t + (c & 1)] = d[c]
     assert np.allclose(z, x @ w.T, rtol=1e-12, atol=1e-12)
+
+
+def test_bf16_mma_fragments_give_the_group_dot_products():
+    # The bf16 decode GEMV: lane (g, t) holds elements 8t .. 8t+7 of rows g and g+8 per group of
+    # 32 (four words of two elements); MMA h takes words 2h (a0 / a1) and 2h+1 (a2 / a3), and B
+    # words 2h, 2h+1 of the lane's 16 input bytes of column g (elements 8t + 4h .. +3).  The
+    # two MMAs must sum to the plain dot products.
+    rng = np.random.default_rng(11)
+    w = rng.standard_normal((16, 32))
+    x = rng.standard_normal((32, 8))
+    D = np.zeros((16, 8))
+    for h in range(2):
+        a_regs, b_regs = [], []
+        for lane in range(32):
+            g, t = lane >> 2, lane & 3
+            def word(row, wi):
+                e0 = 8 * t + 2 * wi
+                return w[row, e0:e0 + 2]
+            a_regs.append((word(g, 2 * h), word(g + 8, 2 * h), word(g, 2 * h + 1), word(g + 8, 2 * h + 1)))
+            k0 = 8 * t + 4 * h
+            b_regs.append((x[k0:k0 + 2, g], x[k0 + 2:k0 + 4, g]))
+        D += _mma_m16n8k16(a_regs, b_regs)
+    assert np.allclose(D, w @ x, rtol=1e-12, atol=1e-12)
