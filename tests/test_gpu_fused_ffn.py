@@ -136,11 +136,12 @@ def test_per_pass_kernels_split_around_the_fill_wait(tensor, batch, per_pass):
         assert np.array_equal(oa, ob)
 
 
-@pytest.mark.parametrize("wdtype,batch", [("int4", 1), ("int4", 8), ("nvfp4", 1), ("nvfp4", 8)])
+@pytest.mark.parametrize("wdtype,batch", [("int4", 1), ("int4", 8), ("nvfp4", 1), ("nvfp4", 8), ("bf16", 8)])
 def test_int4_tensor_core_gemv_against_cuda_cores_and_oracle(wdtype, batch):
-    # the packed-weight decode GEMV on mma.sync (int4: int8 products; NVFP4: f16 products)
-    # and on the fp32 pipes: the same routing and cache trace, outputs that differ only by
-    # summation order (and, for NVFP4, h rounded to f16), both within the oracle's bound
+    # the decode GEMV on mma.sync (int4: int8 products; NVFP4: f16 products; bf16 from 2 tokens:
+    # bf16 products, h as hi + lo) and on the fp32 pipes: the same routing and cache trace,
+    # outputs that differ only by summation order (and the h operand's rounding), both within
+    # the oracle's bound
     cfg = synth.MoeConfig("%s-tc" % wdtype, L=2, E=32, H=1024, I=512, k=8, gating="sigmoid", wdtype=wdtype,
                           shared=True, C=64, tokens=16 * batch, batches=(batch,), process="ar1", mode="decode")
     a = _run(cfg, fused=False, batch=batch, oracle=True, int4_tensor=True)
