@@ -203,7 +203,8 @@ router_logits_tiled_kernel(const XT* __restrict__ x, const float* __restrict__ w
 // lanes of a half-warp read 16 consecutive router rows; rows are padded by 16 bytes so that
 // those 16-byte reads fall on distinct banks.  The two-level sum of router_logits_tiled_kernel
 // (a partial per K step of 32, then the accumulator), bit for bit.  Needs H % 32 == 0 and
-// 16-byte aligned x and w.
+// 16-byte aligned x and w.  The launcher runs it for fp32 x; bf16 x goes to the tf32 kernel
+// below (the template keeps both, so a bf16 instance stays a bit-exact fp32-pipe reference).
 constexpr int PT = 64, PE = 64, PK = 32, PS = 3;
 template <typename XT>
 struct RouterPipe {
