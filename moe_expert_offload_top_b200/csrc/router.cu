@@ -158,7 +158,7 @@ router_logits_tiled_kernel(const XT* __restrict__ x, const float* __restrict__ w
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;   // 16 x 16 threads
   float acc[4][4] = {};
   for (int k0 = 0; k0 < H; k0 += RK) {
-    // 64 x 16 of x and of w: 1024 elements each, 4 per thread
+    // 64 x 32 of x and of w: 2048 elements each, 8 per thread
     for (int i = threadIdx.x; i < RT * RK; i += 256) {
       const int r = i / RK, c = i % RK;
       float xv = 0.f, wv = 0.f;
