@@ -308,9 +308,9 @@ router_logits_pipe_kernel(const XT* __restrict__ x, const float* __restrict__ w,
 // within 2^-21 of |x w| (lo's truncation).  mma.sync.m16n8k8 (tf32 x tf32, exact products,
 // fp32 accumulators) multiplies.  Each K step of 32 sums into a fresh partial (four k8 MMAs,
 // hi then lo each), added to the logit's accumulator step by step: the two-level sum of the
-// SIMT kernels, though not their rounding.  The CTA tile is 64 tokens x 64 experts, 4 warps
-// of 32 x 32 (2 m16 x 4 n8 MMA tiles); the K steps stream through router_logits_pipe_kernel's
-// 3-stage cp.async ring.  Fragments (m16n8k8, tf32), lane (g, t) = (lane / 4, lane % 4):
+// SIMT kernels, though not their rounding.  The CTA tile is 64 tokens x 64 experts, kTfWarps
+// warps of (64 / (kTfWarps / 2)) x 32 (MT m16 x 4 n8 MMA tiles); the K steps stream through
+// router_logits_pipe_kernel's 3-stage cp.async ring.  Fragments (m16n8k8, tf32), lane (g, t) = (lane / 4, lane % 4):
 // a0 = A[g][t], a1 = A[g+8][t], a2 = A[g][t+4], a3 = A[g+8][t+4]; b0 = B[t][g], b1 = B[t+4][g];
 // d0, d1 = D[g][2t], D[g][2t+1], d2, d3 = D[g+8][2t], D[g+8][2t+1]; A = x (tokens x k), B[k][n]
 // = w[n][k].  Needs H % 32 == 0 and 16-byte aligned x and w.
@@ -324,33 +324,38 @@ FT_DEVICE void tf32_split(float w, uint32_t& hi, uint32_t& lo) {
   lo = __float_as_uint(w - __uint_as_float(hi));
 }
 
-__global__ void __launch_bounds__(128)
+#ifndef FT_ROUTER_TF32_WARPS
+#define FT_ROUTER_TF32_WARPS 4
+#endif
+constexpr int kTfWarps = FT_ROUTER_TF32_WARPS;   // 4 or 8
+constexpr int kTfMt = 8 / kTfWarps;              // m16 tiles per warp
+__global__ void __launch_bounds__(32 * kTfWarps)
 router_logits_tf32_kernel(const uint16_t* __restrict__ x, const float* __restrict__ w, int T, int H, int E,
                           float* __restrict__ z) {
   using P = RouterPipe<uint16_t>;
   extern __shared__ __align__(16) unsigned char rsm[];
   const int t0 = blockIdx.x * PT, e0 = blockIdx.y * PE;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;   // the warp's tokens and experts in the tile
+  const int wm = (warp >> 1) * 16 * kTfMt, wn = (warp & 1) * 32;   // the warp's tokens and experts in the tile
   const int nk = H / PK;
   const uint32_t base = (uint32_t)__cvta_generic_to_shared(rsm);
   constexpr int XP = PK * 2 / 16, WP = PK * 4 / 16;   // 16-byte pieces of an x row, a router row
   auto issue = [&](int ks, int st) {
     const uint32_t sx = base + st * P::kStage, sw = sx + PT * P::kXRow;
-    for (int i = threadIdx.x; i < PT * XP; i += 128) {
+    for (int i = threadIdx.x; i < PT * XP; i += 32 * kTfWarps) {
       const int r = i / XP, c = i % XP;
       const uint16_t* src = x + (size_t)min(t0 + r, T - 1) * H + (size_t)ks * PK + c * 8;
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sx + r * P::kXRow + c * 16), "l"(src) : "memory");
     }
-    for (int i = threadIdx.x; i < PE * WP; i += 128) {
+    for (int i = threadIdx.x; i < PE * WP; i += 32 * kTfWarps) {
       const int r = i / WP, c = i % WP;
       const float* src = w + (size_t)min(e0 + r, E - 1) * H + (size_t)ks * PK + c * 4;
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sw + r * P::kWRow + c * 16), "l"(src) : "memory");
     }
   };
-  float acc[2][4][4];
+  float acc[kTfMt][4][4];
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < kTfMt; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
   for (int s = 0; s < PS - 1; ++s) {
@@ -364,16 +369,16 @@ router_logits_tf32_kernel(const uint16_t* __restrict__ x, const float* __restric
     asm volatile("cp.async.commit_group;" ::: "memory");
     const unsigned char* sx = rsm + (ks % PS) * P::kStage;
     const unsigned char* sw = sx + PT * P::kXRow;
-    float part[2][4][4];
+    float part[kTfMt][4][4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < kTfMt; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) part[i][j][0] = part[i][j][1] = part[i][j][2] = part[i][j][3] = 0.f;
 #pragma unroll
     for (int k0 = 0; k0 < PK; k0 += 8) {
-      uint32_t a[2][4];
+      uint32_t a[kTfMt][4];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < kTfMt; ++i) {
         const unsigned short* r0 = reinterpret_cast<const unsigned short*>(sx + (wm + 16 * i + g) * P::kXRow) + k0 + t;
         const unsigned short* r1 = reinterpret_cast<const unsigned short*>(sx + (wm + 16 * i + g + 8) * P::kXRow) + k0 + t;
         a[i][0] = (uint32_t)r0[0] << 16;
@@ -388,14 +393,14 @@ router_logits_tf32_kernel(const uint16_t* __restrict__ x, const float* __restric
         tf32_split(wr[0], h0, l0);
         tf32_split(wr[4], h1, l1);
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kTfMt; ++i) {
           mma_tf32(part[i][j], a[i], h0, h1);
           mma_tf32(part[i][j], a[i], l0, l1);
         }
       }
     }
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < kTfMt; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -403,7 +408,7 @@ router_logits_tf32_kernel(const uint16_t* __restrict__ x, const float* __restric
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < kTfMt; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -633,7 +638,8 @@ cudaError_t launch_router_logits_tiled(const void* x, bool x_bf16, const float* 
       auto kern = router_logits_tf32_kernel;
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RouterPipe<uint16_t>::kBytes);
       if (e != cudaSuccess) return e;
-      kern<<<pgrid, 128, RouterPipe<uint16_t>::kBytes, s>>>(static_cast<const uint16_t*>(x), w_router, T, H, E, logits);
+      kern<<<pgrid, 32 * kTfWarps, RouterPipe<uint16_t>::kBytes, s>>>(static_cast<const uint16_t*>(x), w_router, T, H, E,
+                                                                       logits);
     } else {
       auto kern = router_logits_pipe_kernel<float>;
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RouterPipe<float>::kBytes);
