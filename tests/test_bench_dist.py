@@ -95,3 +95,26 @@ def test_reference_arm_json_line():
     out1 = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
                            "--warmup", "3"], cwd=ROOT, env=env1, capture_output=True, text=True, timeout=120)
     assert out1.returncode == 0 and out1.stdout.strip() == ""
+
+
+def test_traffic_ratio_only_while_the_sources_hash_the_same(tmp_path):
+    # the bench reports an ncu traffic figure for a kernel only while its sources hash to the
+    # value recorded with the capture; any edit turns it into null with the current hash
+    import hashlib
+    sys.path.insert(0, ROOT)
+    import bench
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1\n")
+    rel = os.path.relpath(str(src), ROOT)
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()
+    bench.TRAFFIC["_probe"] = {"sources": [rel], "sha256": sha, "ratio": 1.25, "capture": "probe capture"}
+    try:
+        assert bench.kernel_traffic("_probe", 100.0) == (125.0, "probe capture")
+        src.write_text("kernel v2\n")
+        traffic, why = bench.kernel_traffic("_probe", 100.0)
+        assert traffic is None and hashlib.sha256(src.read_bytes()).hexdigest()[:12] in why
+    finally:
+        del bench.TRAFFIC["_probe"]
+    for key in bench.TRAFFIC:      # every recorded figure names its capture and its sources exist
+        t = bench.TRAFFIC[key]
+        assert t["capture"] and all(os.path.exists(os.path.join(ROOT, r)) for r in t["sources"])
