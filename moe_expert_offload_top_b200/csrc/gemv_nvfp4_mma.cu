@@ -30,7 +30,7 @@
 // g+8 of each tile, and (lanes of a token column) the column's 64 bytes, into its own slots
 // of a cp.async ring, S - 1 groups ahead; stages hold input bytes for the launch's columns
 // only; the CTA's block scales are staged in shared memory once; the W warps of a CTA split
-// the reduction axis (W = 4 for gate/up, 1 for down) and add their sums in warp order; both
+// the reduction axis (W = 4 for gate/up, 2 for down) and add their sums in warp order; both
 // passes are programmatic dependents of the slicing kernel before them.
 #include "decode_gemv.cuh"
 #include "gemv_ring.cuh"
@@ -46,7 +46,7 @@ using namespace ring;
 #define FT_NVFP4_GU_WARPS 4
 #endif
 #ifndef FT_NVFP4_DOWN_WARPS
-#define FT_NVFP4_DOWN_WARPS 1
+#define FT_NVFP4_DOWN_WARPS 2
 #endif
 constexpr int kWarpsPerSm = 16;   // resident warps per SM: caps the registers
 constexpr int kDownTiles = 2;     // 16-row tiles of a down CTA
